@@ -1,0 +1,430 @@
+"""Benchmark: batched row-wise TopK on B200, effective HBM GB/s (and rows/s).
+
+One step = one ``dsel_topk`` call over one batch of the selected workload (default:
+the bfloat16 Lightning-Indexer batch, 64 rows x 131,072 positions, k = 512,
+unsorted, indices only, int32).  Steps rotate over input copies whose total size is
+more than four times the L2 cache, so every step reads its input from HBM.  The
+timed region is CUDA-graph replays of those steps, bracketed by a barrier and a
+device synchronise, timed with CUDA events on the launching stream; the max over
+ranks is reported.  Under torchrun every rank processes its own batch (weak
+scaling, no collective on the data path).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                       [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "effective HBM GB/s and rows/s for TopK (bf16 k=512; fp32 V=129,280) on 1 B200"
+KERNEL_SOURCES = ["row_wise_topk_b200/csrc/dsel_device.cuh", "row_wise_topk_b200/csrc/dsel_kernels.cuh",
+                  "row_wise_topk_b200/csrc/dsel_api.cu", "row_wise_topk_b200/csrc/dsel_plan.cpp",
+                  "row_wise_topk_b200/csrc/dsel_plan.h"]
+FALLBACK_HBM_GBS = 6650.0
+
+
+def make_workload(name: str) -> W.Workload:
+    if name == "indexer":
+        return W.indexer_drift()
+    if name == "indexer_varlen":
+        return W.indexer_varlen()
+    if name.startswith("sampler"):        # sampler_B_k, e.g. sampler_256_4096
+        _, b, k = name.split("_")
+        return W.sampler_logits(int(b), int(k))
+    if name.startswith("long"):           # long_1_1000 (1 x 2^28) or long_16_4096 (16 x 2^24)
+        _, r, k = name.split("_")
+        r = int(r)
+        return W.long_rows(r, (1 << 28) if r == 1 else (1 << 24), int(k), "uniform")
+    if name == "pr1":
+        return W.pr1_duplicates()
+    raise SystemExit(f"unknown workload {name}")
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(workload: str):
+    """Per-launch DRAM bytes of the streaming kernel from a committed ncu summary, if
+    it was taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    e = d.get(workload)
+    if not e or e.get("kernel_hash") != kernel_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sel = [l for t, l in self.lines if self.t0 is None or (self.t0 - 0.06 <= t <= self.t1 + 0.06)]
+        if not sel:
+            sel = [l for _, l in self.lines[-3:]]
+        mhz, max_mhz, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in sel:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                max_mhz = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max_mhz, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+def physical_gpu_index(local: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+    if local < len(vis) and vis[local].strip().isdigit():
+        return int(vis[local])
+    return local
+
+
+# --------------------------------------------------------------------------- #
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl" if args.impl == "ours" else "gloo",
+                                timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return world, rank, local, pg
+
+
+def max_over_ranks(value: float, pg, device=None) -> float:
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_throughput(w: W.Workload, budget_s: float):
+    """Times the CPU oracle (as it stands) on whole rows of the workload until the
+    budget is spent; returns (GB/s effective, rows/s, rows timed)."""
+    import oracle.topk_oracle as O
+    lens = w.valid_lengths()
+    idx_b = 4 if w.index_dtype == "i32" else 8
+    val_b = w.elem_bytes if w.return_value else 0
+    done_rows, done_bytes, t_used = 0, 0, 0.0
+    r = 0
+    while t_used < budget_s and done_rows < 100000:
+        sub = slice(r % w.rows, r % w.rows + 1)
+        end = None if w.end is None else w.end[sub]
+        t0 = time.perf_counter()
+        O.oracle_topk(w.x[sub], w.dtype, w.k, end=end, sorted_index=w.sorted_index,
+                      return_value=w.return_value, index_dtype=w.index_dtype, nan_mode=w.nan_mode)
+        t_used += time.perf_counter() - t0
+        done_rows += 1
+        done_bytes += int(lens[r % w.rows]) * w.elem_bytes + w.k * (idx_b + val_b) + (4 if w.end is not None else 0)
+        r += 1
+    return done_bytes / t_used / 1e9, done_rows / t_used, done_rows, t_used
+
+
+def run_reference(args, w, world, rank):
+    """Reference arm: the CPU oracle timed on the host cores, one bounded sample of
+    the workload per step (rank 0 only)."""
+    if rank != 0:
+        return
+    per_step_budget = max(0.5, 60.0 / max(args.steps + args.warmup, 1))
+    for _ in range(args.warmup):
+        cpu_oracle_throughput(w, per_step_budget / 4)
+    vals, rows_s, nrows, secs = [], [], 0, 0.0
+    for _ in range(args.steps):
+        gbs, rps, n, t = cpu_oracle_throughput(w, per_step_budget)
+        vals.append(gbs)
+        rows_s.append(rps)
+        nrows += n
+        secs += t
+    value = statistics.median(vals)
+    sample = f"{nrows} whole rows of {w.name} over {args.steps} steps ({secs:.1f} s of CPU time)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "rows_per_s": round(statistics.median(rows_s), 2), "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1000.0 * secs / max(args.steps, 1), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic", "config": workload_config(args, w, world),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(args, w, world):
+    return {"workload": w.name, "rows": w.rows, "row_stride": w.row_stride, "k": w.k,
+            "dtype": w.dtype, "sorted_index": w.sorted_index, "return_value": w.return_value,
+            "index_dtype": w.index_dtype, "end": w.end is not None,
+            "global_batch": w.rows * world, "parallelism": f"dp{world} (rows per rank, no collective)",
+            "l2": "inputs rotate over copies totalling > 4x L2, so every step reads HBM"}
+
+
+def run_ours(args, w, world, rank, local, pg):
+    import torch
+    import row_wise_topk_b200 as T
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=dev)
+    eb = w.elem_bytes
+    in_bytes = w.rows * w.row_stride * eb
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    n_copies = int(max(2, min(64, -(-4 * l2 // in_bytes) + 1)))
+    signed = w.x.view(np.int16) if eb == 2 else w.x.view(np.int32)
+    host = torch.from_numpy(np.ascontiguousarray(signed)).pin_memory()
+    copies = [torch.empty_like(host, device=dev) for _ in range(n_copies)]
+    for c in copies:
+        c.copy_(host, non_blocking=True)
+    end_dev = None if w.end is None else torch.from_numpy(w.end).to(dev)
+    itorch = torch.int32 if w.index_dtype == "i32" else torch.int64
+    idx_out = torch.empty((w.rows, w.k), dtype=itorch, device=dev)
+    val_out = torch.empty((w.rows, w.k), dtype=copies[0].dtype, device=dev) if w.return_value else None
+    dt = T.DSEL_BF16 if w.dtype == "bf16" else T.DSEL_F32
+    idt = T.DSEL_I32 if w.index_dtype == "i32" else T.DSEL_I64
+    nm = T.DSEL_NAN_FLAG if w.nan_mode == "flag" else T.DSEL_NAN_TRAP
+    sptr = stream.cuda_stream
+
+    def step(i):
+        st = T.dsel_topk(copies[i % n_copies].data_ptr(), dt, w.rows, w.row_stride,
+                         None if end_dev is None else end_dev.data_ptr(), w.k, w.sorted_index,
+                         w.return_value, idt, nm, None if val_out is None else val_out.data_ptr(),
+                         idx_out.data_ptr(), sptr)
+        if st != 0:
+            raise T.DselError(st)
+
+    torch.cuda.synchronize(dev)
+    # one eager call first (sets kernel attributes, allocates any workspace)
+    with torch.cuda.stream(stream):
+        step(0)
+    torch.cuda.synchronize(dev)
+
+    # graph of S steps (S = number of input copies, so each replay touches every copy once)
+    S = n_copies
+    graph = torch.cuda.CUDAGraph()
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(S)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(S)]
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(S):
+            ev_a[i].record()
+            step(i)
+            ev_b[i].record()
+    rem = args.steps % S
+    graph_rem = None
+    if rem:
+        graph_rem = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_rem, stream=stream):
+            for i in range(rem):
+                step(i)
+    full = args.steps // S
+
+    plan = T.dsel_plan(dt, w.rows, w.row_stride, w.k,
+                       num_sms=torch.cuda.get_device_properties(dev).multi_processor_count)[1]
+    launches_per_step = 1 + (1 if plan["groups"] > 1 else 0)
+
+    # warm-up
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, -(-args.warmup // S))):
+            graph.replay()
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(physical_gpu_index(local))
+    sampler.start()
+    time.sleep(0.3)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler.mark("t0")
+    with torch.cuda.stream(stream):
+        t_start.record()
+        for _ in range(full):
+            graph.replay()
+        if graph_rem is not None:
+            graph_rem.replay()
+        t_end.record()
+    torch.cuda.synchronize(dev)
+    sampler.mark("t1")
+    if pg is not None:
+        pg.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    # per-step device times from the last full replay (events inside the graph)
+    per_step_ms = [ev_a[i].elapsed_time(ev_b[i]) for i in range(S)] if full else [elapsed_ms / args.steps]
+    time.sleep(0.2)
+    clocks = sampler.stop()
+
+    elapsed_ms = max_over_ranks(elapsed_ms, pg, dev)
+    ms_per_step = elapsed_ms / args.steps
+    eff = w.effective_bytes()
+    value = world * eff * args.steps / (elapsed_ms / 1e3) / 1e9
+    rows_per_s = world * w.rows * args.steps / (elapsed_ms / 1e3)
+
+    # roofline of the streaming kernel: algorithmic bytes per launch / launch time
+    kern_ms = statistics.mean(per_step_ms)
+    peak, peak_kind = hbm_peak()
+    achieved = eff / (kern_ms / 1e3) / 1e9
+    traffic = recorded_traffic(args.workload)
+
+    # end to end through the public API: pinned H2D of the batch, the call, D2H of
+    # the indices (and values), every step
+    e2e_steps = max(3, min(args.steps, 50))
+    host_idx = torch.empty_like(idx_out, device="cpu").pin_memory()
+    host_val = None if val_out is None else torch.empty_like(val_out, device="cpu").pin_memory()
+    x_e2e = copies[0]
+    xv = x_e2e.view(torch.bfloat16 if eb == 2 else torch.float32)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record()
+        for i in range(e2e_steps):
+            x_e2e.copy_(host, non_blocking=True)
+            T.topk(xv, w.k, end=end_dev, sorted_index=w.sorted_index,
+                   return_value=bool(w.return_value), index_dtype=itorch, nan_mode=w.nan_mode,
+                   out=(val_out, idx_out), stream=sptr)
+            host_idx.copy_(idx_out, non_blocking=True)
+            if host_val is not None:
+                host_val.copy_(val_out, non_blocking=True)
+        e1.record()
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg, dev) / e2e_steps
+    h2d = in_bytes
+    d2h = idx_out.numel() * idx_out.element_size() + (0 if val_out is None else val_out.numel() * val_out.element_size())
+    e2e_value = world * eff / (e2e_ms / 1e3) / 1e9
+
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        gbs, rps, nrows, secs = cpu_oracle_throughput(w, args.cpu_seconds)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{nrows} whole rows of {w.name} ({secs:.1f} s, single thread numpy)",
+               "rows_per_s": round(rps, 2)}
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "rows_per_s": round(rows_per_s, 1),
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic", "config": workload_config(args, w, world),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
+                     "kernel": "topk_stream_kernel" + ("+topk_merge_kernel" if launches_per_step > 1 else ""),
+                     "launch_ms": round(kern_ms, 5)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "plan": {k_: plan[k_] for k_ in ("cluster", "groups", "stages", "smem_bytes")},
+        "input_copies": n_copies,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="indexer")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local, pg = dist_setup(args)
+    w = make_workload(args.workload)
+    try:
+        if args.impl == "reference":
+            run_reference(args, w, world, rank)
+        else:
+            run_ours(args, w, world, rank, local, pg)
+    finally:
+        if pg is not None:
+            pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,172 @@
+/*
+ * dsel.h -- C ABI of the B200 (sm_100a) batched row-wise TopK library.
+ *
+ * The operation (what every entry point computes)
+ * -----------------------------------------------
+ * For each row r of a batch, select the k largest entries (k <= 4096) and return
+ * their indices, and optionally their values.  This is the selection kernel of
+ * DeepSeek Sparse Attention's Lightning Indexer (bfloat16 scores, tuned for
+ * k = 512) and of the sampler (float32 logits, vocabulary ~129,280):
+ *   - "Inside DeepSeek V4.1's New Open Inference Toolkit", section "DeepSelect: a
+ *     fast, deliberately narrow TopK" (dtypes, k <= 4096, row alignment, options,
+ *     NaN policy);
+ *   - "DeepSeek releases DeepSelect, a TopK kernel for sparse attention and
+ *     sampling" (narracomm): the method paragraph (threshold T, contiguous blocks
+ *     of size B in random order, candidate buffer, radix select back to k when the
+ *     buffer reaches k + B2), the coverage paragraph (bf16 / f32, int32 / int64
+ *     indices), the paragraph on install and switches (stride requirement,
+ *     sorted_index, return_value) and the NaN paragraph;
+ *   - "DeepSeek 在 GitHub 发布 DeepSelect v1.0.0" (aifluxnews), section "PyTorch 接口与
+ *     CUDA 环境要求" (per-row `end`, output stride constraints, NaN trap).
+ *
+ * Result definition: the k entries of row r that come first in the total order
+ * "value descending, then index ascending", where -0.0 equals +0.0 and both
+ * infinities are ordinary values.  The result is therefore unique and the library
+ * is deterministic (the pages promise stable results: "DeepSeek开源DeepSelect：
+ * 比torch.topk快二十倍！", section "DeepSelect 的差异化设计").
+ *
+ * Layout and ownership (all entry points)
+ * ---------------------------------------
+ *   x            device pointer, rows x row_stride elements, row-major, rows
+ *                contiguous in the last dimension; 16-byte aligned.
+ *   row_stride   elements between row starts; a multiple of
+ *                dsel_stride_requirement(dtype) (the caller pads).
+ *   end          device pointer to int32[rows] or NULL.  Row r's valid range is
+ *                [0, end[r]); NULL means every row is row_stride long.  Entries at
+ *                or past end[r] are never read as candidates.
+ *   indices_out  device pointer, rows x k, contiguous (row stride k), int32 or
+ *                int64 per index_dtype; indices are relative to the row start.
+ *   values_out   device pointer, rows x k, contiguous, same dtype as x, holding the
+ *                selected elements' original bits; NULL iff return_value == 0.
+ *   stream       a cudaStream_t passed as void* (NULL = legacy default stream).
+ * The caller owns all memory.  Calls are asynchronous on `stream` and never
+ * synchronise the host.  Plans that split one row over several thread-block
+ * clusters use a per-(device, stream) workspace that the library allocates once
+ * (cudaMalloc, outside any stream capture) and reuses; all other plans allocate
+ * nothing.
+ *
+ * Special rows and sentinel values
+ *   - end[r] <= k ("short row"): all end[r] entries are returned in index order
+ *     and the NaN check is skipped (narracomm NaN paragraph); slots end[r]..k-1
+ *     hold index DSEL_IDX_PAD and value -inf.
+ *   - a NaN in a row with end[r] > k: DSEL_NAN_TRAP (default, the pages'
+ *     abort_when_nan_found=True) executes the PTX `trap` instruction, which
+ *     aborts the CUDA context; DSEL_NAN_FLAG instead writes DSEL_IDX_NAN in every
+ *     index slot of that row and a quiet NaN in every value slot.
+ *   - end[r] < 0 or end[r] > row_stride: DSEL_NAN_FLAG writes DSEL_IDX_BAD_END
+ *     (values quiet NaN); DSEL_NAN_TRAP clamps end[r] to [0, row_stride].
+ *
+ * Errors: every argument check runs on the host before any launch; a failed
+ * check returns a negative DSEL_ERR_* code and launches nothing.
+ */
+#ifndef DSEL_H_
+#define DSEL_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSEL_API __attribute__((visibility("default")))
+
+/* dtype */
+#define DSEL_BF16 0
+#define DSEL_F32 1
+/* index_dtype */
+#define DSEL_I32 0
+#define DSEL_I64 1
+/* nan_mode */
+#define DSEL_NAN_TRAP 0
+#define DSEL_NAN_FLAG 1
+/* sorted_index: 0 = unspecified order, 1 = ascending index,
+ * 2 = value descending (ties by ascending index), float32 only (narracomm: sorting
+ * by value is limited to the float32 CUDA path). */
+#define DSEL_ORDER_NONE 0
+#define DSEL_ORDER_INDEX 1
+#define DSEL_ORDER_VALUE 2
+
+/* sentinel indices */
+#define DSEL_IDX_PAD (-1)
+#define DSEL_IDX_NAN (-2)
+#define DSEL_IDX_BAD_END (-3)
+
+/* status codes */
+#define DSEL_OK 0
+#define DSEL_ERR_DTYPE (-1)        /* dtype not DSEL_BF16 / DSEL_F32 */
+#define DSEL_ERR_INDEX_DTYPE (-2)  /* index_dtype not DSEL_I32 / DSEL_I64 */
+#define DSEL_ERR_K (-3)            /* k < 1 or k > 4096 */
+#define DSEL_ERR_ROWS (-4)         /* rows < 0 */
+#define DSEL_ERR_STRIDE (-5)       /* row_stride < 1, > INT32_MAX, or not a multiple of the requirement */
+#define DSEL_ERR_ALIGN (-6)        /* x not 16-byte aligned */
+#define DSEL_ERR_NULL (-7)         /* x or indices_out is NULL (with rows > 0) */
+#define DSEL_ERR_VALUES (-8)       /* return_value set with values_out NULL, or the reverse */
+#define DSEL_ERR_NAN_MODE (-9)     /* nan_mode not DSEL_NAN_TRAP / DSEL_NAN_FLAG */
+#define DSEL_ERR_ORDER (-10)       /* sorted_index out of range, or value order on bf16 */
+#define DSEL_ERR_DEVICE (-11)      /* current device is not sm_100 */
+#define DSEL_ERR_WORKSPACE (-12)   /* the split-row workspace could not be allocated */
+#define DSEL_ERR_CUDA (-13)        /* a CUDA runtime call failed (launch error forwarded) */
+#define DSEL_ERR_DEVICE_TIMEOUT (-14) /* a kernel gave up a bounded wait (see dsel_device_status) */
+
+/* Launch plan chosen for a call (see dsel_plan). */
+typedef struct {
+  int32_t threads;       /* threads per CTA */
+  int32_t cluster;       /* CTAs per thread-block cluster working on one row */
+  int32_t groups;        /* clusters per row (> 1: split-row plan with a merge launch) */
+  int32_t block;         /* B: elements per contiguous block visited in random order */
+  int32_t b2;            /* B2: the buffer is cut back to k when it holds k + B2 */
+  int32_t round;         /* elements the CTA filters between two buffer checks */
+  int32_t capacity;      /* candidate-buffer slots per CTA (k + B2 + round) */
+  int32_t stages;        /* blocks kept in flight per CTA (shared-memory ring) */
+  int32_t idx_bits;      /* bits of the in-row index used to break ties */
+  int32_t smem_bytes;    /* dynamic shared memory per CTA */
+  int64_t workspace_bytes; /* split-row workspace (0 unless groups > 1) */
+} dsel_plan_t;
+
+/*
+ * dsel_topk -- batched row-wise TopK (the operation described at the top).
+ *   dtype        DSEL_BF16 or DSEL_F32
+ *   rows         number of rows (0 is a no-op)
+ *   row_stride   see above
+ *   end          see above (device, may be NULL)
+ *   k            1..4096
+ *   sorted_index DSEL_ORDER_NONE / DSEL_ORDER_INDEX / DSEL_ORDER_VALUE
+ *   return_value 0 or 1
+ *   index_dtype  DSEL_I32 or DSEL_I64
+ *   nan_mode     DSEL_NAN_TRAP (default behaviour of the pages) or DSEL_NAN_FLAG
+ * Returns DSEL_OK or a DSEL_ERR_* code.
+ */
+DSEL_API int dsel_topk(const void* x, int dtype, int64_t rows, int64_t row_stride,
+                       const int32_t* end, int32_t k, int sorted_index, int return_value,
+                       int index_dtype, int nan_mode, void* values_out, void* indices_out,
+                       void* stream);
+
+/* Row-stride requirement in elements for `dtype` (the pages' get_stride_requirement,
+ * narracomm paragraph on install and switches): 16 for both dtypes, so every row
+ * start is 32-byte (bf16) or 64-byte (f32) aligned.  Returns -1 for a bad dtype. */
+DSEL_API int64_t dsel_stride_requirement(int dtype);
+
+/* Human-readable text for a status code (static storage, never NULL). */
+DSEL_API const char* dsel_status_string(int status);
+
+/* Host-only planner: the plan dsel_topk would use for these arguments on a device
+ * with `num_sms` SMs, `smem_optin` bytes of opt-in shared memory per CTA and
+ * clusters of up to `max_cluster` CTAs.  Makes no CUDA call.  Returns DSEL_OK or
+ * a DSEL_ERR_* code for invalid arguments. */
+DSEL_API int dsel_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k,
+                       int32_t num_sms, int32_t smem_optin, int32_t max_cluster,
+                       dsel_plan_t* out);
+
+/* Reads and clears the device-side status word that kernels set when a bounded
+ * wait runs out (it should never happen).  Synchronises `stream`.  *status_out
+ * receives 0 or DSEL_ERR_DEVICE_TIMEOUT.  Returns DSEL_OK or DSEL_ERR_CUDA. */
+DSEL_API int dsel_device_status(int* status_out, void* stream);
+
+/* Library version string. */
+DSEL_API const char* dsel_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSEL_H_ */

@@ -1,0 +1,271 @@
+// C ABI of the row-wise TopK library: argument checks, planning, launches.
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <vector>
+
+#include "../../include/dsel.h"
+#include "dsel_kernels.cuh"
+#include "dsel_plan.h"
+
+namespace dsel {
+namespace {
+
+static_assert(sizeof(Ctl) <= kSharedFixedBytes, "control block outgrew its reservation");
+
+struct DevInfo {
+  bool ready = false;
+  int sms = 0;
+  int smem_optin = 0;
+  int major = 0;
+  bool attrs_set[2] = {false, false};
+};
+
+std::mutex g_mu;
+DevInfo g_dev[64];
+
+struct Workspace {
+  int dev;
+  void* stream;
+  void* ptr;
+  size_t bytes;
+};
+std::vector<Workspace> g_ws;
+
+int device_info(int dev, DevInfo** out) {
+  if (dev < 0 || dev >= 64) return DSEL_ERR_DEVICE;
+  DevInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int minor = 0;
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return DSEL_ERR_CUDA;
+    if (d.major != 10 || minor != 0) return DSEL_ERR_DEVICE;
+    d.ready = true;
+  }
+  *out = &d;
+  return DSEL_OK;
+}
+
+// One workspace per (device, stream), grown on demand.  Growing frees the old
+// buffer after synchronising the stream that used it.
+int workspace(int dev, void* stream, size_t bytes, void** out) {
+  for (auto& w : g_ws) {
+    if (w.dev == dev && w.stream == stream) {
+      if (w.bytes >= bytes) {
+        *out = w.ptr;
+        return DSEL_OK;
+      }
+      if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSEL_ERR_CUDA;
+      cudaFree(w.ptr);
+      w.ptr = nullptr;
+      w.bytes = 0;
+      if (cudaMalloc(&w.ptr, bytes) != cudaSuccess) return DSEL_ERR_WORKSPACE;
+      w.bytes = bytes;
+      *out = w.ptr;
+      return DSEL_OK;
+    }
+  }
+  void* p = nullptr;
+  if (cudaMalloc(&p, bytes) != cudaSuccess) return DSEL_ERR_WORKSPACE;
+  g_ws.push_back({dev, stream, p, bytes});
+  *out = p;
+  return DSEL_OK;
+}
+
+struct Layout {
+  uint32_t bars, blk, cb, ci, ctl, total;
+};
+
+uint32_t align_up(uint64_t v, uint64_t a) { return static_cast<uint32_t>((v + a - 1) / a * a); }
+
+Layout stream_layout(const dsel_plan_t& pl, int eb) {
+  Layout l{};
+  uint64_t off = align_up(uint64_t(pl.stages) * pl.block * eb, 128);
+  l.bars = uint32_t(off);
+  off += align_up(uint64_t(pl.stages) * 8, 16);
+  l.blk = uint32_t(off);
+  off += align_up(uint64_t(pl.stages) * 4, 16);
+  l.cb = uint32_t(off);
+  off += align_up(uint64_t(pl.capacity) * eb, 16);
+  l.ci = uint32_t(off);
+  off += align_up(uint64_t(pl.capacity) * 4, 16);
+  l.ctl = uint32_t(off);
+  off += align_up(sizeof(Ctl), 16);
+  l.total = uint32_t(off);
+  return l;
+}
+
+Layout merge_layout(const dsel_plan_t& pl, int eb) {
+  Layout l{};
+  uint64_t off = 0;
+  l.cb = 0;
+  off += align_up(uint64_t(pl.capacity) * eb, 16);
+  l.ci = uint32_t(off);
+  off += align_up(uint64_t(pl.capacity) * 4, 16);
+  l.ctl = uint32_t(off);
+  off += align_up(sizeof(Ctl), 16);
+  l.total = uint32_t(off);
+  return l;
+}
+
+template <typename Kern>
+cudaError_t launch_cluster(Kern kern, unsigned grid, int cluster, uint32_t smem, cudaStream_t st,
+                           const KParams& kp) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, kp);
+}
+
+template <int DT>
+int run(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
+  auto sk = topk_stream_kernel<DT, kThreads>;
+  auto mk = topk_merge_kernel<DT, kThreads>;
+  if (!di->attrs_set[DT]) {
+    if (cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) != cudaSuccess ||
+        cudaFuncSetAttribute(sk, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
+        cudaFuncSetAttribute(mk, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) != cudaSuccess ||
+        cudaFuncSetAttribute(mk, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+      return DSEL_ERR_CUDA;
+    di->attrs_set[DT] = true;
+  }
+  const int eb = elem_bytes(DT);
+  const Layout sl = stream_layout(pl, eb);
+  KParams kp = base;
+  kp.off_bars = sl.bars;
+  kp.off_blk = sl.blk;
+  kp.off_cb = sl.cb;
+  kp.off_ci = sl.ci;
+  kp.off_ctl = sl.ctl;
+  const int64_t grid = rows * pl.groups * pl.cluster;
+  if (grid > 0x7FFFFFFF) return DSEL_ERR_ROWS;
+  if (launch_cluster(sk, unsigned(grid), pl.cluster, sl.total, st, kp) != cudaSuccess) return DSEL_ERR_CUDA;
+  if (pl.groups > 1) {
+    const Layout ml = merge_layout(pl, eb);
+    KParams mp = kp;
+    mp.off_cb = ml.cb;
+    mp.off_ci = ml.ci;
+    mp.off_ctl = ml.ctl;
+    const int mc = merge_cluster(pl, base.k);
+    if (launch_cluster(mk, unsigned(rows * mc), mc, ml.total, st, mp) != cudaSuccess) return DSEL_ERR_CUDA;
+  }
+  return DSEL_OK;
+}
+
+}  // namespace
+}  // namespace dsel
+
+using namespace dsel;
+
+extern "C" {
+
+DSEL_API int64_t dsel_stride_requirement(int dtype) {
+  return (dtype == DSEL_BF16 || dtype == DSEL_F32) ? kStrideReq : -1;
+}
+
+DSEL_API const char* dsel_status_string(int status) {
+  switch (status) {
+    case DSEL_OK: return "ok";
+    case DSEL_ERR_DTYPE: return "dtype must be DSEL_BF16 or DSEL_F32";
+    case DSEL_ERR_INDEX_DTYPE: return "index_dtype must be DSEL_I32 or DSEL_I64";
+    case DSEL_ERR_K: return "k must be in [1, 4096]";
+    case DSEL_ERR_ROWS: return "rows must be >= 0 (and the grid must fit)";
+    case DSEL_ERR_STRIDE: return "row_stride must be a positive multiple of dsel_stride_requirement() and <= INT32_MAX";
+    case DSEL_ERR_ALIGN: return "x must be 16-byte aligned";
+    case DSEL_ERR_NULL: return "x and indices_out must not be NULL";
+    case DSEL_ERR_VALUES: return "values_out must be non-NULL exactly when return_value is set";
+    case DSEL_ERR_NAN_MODE: return "nan_mode must be DSEL_NAN_TRAP or DSEL_NAN_FLAG";
+    case DSEL_ERR_ORDER: return "sorted_index must be 0, 1 or 2 (2, value order, needs float32 input)";
+    case DSEL_ERR_DEVICE: return "the current device is not an sm_100 GPU";
+    case DSEL_ERR_WORKSPACE: return "could not allocate the split-row workspace";
+    case DSEL_ERR_CUDA: return "a CUDA runtime call failed";
+    case DSEL_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+    default: return "unknown status";
+  }
+}
+
+DSEL_API const char* dsel_version(void) { return "dsel 0.1.0 (sm_100a)"; }
+
+DSEL_API int dsel_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t num_sms,
+                       int32_t smem_optin, int32_t max_cluster, dsel_plan_t* out) {
+  return make_plan(dtype, rows, row_stride, k, num_sms, smem_optin, max_cluster, out);
+}
+
+DSEL_API int dsel_topk(const void* x, int dtype, int64_t rows, int64_t row_stride, const int32_t* end,
+                       int32_t k, int sorted_index, int return_value, int index_dtype, int nan_mode,
+                       void* values_out, void* indices_out, void* stream) {
+  int st = check_shape(dtype, rows, row_stride, k);
+  if (st != DSEL_OK) return st;
+  if (index_dtype != DSEL_I32 && index_dtype != DSEL_I64) return DSEL_ERR_INDEX_DTYPE;
+  if (nan_mode != DSEL_NAN_TRAP && nan_mode != DSEL_NAN_FLAG) return DSEL_ERR_NAN_MODE;
+  if (sorted_index < DSEL_ORDER_NONE || sorted_index > DSEL_ORDER_VALUE ||
+      (sorted_index == DSEL_ORDER_VALUE && dtype != DSEL_F32))
+    return DSEL_ERR_ORDER;
+  if (return_value != 0 && return_value != 1) return DSEL_ERR_VALUES;
+  if (rows == 0) return DSEL_OK;
+  if (x == nullptr || indices_out == nullptr) return DSEL_ERR_NULL;
+  if ((return_value != 0) != (values_out != nullptr)) return DSEL_ERR_VALUES;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) != 0) return DSEL_ERR_ALIGN;
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSEL_ERR_CUDA;
+  DevInfo* di = nullptr;
+  st = device_info(dev, &di);
+  if (st != DSEL_OK) return st;
+  dsel_plan_t pl;
+  st = make_plan(dtype, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster, &pl);
+  if (st != DSEL_OK) return st;
+
+  KParams kp = {};
+  kp.x = x;
+  kp.end = end;
+  kp.values_out = values_out;
+  kp.indices_out = indices_out;
+  kp.rows = rows;
+  kp.row_stride = row_stride;
+  kp.k = k;
+  kp.groups = pl.groups;
+  kp.b2 = pl.b2;
+  kp.stages = pl.stages;
+  kp.idx_bits = pl.idx_bits;
+  kp.order = sorted_index;
+  kp.return_value = return_value;
+  kp.index_i64 = index_dtype == DSEL_I64;
+  kp.nan_flag = nan_mode == DSEL_NAN_FLAG;
+  if (pl.groups > 1) {
+    void* ws = nullptr;
+    st = workspace(dev, stream, size_t(pl.workspace_bytes), &ws);
+    if (st != DSEL_OK) return st;
+    kp.ws_pairs = static_cast<uint2*>(ws);
+    kp.ws_meta = reinterpret_cast<int2*>(static_cast<char*>(ws) + rows * pl.groups * int64_t(k) * 8);
+  }
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return dtype == DSEL_BF16 ? run<DSEL_BF16>(kp, pl, rows, cs, di) : run<DSEL_F32>(kp, pl, rows, cs, di);
+}
+
+DSEL_API int dsel_device_status(int* status_out, void* stream) {
+  if (status_out == nullptr) return DSEL_ERR_NULL;
+  int v = 0, zero = 0;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyFromSymbolAsync(&v, g_device_status, sizeof(int), 0, cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+      cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+      cudaStreamSynchronize(cs) != cudaSuccess)
+    return DSEL_ERR_CUDA;
+  *status_out = v;
+  return DSEL_OK;
+}
+
+}  // extern "C"

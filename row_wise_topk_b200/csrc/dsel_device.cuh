@@ -1,0 +1,428 @@
+// Device building blocks for the row-wise TopK kernels (sm_100a).
+//
+// Method ("DeepSeek releases DeepSelect, a TopK kernel for sparse attention and
+// sampling", narracomm, method paragraph): a threshold T starts at -inf and only
+// rises; the row is read once, in contiguous blocks of B elements visited in a
+// random order; entries above T go to a candidate buffer in shared memory; when
+// the buffer holds k + B2 entries a radix select cuts it back to exactly k and
+// raises T to the k-th entry.
+//
+// Choices made here for B200:
+//   * blocks move global -> shared memory with the bulk-copy (TMA) engine
+//     (cp.async.bulk, completion on a per-stage mbarrier), many blocks in flight;
+//   * T is a composite (key, index) so that "above T" respects the tie rule
+//     (value descending, then index ascending) exactly, and a cheap float test
+//     (max of a 16-byte vector >= T, unordered) screens vectors before the exact
+//     test;  NaN fails every ordered compare, so the same test also catches NaN;
+//   * rows are split into contiguous slices handled by the CTAs of a
+//     thread-block cluster; CTAs share T through distributed shared memory and
+//     run the final radix select on the sum of their histograms.
+#pragma once
+
+#include <cooperative_groups.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dsel.h"
+
+namespace cg = cooperative_groups;
+
+namespace dsel {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // bounded waits: 2 s
+constexpr int kDigitBits = 8;
+constexpr int kBins = 1 << kDigitBits;
+
+__device__ int g_device_status;                    // DSEL_ERR_DEVICE_TIMEOUT when a wait gave up
+
+// --------------------------------------------------------------------------- //
+// Element traits: order-preserving keys.  Canonicalising -0 to +0 first makes
+// the two zeros one key; for every other non-NaN pattern, a larger value gives
+// a larger unsigned key (sign bit set -> invert all bits, else set the sign bit).
+// --------------------------------------------------------------------------- //
+template <int DT> struct Elem;
+
+template <> struct Elem<DSEL_BF16> {
+  using bits_t = uint16_t;
+  static constexpr int kKeyBits = 16;
+  static constexpr int kBytes = 2;
+  static constexpr int kPerVec = 8;
+  static constexpr uint32_t kQNaN = 0x7FC0u;
+  static constexpr uint32_t kNegInf = 0xFF80u;
+  __device__ __forceinline__ static uint32_t key(uint32_t b) {
+    b = (b == 0x8000u) ? 0u : b;
+    return (b & 0x8000u) ? (~b & 0xFFFFu) : (b | 0x8000u);
+  }
+  __device__ __forceinline__ static uint32_t bits_of_key(uint32_t k) {
+    return (k & 0x8000u) ? (k & 0x7FFFu) : (~k & 0xFFFFu);
+  }
+  __device__ __forceinline__ static bool is_nan(uint32_t b) { return (b & 0x7FFFu) > 0x7F80u; }
+};
+
+template <> struct Elem<DSEL_F32> {
+  using bits_t = uint32_t;
+  static constexpr int kKeyBits = 32;
+  static constexpr int kBytes = 4;
+  static constexpr int kPerVec = 4;
+  static constexpr uint32_t kQNaN = 0x7FC00000u;
+  static constexpr uint32_t kNegInf = 0xFF800000u;
+  __device__ __forceinline__ static uint32_t key(uint32_t b) {
+    b = (b == 0x80000000u) ? 0u : b;
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  }
+  __device__ __forceinline__ static uint32_t bits_of_key(uint32_t k) {
+    return (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  }
+  __device__ __forceinline__ static bool is_nan(uint32_t b) {
+    return (b & 0x7FFFFFFFu) > 0x7F800000u;
+  }
+};
+
+// Element e of a 16-byte vector (e is a compile-time constant after unrolling).
+template <int DT>
+__device__ __forceinline__ uint32_t vec_elem(const uint4& v, int e) {
+  uint32_t w = (DT == DSEL_BF16) ? ((e >> 1) == 0 ? v.x : (e >> 1) == 1 ? v.y : (e >> 1) == 2 ? v.z : v.w)
+                                 : (e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w);
+  if (DT == DSEL_BF16) return (e & 1) ? (w >> 16) : (w & 0xFFFFu);
+  return w;
+}
+
+// --------------------------------------------------------------------------- //
+// Screening test: true when some element of the vector may rank above T or is
+// NaN.  `tv` is the threshold's value bits (bf16 pattern duplicated in both
+// halves, or the f32 pattern).  Unordered >= is true for NaN on either side,
+// so the initial T (a NaN pattern: key 0) lets everything through.
+// --------------------------------------------------------------------------- //
+__device__ __forceinline__ uint32_t bf16x2_max_nan(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ bool bf16x2_any_geu(uint32_t a, uint32_t t) {
+  uint32_t r;
+  asm("{\n\t.reg .pred p, q;\n\t"
+      "setp.geu.bf16x2 p|q, %1, %2;\n\t"
+      "or.pred p, p, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r) : "r"(a), "r"(t));
+  return r != 0u;
+}
+
+__device__ __forceinline__ float f32_max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+template <int DT>
+__device__ __forceinline__ bool screen(const uint4& v, uint32_t tv) {
+  if (DT == DSEL_BF16) {
+    uint32_t m = bf16x2_max_nan(bf16x2_max_nan(v.x, v.y), bf16x2_max_nan(v.z, v.w));
+    return bf16x2_any_geu(m, tv);
+  } else {
+    float m = f32_max_nan(f32_max_nan(__uint_as_float(v.x), __uint_as_float(v.y)),
+                          f32_max_nan(__uint_as_float(v.z), __uint_as_float(v.w)));
+    return !(m < __uint_as_float(tv));
+  }
+}
+
+// --------------------------------------------------------------------------- //
+// PTX wrappers: mbarrier + bulk copy + timers.
+// --------------------------------------------------------------------------- //
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0u;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on a stage barrier; false when the limit ran out.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > kWaitLimitNs) {
+      atomicExch(&g_device_status, DSEL_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void nan_trap() { asm volatile("trap;"); }
+
+// --------------------------------------------------------------------------- //
+// Shared control block (one per CTA, after the candidate arrays).
+// --------------------------------------------------------------------------- //
+struct __align__(16) Ctl {
+  unsigned long long t_w;   // threshold composite (key << 32 | ~index); peers read it
+  int cnt;                  // candidates in the buffer
+  int nan_found;
+  int abort;
+  int x_cnt;                // exchanged with peers in the final phase
+  int x_nan;
+  int x_kept;
+  int tot;
+  int any_nan;
+  int kept_off;
+  int sel_digit, sel_above, sel_bucket;
+  int wsum[33];
+  int hist[2][kBins];
+  int hsum[kBins];
+};
+
+// Composite threshold word: larger means "ranks earlier".
+__device__ __forceinline__ unsigned long long make_w(uint32_t key, uint32_t idx) {
+  return (static_cast<unsigned long long>(key) << 32) | static_cast<uint32_t>(~idx);
+}
+
+// Radix word V = key << idx_bits | (idx_mask - idx): larger V ranks earlier and
+// V is unique within a row.
+template <int DT>
+__device__ __forceinline__ uint64_t make_v(uint32_t bits, uint32_t idx, int idx_bits,
+                                           uint32_t idx_mask) {
+  return (static_cast<uint64_t>(Elem<DT>::key(bits)) << idx_bits) | (idx_mask - idx);
+}
+
+struct SelResult {
+  uint64_t prefix;
+  int depth;
+};
+
+// Warp-inclusive scan.
+__device__ __forceinline__ int warp_incl_scan(int x, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  return x;
+}
+
+// Block-wide exclusive scan; every thread gets its offset and the total.
+template <int THREADS>
+__device__ __forceinline__ int block_excl_scan(int x, Ctl& ctl, int& total) {
+  constexpr int NW = THREADS / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = warp_incl_scan(x, lane);
+  if (lane == 31) ctl.wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < NW ? ctl.wsum[lane] : 0;
+    int wi = warp_incl_scan(w, lane);
+    if (lane < NW) ctl.wsum[lane] = wi - w;
+    if (lane == 31) ctl.wsum[32] = wi;
+  }
+  __syncthreads();
+  int res = ctl.wsum[warp] + incl - x;
+  total = ctl.wsum[32];
+  __syncthreads();
+  return res;
+}
+
+// --------------------------------------------------------------------------- //
+// MSB-first radix select over V.  Finds (prefix, depth) such that exactly `need`
+// candidates have their top `depth` bits >= prefix.  In cluster mode every CTA
+// holds part of the candidates; histograms are summed over the cluster through
+// distributed shared memory and every CTA takes the same decision.
+// --------------------------------------------------------------------------- //
+template <int DT, int THREADS, bool CLUSTER>
+__device__ SelResult radix_select(const typename Elem<DT>::bits_t* cb, const uint32_t* ci, int cnt,
+                                  int need, int idx_bits, Ctl& ctl, cg::cluster_group& cluster) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int total_bits = Elem<DT>::kKeyBits + idx_bits;
+  const uint32_t idx_mask = idx_bits >= 32 ? 0xFFFFFFFFu : ((1u << idx_bits) - 1u);
+  uint64_t prefix = 0;
+  int depth = 0;
+  int par = 0;
+  while (true) {
+    const int dbits = min(kDigitBits, total_bits - depth);
+    const int shift = total_bits - depth - dbits;
+    const uint32_t dmask = (1u << dbits) - 1u;
+    int* h = ctl.hist[par];
+    for (int i = tid; i < kBins; i += THREADS) h[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < cnt; i += THREADS) {
+      const uint64_t v = make_v<DT>(cb[i], ci[i], idx_bits, idx_mask);
+      if ((v >> (shift + dbits)) == prefix) atomicAdd(&h[static_cast<uint32_t>(v >> shift) & dmask], 1);
+    }
+    const int* H = h;
+    if (CLUSTER) {
+      cluster.sync();
+      const int nr = static_cast<int>(cluster.num_blocks());
+      for (int b = tid; b < kBins; b += THREADS) {
+        int s = 0;
+        for (int r = 0; r < nr; ++r) s += cluster.map_shared_rank(h, r)[b];
+        ctl.hsum[b] = s;
+      }
+      H = ctl.hsum;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int c[kBins / 32];
+      int s = 0;
+#pragma unroll
+      for (int j = 0; j < kBins / 32; ++j) {
+        c[j] = H[kBins - 1 - (lane * (kBins / 32) + j)];
+        s += c[j];
+      }
+      const int incl = warp_incl_scan(s, lane);
+      int acc = incl - s;
+      if (acc < need && need <= incl) {
+        bool done = false;
+#pragma unroll
+        for (int j = 0; j < kBins / 32; ++j) {
+          if (!done && acc + c[j] >= need) {
+            ctl.sel_digit = kBins - 1 - (lane * (kBins / 32) + j);
+            ctl.sel_above = acc;
+            ctl.sel_bucket = c[j];
+            done = true;
+          }
+          acc += c[j];
+        }
+      }
+    }
+    __syncthreads();
+    const int digit = ctl.sel_digit, above = ctl.sel_above, bucket = ctl.sel_bucket;
+    need -= above;
+    prefix = (prefix << dbits) | static_cast<uint64_t>(digit);
+    depth += dbits;
+    par ^= 1;
+    if (need == bucket || depth == total_bits) break;
+  }
+  return {prefix, depth};
+}
+
+// Keep the candidates whose top `depth` bits are >= prefix, preserving their order
+// (each thread owns a contiguous run of EPT slots).  Returns the kept count.
+template <int DT, int THREADS>
+__device__ int stable_compact(typename Elem<DT>::bits_t* cb, uint32_t* ci, int cnt, SelResult sel,
+                              int idx_bits, Ctl& ctl) {
+  using bits_t = typename Elem<DT>::bits_t;
+  constexpr int EPT = 8;
+  const int tid = threadIdx.x;
+  const int total_bits = Elem<DT>::kKeyBits + idx_bits;
+  const uint32_t idx_mask = idx_bits >= 32 ? 0xFFFFFFFFu : ((1u << idx_bits) - 1u);
+  const int sh = total_bits - sel.depth;
+  int out = 0;
+  for (int base = 0; base < cnt; base += THREADS * EPT) {
+    bits_t b[EPT];
+    uint32_t ix[EPT];
+    uint32_t km = 0;
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) {
+      const int i = base + tid * EPT + e;
+      b[e] = 0;
+      ix[e] = 0;
+      if (i < cnt) {
+        b[e] = cb[i];
+        ix[e] = ci[i];
+        if ((make_v<DT>(b[e], ix[e], idx_bits, idx_mask) >> sh) >= sel.prefix) km |= 1u << e;
+      }
+    }
+    int total;
+    int pos = out + block_excl_scan<THREADS>(__popc(km), ctl, total);
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) {
+      if (km & (1u << e)) {
+        cb[pos] = b[e];
+        ci[pos] = ix[e];
+        ++pos;
+      }
+    }
+    out += total;
+  }
+  __syncthreads();
+  return out;
+}
+
+// Threshold word for a selection result: the smallest V with that prefix.
+__device__ __forceinline__ unsigned long long threshold_of(SelResult sel, int key_bits, int idx_bits) {
+  const int total_bits = key_bits + idx_bits;
+  const uint32_t idx_mask = idx_bits >= 32 ? 0xFFFFFFFFu : ((1u << idx_bits) - 1u);
+  const uint64_t v = sel.prefix << (total_bits - sel.depth);
+  const uint32_t key = static_cast<uint32_t>(v >> idx_bits);
+  const uint32_t rev = static_cast<uint32_t>(v) & idx_mask;
+  return make_w(key, idx_mask - rev);
+}
+
+// Bitonic sort of m (<= capacity, padded to a power of two) candidates in shared
+// memory.  BY_VALUE: value descending, then index ascending; else index ascending.
+template <int DT, int THREADS, bool BY_VALUE>
+__device__ void bitonic_sort(typename Elem<DT>::bits_t* cb, uint32_t* ci, int m) {
+  const int tid = threadIdx.x;
+  int M = 1;
+  while (M < m) M <<= 1;
+  for (int i = m + tid; i < M; i += THREADS) {
+    ci[i] = 0xFFFFFFFFu;
+    cb[i] = static_cast<typename Elem<DT>::bits_t>(Elem<DT>::kNegInf);
+  }
+  __syncthreads();
+  for (int size = 2; size <= M; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = tid; t < (M >> 1); t += THREADS) {
+        const int lo = 2 * t - (t & (stride - 1));
+        const int hi = lo + stride;
+        const bool asc = (lo & size) == 0;
+        const uint32_t ia = ci[lo], ib = ci[hi];
+        bool gt;
+        if (BY_VALUE) {
+          // sort key ascending = (inverted key, index): value desc then index asc.
+          // Padding (index 0xFFFFFFFF, -inf) lands after every real entry.
+          const uint64_t ka = (static_cast<uint64_t>(~Elem<DT>::key(cb[lo])) << 32) | ia;
+          const uint64_t kb = (static_cast<uint64_t>(~Elem<DT>::key(cb[hi])) << 32) | ib;
+          gt = ka > kb;
+        } else {
+          gt = ia > ib;
+        }
+        if (gt == asc) {
+          const auto ba = cb[lo];
+          cb[lo] = cb[hi];
+          cb[hi] = ba;
+          ci[lo] = ib;
+          ci[hi] = ia;
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+}  // namespace dsel

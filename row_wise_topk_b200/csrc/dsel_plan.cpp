@@ -1,0 +1,86 @@
+// Launch planner: picks the CTA shape, the row split and the ring depth.
+//
+// The pages fix only B = B2 = 1024 for k = 512 ("DeepSeek releases DeepSelect, a
+// TopK kernel for sparse attention and sampling", method paragraph) and say both
+// should sit "on the order of k"; everything else here is this library's choice
+// for a 148-SM B200:
+//   * one CTA per row while there are at least as many rows as SMs;
+//   * otherwise each row is cut into S contiguous slices, one CTA each, grouped in
+//     thread-block clusters of C CTAs that share the threshold and merge through
+//     distributed shared memory; rows too long for one cluster (S > max_cluster)
+//     get G clusters and a second, merging launch;
+//   * the shared-memory ring holds as many blocks in flight as fit next to the
+//     candidate buffer (up to the whole slice).
+#include "dsel_plan.h"
+
+#include <algorithm>
+
+namespace dsel {
+
+int check_shape(int dtype, int64_t rows, int64_t row_stride, int32_t k) {
+  if (dtype != DSEL_BF16 && dtype != DSEL_F32) return DSEL_ERR_DTYPE;
+  if (k < 1 || k > kMaxK) return DSEL_ERR_K;
+  if (rows < 0) return DSEL_ERR_ROWS;
+  if (row_stride < 1 || row_stride > INT32_MAX || row_stride % kStrideReq != 0)
+    return DSEL_ERR_STRIDE;
+  return DSEL_OK;
+}
+
+static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+static int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t num_sms,
+              int32_t smem_optin, int32_t max_cluster, dsel_plan_t* out) {
+  int st = check_shape(dtype, rows, row_stride, k);
+  if (st != DSEL_OK) return st;
+  if (out == nullptr || num_sms < 1 || smem_optin < 48 * 1024 || max_cluster < 1)
+    return DSEL_ERR_DEVICE;
+
+  const int eb = elem_bytes(dtype);
+  dsel_plan_t p{};
+  p.threads = kThreads;
+  p.block = kBlockElems;
+  p.round = kRoundElems;
+  p.b2 = k <= 1024 ? 1024 : std::min(k, 2048);
+  p.capacity = int(round_up(std::max<int64_t>(k + p.b2 + p.round, next_pow2(k)), 32));
+  p.idx_bits = ceil_log2_u64(uint64_t(row_stride));
+
+  // Row split.
+  int64_t splits = 1;
+  if (rows < num_sms) {
+    splits = num_sms / std::max<int64_t>(rows, 1);
+    splits = std::min<int64_t>(splits, std::max<int64_t>(1, row_stride / kMinSliceElems));
+    splits = std::max<int64_t>(splits, 1);
+  }
+  int64_t cluster = std::min<int64_t>(splits, max_cluster);
+  int64_t groups = std::max<int64_t>(1, splits / cluster);
+  // the merge holds all groups' partial results across at most kMaxCluster CTAs
+  const int64_t max_groups =
+      std::min<int64_t>(kMaxGroups, std::max<int64_t>(1, int64_t(kMaxCluster) * p.capacity / k));
+  groups = std::min(groups, max_groups);
+  p.cluster = int(cluster);
+  p.groups = int(groups);
+
+  // Ring depth.
+  const int64_t slice = round_up(ceil_div(row_stride, groups * cluster), kStrideReq);
+  const int64_t nb_max = ceil_div(slice, p.block);
+  const int64_t per_round = p.round / p.block;
+  const int64_t base = stream_smem_bytes(0, p.block, p.capacity, eb) + 256;
+  const int64_t per_stage = int64_t(p.block) * eb + 8 + 4;
+  int64_t stages = (int64_t(smem_optin) - base) / per_stage;
+  stages = std::min<int64_t>(stages, kMaxStages);
+  stages = std::min<int64_t>(stages, std::max<int64_t>(nb_max, per_round));
+  stages = std::max<int64_t>(stages, per_round);
+  p.stages = int(stages);
+  const int64_t smem = stream_smem_bytes(stages, p.block, p.capacity, eb);
+  if (smem > smem_optin) return DSEL_ERR_K;
+  p.smem_bytes = int(smem);
+
+  // Split-row workspace: each cluster leaves up to k (bits, index) pairs and a
+  // (count, flags) word per row.
+  p.workspace_bytes = groups > 1 ? rows * groups * (int64_t(k) * 8 + 8) : 0;
+  *out = p;
+  return DSEL_OK;
+}
+
+}  // namespace dsel

@@ -1,0 +1,67 @@
+// Host-side launch planner for the row-wise TopK kernels.  Pure C++: no CUDA call,
+// so it is unit-tested on machines without a GPU through dsel_plan().
+#pragma once
+#include <cstdint>
+
+#include "../../include/dsel.h"
+
+namespace dsel {
+
+// Compile-time CTA shapes.  The streaming kernel is instantiated for exactly
+// these (dtype, threads) pairs; the planner only ever returns one of them.
+constexpr int kThreads = 512;
+constexpr int kVecBytes = 16;                 // one 128-bit load per thread per step
+constexpr int kRoundElems = 4096;             // elements filtered between buffer checks
+constexpr int kBlockElems = 1024;             // B: the pages' setting for k = 512
+constexpr int kStrideReq = 16;                // row_stride multiple (elements)
+constexpr int kMaxStages = 128;               // ring depth cap (one mbarrier per stage)
+constexpr int kMinSliceElems = 8192;          // smallest row share worth its own CTA
+constexpr int kSharedFixedBytes = 4096;       // scalars, histograms, scan scratch
+constexpr int kMaxK = 4096;
+constexpr int kMaxCluster = 8;               // portable cluster size
+constexpr int kMaxGroups = 255;               // clusters per row (merge keeps one prefix per group)
+
+inline int elem_bytes(int dtype) { return dtype == DSEL_BF16 ? 2 : 4; }
+
+// Vectors per thread per round: the round is kRoundElems for both dtypes.
+inline int vectors_per_thread(int dtype) {
+  return kRoundElems / (kThreads * (kVecBytes / elem_bytes(dtype)));
+}
+
+inline int ceil_log2_u64(uint64_t v) {   // smallest b with 2^b >= v (v >= 1)
+  int b = 0;
+  while ((uint64_t(1) << b) < v) ++b;
+  return b;
+}
+
+inline int next_pow2(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+// CTAs per row in the merge launch of a split-row plan: enough that each holds at
+// most `capacity` of the groups' partial results.
+inline int merge_cluster(const dsel_plan_t& p, int k) {
+  const int64_t total = int64_t(p.groups) * k;
+  int c = int((total + p.capacity - 1) / p.capacity);
+  if (c < 1) c = 1;
+  if (c > kMaxCluster) c = kMaxCluster;
+  return c;
+}
+
+// Shared-memory bytes of the streaming kernel for a plan (upper bound of the
+// device layout: ring, mbarriers, block table, candidate arrays, control block).
+inline int64_t stream_smem_bytes(int64_t stages, int64_t block, int64_t capacity, int eb) {
+  auto up = [](int64_t v, int64_t a) { return (v + a - 1) / a * a; };
+  return up(stages * block * eb, 128) + up(stages * 8, 16) + up(stages * 4, 16) +
+         up(capacity * eb, 16) + up(capacity * 4, 16) + kSharedFixedBytes;
+}
+
+int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t num_sms,
+              int32_t smem_optin, int32_t max_cluster, dsel_plan_t* out);
+
+// Argument checks shared by dsel_topk and dsel_plan (host only).
+int check_shape(int dtype, int64_t rows, int64_t row_stride, int32_t k);
+
+}  // namespace dsel

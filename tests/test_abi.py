@@ -1,0 +1,132 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, validates arguments on the host before touching CUDA, and the
+host-side planner returns consistent plans."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import row_wise_topk_b200 as T
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "dsel.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"DSEL_API\s+[\w\s\*]+?\b(dsel_\w+)\s*\(", text)
+
+
+def header_define(name):
+    m = re.search(r"#define\s+%s\s+\(?(-?\d+)\)?" % name, open(HEADER).read())
+    return int(m.group(1))
+
+
+def test_every_declared_symbol_is_exported():
+    syms = declared_symbols()
+    assert "dsel_topk" in syms and len(syms) >= 6
+    lib = ctypes.CDLL(T.LIB_PATH)
+    for s in syms:
+        assert hasattr(lib, s), s
+
+
+def test_python_constants_match_header():
+    for name in ["DSEL_BF16", "DSEL_F32", "DSEL_I32", "DSEL_I64", "DSEL_NAN_TRAP", "DSEL_NAN_FLAG",
+                 "DSEL_ORDER_NONE", "DSEL_ORDER_INDEX", "DSEL_ORDER_VALUE", "DSEL_IDX_PAD",
+                 "DSEL_IDX_NAN", "DSEL_IDX_BAD_END", "DSEL_OK"]:
+        assert getattr(T, name) == header_define(name), name
+
+
+def test_stride_requirement_and_strings():
+    assert T.dsel_stride_requirement(T.DSEL_BF16) == 16
+    assert T.dsel_stride_requirement(T.DSEL_F32) == 16
+    assert T.dsel_stride_requirement(7) == -1
+    for code in range(0, -15, -1):
+        s = T.dsel_status_string(code)
+        assert s and s != "unknown status", code
+    assert T.dsel_status_string(-99) == "unknown status"
+    assert "sm_100a" in T.dsel_version()
+
+
+def call(**kw):
+    a = dict(x=0x1000, dtype=T.DSEL_F32, rows=4, row_stride=8192, end=None, k=64, sorted_index=1,
+             return_value=1, index_dtype=T.DSEL_I64, nan_mode=T.DSEL_NAN_TRAP, values_out=0x2000,
+             indices_out=0x3000, stream=None)
+    a.update(kw)
+    return T.dsel_topk(**a)
+
+
+@pytest.mark.parametrize("kw,err", [
+    (dict(dtype=2), "DSEL_ERR_DTYPE"),
+    (dict(k=0), "DSEL_ERR_K"),
+    (dict(k=4097), "DSEL_ERR_K"),
+    (dict(rows=-1), "DSEL_ERR_ROWS"),
+    (dict(row_stride=8190), "DSEL_ERR_STRIDE"),
+    (dict(row_stride=0), "DSEL_ERR_STRIDE"),
+    (dict(row_stride=1 << 32), "DSEL_ERR_STRIDE"),
+    (dict(index_dtype=3), "DSEL_ERR_INDEX_DTYPE"),
+    (dict(nan_mode=2), "DSEL_ERR_NAN_MODE"),
+    (dict(sorted_index=3), "DSEL_ERR_ORDER"),
+    (dict(sorted_index=2, dtype=T.DSEL_BF16), "DSEL_ERR_ORDER"),
+    (dict(x=None), "DSEL_ERR_NULL"),
+    (dict(indices_out=None), "DSEL_ERR_NULL"),
+    (dict(values_out=None), "DSEL_ERR_VALUES"),
+    (dict(return_value=0), "DSEL_ERR_VALUES"),
+    (dict(return_value=2), "DSEL_ERR_VALUES"),
+    (dict(x=0x1004), "DSEL_ERR_ALIGN"),
+])
+def test_host_argument_checks(kw, err):
+    assert call(**kw) == header_define(err)
+
+
+def test_zero_rows_is_a_noop():
+    assert call(rows=0, x=None, indices_out=None, values_out=None, return_value=0) == 0
+
+
+PEAK = dict(num_sms=148, smem_optin=232448, max_cluster=8)
+
+
+@pytest.mark.parametrize("dtype,rows,stride,k", [
+    (T.DSEL_F32, 4, 8192, 64),
+    (T.DSEL_BF16, 64, 131072, 512),
+    (T.DSEL_BF16, 4096, 16384, 512),
+    (T.DSEL_F32, 1, 129280, 50), (T.DSEL_F32, 8, 129280, 1024), (T.DSEL_F32, 64, 129280, 4096),
+    (T.DSEL_F32, 256, 129280, 4096),
+    (T.DSEL_F32, 1, 1 << 28, 1000), (T.DSEL_F32, 16, 1 << 24, 4096),
+    (T.DSEL_BF16, 3, 16, 4096), (T.DSEL_F32, 1, 16, 1),
+])
+def test_plan_invariants(dtype, rows, stride, k):
+    st, p = T.dsel_plan(dtype, rows, stride, k, **PEAK)
+    assert st == 0
+    eb = 2 if dtype == T.DSEL_BF16 else 4
+    assert p["smem_bytes"] <= PEAK["smem_optin"]
+    assert p["capacity"] >= k + p["b2"] + p["round"]
+    assert p["capacity"] >= 1 << (k - 1).bit_length()          # room for the bitonic padding
+    assert p["stages"] >= p["round"] // p["block"]
+    assert p["round"] % p["block"] == 0 and (p["block"] * eb) % 16 == 0
+    assert 1 <= p["cluster"] <= PEAK["max_cluster"]
+    assert p["groups"] >= 1 and p["groups"] * k <= 8 * p["capacity"]
+    assert (1 << p["idx_bits"]) >= stride
+    assert p["idx_bits"] + 8 * eb <= 63
+    if p["groups"] > 1:
+        assert p["workspace_bytes"] >= rows * p["groups"] * k * 8
+    else:
+        assert p["workspace_bytes"] == 0
+    # the row is split at most once per SM
+    assert rows * p["cluster"] * p["groups"] <= max(rows, PEAK["num_sms"])
+
+
+def test_plan_splits():
+    # many rows: one CTA per row
+    assert T.dsel_plan(T.DSEL_BF16, 4096, 16384, 512, **PEAK)[1]["cluster"] == 1
+    # 64 indexer rows: two CTAs per row
+    p = T.dsel_plan(T.DSEL_BF16, 64, 131072, 512, **PEAK)[1]
+    assert (p["cluster"], p["groups"]) == (2, 1)
+    # a single 2^28 row uses several clusters
+    p = T.dsel_plan(T.DSEL_F32, 1, 1 << 28, 1000, **PEAK)[1]
+    assert p["groups"] > 1 and p["cluster"] == 8
+
+
+def test_plan_rejects_bad_args():
+    assert T.dsel_plan(T.DSEL_F32, 4, 8191, 64, **PEAK)[0] == header_define("DSEL_ERR_STRIDE")
+    assert T.dsel_plan(T.DSEL_F32, 4, 8192, 5000, **PEAK)[0] == header_define("DSEL_ERR_K")
