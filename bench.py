@@ -283,8 +283,8 @@ def run_ours(args, w, world, rank, local, pg):
     # graph of S steps (S = number of input copies, so each replay touches every copy once)
     S = n_copies
     graph = torch.cuda.CUDAGraph()
-    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(S)]
-    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(S)]
+    ev_a = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(S)]
+    ev_b = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(S)]
     with torch.cuda.graph(graph, stream=stream):
         for i in range(S):
             ev_a[i].record()
@@ -331,7 +331,10 @@ def run_ours(args, w, world, rank, local, pg):
         pg.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
     # per-step device times from the last full replay (events inside the graph)
-    per_step_ms = [ev_a[i].elapsed_time(ev_b[i]) for i in range(S)] if full else [elapsed_ms / args.steps]
+    try:
+        per_step_ms = [ev_a[i].elapsed_time(ev_b[i]) for i in range(S)] if full else [elapsed_ms / args.steps]
+    except Exception:      # event nodes unavailable: fall back to the region average
+        per_step_ms = [elapsed_ms / args.steps]
     time.sleep(0.2)
     clocks = sampler.stop()
 

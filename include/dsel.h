@@ -107,6 +107,7 @@ extern "C" {
 #define DSEL_ERR_WORKSPACE (-12)   /* the split-row workspace could not be allocated */
 #define DSEL_ERR_CUDA (-13)        /* a CUDA runtime call failed (launch error forwarded) */
 #define DSEL_ERR_DEVICE_TIMEOUT (-14) /* a kernel gave up a bounded wait (see dsel_device_status) */
+#define DSEL_ERR_UNAVAILABLE (-15) /* the entry point is not part of this build */
 
 /* Launch plan chosen for a call (see dsel_plan). */
 typedef struct {
@@ -161,6 +162,17 @@ DSEL_API int dsel_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k,
  * wait runs out (it should never happen).  Synchronises `stream`.  *status_out
  * receives 0 or DSEL_ERR_DEVICE_TIMEOUT.  Returns DSEL_OK or DSEL_ERR_CUDA. */
 DSEL_API int dsel_device_status(int* status_out, void* stream);
+
+/* Per-CTA counters of the last streaming launch, for tuning.  Only builds made
+ * with -DDSEL_STATS record them; other builds return DSEL_ERR_UNAVAILABLE.
+ * host_out receives n_ctas x 16 uint64 (CTA = blockIdx.x of the streaming kernel):
+ * stream cycles, final-phase cycles, compaction cycles, compactions, candidates
+ * appended, screened vectors sent to the exact test, rounds, final buffer count,
+ * then cycle times (from kernel start, thread 0) of: set-up done, prologue
+ * issued, first round filtered, first round barrier, first compaction done,
+ * stream done; then thread 0's cycles waiting for blocks, and total cycles.
+ * Synchronises `stream`. */
+DSEL_API int dsel_debug_stats(uint64_t* host_out, int64_t n_ctas, void* stream);
 
 /* Library version string. */
 DSEL_API const char* dsel_version(void);

@@ -15,7 +15,9 @@ import os
 from typing import Optional, Tuple
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdsel.so")
+# ROW_WISE_TOPK_LIB may name another build of this same library (for example the
+# counter-instrumented libdsel_stats.so); it must sit in this package directory.
+LIB_PATH = os.path.join(_HERE, os.path.basename(os.environ.get("ROW_WISE_TOPK_LIB", "libdsel.so")))
 
 # Constants of include/dsel.h
 DSEL_BF16, DSEL_F32 = 0, 1
@@ -54,7 +56,7 @@ class DselError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m row_wise_topk_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python row_wise_topk_b200/build.py` "
             "(the CUDA library is required; there is no fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     c_int, c_i64, vp = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
@@ -70,6 +72,8 @@ def _load() -> ctypes.CDLL:
                               ctypes.c_int32, ctypes.POINTER(DselPlan)]
     lib.dsel_device_status.restype = c_int
     lib.dsel_device_status.argtypes = [ctypes.POINTER(c_int), vp]
+    lib.dsel_debug_stats.restype = c_int
+    lib.dsel_debug_stats.argtypes = [ctypes.c_void_p, c_i64, vp]
     lib.dsel_version.restype = ctypes.c_char_p
     lib.dsel_version.argtypes = []
     return lib
@@ -113,6 +117,16 @@ def dsel_device_status(stream: Optional[int] = None) -> int:
     if st != DSEL_OK:
         raise DselError(st)
     return out.value
+
+
+def dsel_debug_stats(n_ctas: int, stream: Optional[int] = None):
+    """Per-CTA counters of the last streaming launch (counter builds only), as a
+    list of 16-tuples; raises DselError(DSEL_ERR_UNAVAILABLE) otherwise."""
+    buf = (ctypes.c_uint64 * (16 * n_ctas))()
+    st = lib.dsel_debug_stats(ctypes.cast(buf, ctypes.c_void_p), n_ctas, stream)
+    if st != DSEL_OK:
+        raise DselError(st)
+    return [tuple(buf[16 * i: 16 * i + 16]) for i in range(n_ctas)]
 
 
 def dsel_version() -> str:

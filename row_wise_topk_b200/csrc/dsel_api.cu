@@ -75,42 +75,6 @@ int workspace(int dev, void* stream, size_t bytes, void** out) {
   return DSEL_OK;
 }
 
-struct Layout {
-  uint32_t bars, blk, cb, ci, ctl, total;
-};
-
-uint32_t align_up(uint64_t v, uint64_t a) { return static_cast<uint32_t>((v + a - 1) / a * a); }
-
-Layout stream_layout(const dsel_plan_t& pl, int eb) {
-  Layout l{};
-  uint64_t off = align_up(uint64_t(pl.stages) * pl.block * eb, 128);
-  l.bars = uint32_t(off);
-  off += align_up(uint64_t(pl.stages) * 8, 16);
-  l.blk = uint32_t(off);
-  off += align_up(uint64_t(pl.stages) * 4, 16);
-  l.cb = uint32_t(off);
-  off += align_up(uint64_t(pl.capacity) * eb, 16);
-  l.ci = uint32_t(off);
-  off += align_up(uint64_t(pl.capacity) * 4, 16);
-  l.ctl = uint32_t(off);
-  off += align_up(sizeof(Ctl), 16);
-  l.total = uint32_t(off);
-  return l;
-}
-
-Layout merge_layout(const dsel_plan_t& pl, int eb) {
-  Layout l{};
-  uint64_t off = 0;
-  l.cb = 0;
-  off += align_up(uint64_t(pl.capacity) * eb, 16);
-  l.ci = uint32_t(off);
-  off += align_up(uint64_t(pl.capacity) * 4, 16);
-  l.ctl = uint32_t(off);
-  off += align_up(sizeof(Ctl), 16);
-  l.total = uint32_t(off);
-  return l;
-}
-
 template <typename Kern>
 cudaError_t launch_cluster(Kern kern, unsigned grid, int cluster, uint32_t smem, cudaStream_t st,
                            const KParams& kp) {
@@ -142,23 +106,27 @@ int run(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t s
     di->attrs_set[DT] = true;
   }
   const int eb = elem_bytes(DT);
-  const Layout sl = stream_layout(pl, eb);
+  const SmemLayout sl = stream_layout(pl.stages, pl.block, pl.capacity, int64_t(base.k) + pl.b2, eb);
   KParams kp = base;
   kp.off_bars = sl.bars;
   kp.off_blk = sl.blk;
   kp.off_cb = sl.cb;
   kp.off_ci = sl.ci;
+  kp.off_holes = sl.holes;
   kp.off_ctl = sl.ctl;
+  kp.gather = int64_t(pl.cluster) * base.k <= pl.capacity;
   const int64_t grid = rows * pl.groups * pl.cluster;
   if (grid > 0x7FFFFFFF) return DSEL_ERR_ROWS;
   if (launch_cluster(sk, unsigned(grid), pl.cluster, sl.total, st, kp) != cudaSuccess) return DSEL_ERR_CUDA;
   if (pl.groups > 1) {
-    const Layout ml = merge_layout(pl, eb);
+    const SmemLayout ml = merge_layout(pl.capacity, int64_t(base.k) + pl.b2, eb);
     KParams mp = kp;
     mp.off_cb = ml.cb;
     mp.off_ci = ml.ci;
+    mp.off_holes = ml.holes;
     mp.off_ctl = ml.ctl;
     const int mc = merge_cluster(pl, base.k);
+    mp.gather = int64_t(mc) * base.k <= pl.capacity;
     if (launch_cluster(mk, unsigned(rows * mc), mc, ml.total, st, mp) != cudaSuccess) return DSEL_ERR_CUDA;
   }
   return DSEL_OK;
@@ -192,8 +160,34 @@ DSEL_API const char* dsel_status_string(int status) {
     case DSEL_ERR_WORKSPACE: return "could not allocate the split-row workspace";
     case DSEL_ERR_CUDA: return "a CUDA runtime call failed";
     case DSEL_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+    case DSEL_ERR_UNAVAILABLE: return "not available in this build";
     default: return "unknown status";
   }
+}
+
+DSEL_API int dsel_debug_stats(uint64_t* host_out, int64_t n_ctas, void* stream) {
+#ifdef DSEL_STATS
+  if (host_out == nullptr || n_ctas < -1) return DSEL_ERR_NULL;
+  const int64_t n = n_ctas < kStatsCtas ? n_ctas : kStatsCtas;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (n_ctas == -1) {   // the per-round timeline instead (4 x 64 x 6 values)
+    if (cudaMemcpyFromSymbolAsync(host_out, g_trace, sizeof(long long) * 4 * kTraceRounds * kTraceEvents, 0,
+                                  cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+        cudaStreamSynchronize(cs) != cudaSuccess)
+      return DSEL_ERR_CUDA;
+    return DSEL_OK;
+  }
+  if (cudaMemcpyFromSymbolAsync(host_out, g_stats, size_t(n) * kStatsFields * sizeof(uint64_t), 0,
+                                cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+      cudaStreamSynchronize(cs) != cudaSuccess)
+    return DSEL_ERR_CUDA;
+  return DSEL_OK;
+#else
+  (void)host_out;
+  (void)n_ctas;
+  (void)stream;
+  return DSEL_ERR_UNAVAILABLE;
+#endif
 }
 
 DSEL_API const char* dsel_version(void) { return "dsel 0.1.0 (sm_100a)"; }

@@ -115,6 +115,42 @@ __device__ __forceinline__ float f32_max_nan(float a, float b) {
   return d;
 }
 
+// Candidate mask of a vector: bit e set when element e is >= T as a float, or NaN
+// (unordered compare).  A superset of the elements that can rank above T.
+__device__ __forceinline__ uint32_t bf16x2_geu_mask(uint32_t a, uint32_t t) {
+  uint32_t r;
+  asm("{\n\t.reg .pred p, q;\n\t"
+      "setp.geu.bf16x2 p|q, %1, %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "@q or.b32 %0, %0, 2;\n\t}"
+      : "=r"(r) : "r"(a), "r"(t));
+  return r;
+}
+
+template <int DT>
+__device__ __forceinline__ uint32_t candidate_mask(const uint4& v, uint32_t tv) {
+  if (DT == DSEL_BF16) {
+    return bf16x2_geu_mask(v.x, tv) | (bf16x2_geu_mask(v.y, tv) << 2) | (bf16x2_geu_mask(v.z, tv) << 4) |
+           (bf16x2_geu_mask(v.w, tv) << 6);
+  } else {
+    const float t = __uint_as_float(tv);
+    return (!(__uint_as_float(v.x) < t) ? 1u : 0u) | (!(__uint_as_float(v.y) < t) ? 2u : 0u) |
+           (!(__uint_as_float(v.z) < t) ? 4u : 0u) | (!(__uint_as_float(v.w) < t) ? 8u : 0u);
+  }
+}
+
+// Element e (a run-time value) of a 16-byte vector, without local memory.
+template <int DT>
+__device__ __forceinline__ uint32_t vec_elem_dyn(const uint4& v, int e) {
+  if (DT == DSEL_BF16) {
+    const int wi = e >> 1;
+    const uint32_t w = wi < 2 ? (wi == 0 ? v.x : v.y) : (wi == 2 ? v.z : v.w);
+    return (w >> ((e & 1) * 16)) & 0xFFFFu;
+  } else {
+    return e < 2 ? (e == 0 ? v.x : v.y) : (e == 2 ? v.z : v.w);
+  }
+}
+
 template <int DT>
 __device__ __forceinline__ bool screen(const uint4& v, uint32_t tv) {
   if (DT == DSEL_BF16) {
@@ -191,21 +227,27 @@ __device__ __forceinline__ void nan_trap() { asm volatile("trap;"); }
 // --------------------------------------------------------------------------- //
 // Shared control block (one per CTA, after the candidate arrays).
 // --------------------------------------------------------------------------- //
+constexpr int kWarpsMax = 32;
+
 struct __align__(16) Ctl {
-  unsigned long long t_w;   // threshold composite (key << 32 | ~index); peers read it
-  int cnt;                  // candidates in the buffer
+  unsigned long long t_w;       // threshold word raised by peers (atomicMax); own T lives in registers
+  unsigned long long x_vlo, x_vhi;
+  unsigned long long wv[kWarpsMax];   // per-warp radix-word maxima
   int nan_found;
   int abort;
-  int x_cnt;                // exchanged with peers in the final phase
-  int x_nan;
-  int x_kept;
-  int tot;
-  int any_nan;
-  int kept_off;
-  int sel_digit, sel_above, sel_bucket;
-  int wsum[33];
-  int hist[2][kBins];
+  int hb;                       // index of a histogram that is all zero
+  int x_cnt, x_nan, x_kept;     // exchanged with peers in the final phase
+  int sel_flag;
+  int wc[2][kWarpsMax];         // per-warp counts, by round parity
+  int wm[kWarpsMax];            // per-warp counts (compaction movers)
+  int hist[3][kBins];
   int hsum[kBins];
+#ifdef DSEL_STATS
+  unsigned long long st_compact_cycles;
+  int st_compactions;
+  int st_appended;
+  int st_slow_vectors;
+#endif
 };
 
 // Composite threshold word: larger means "ranks earlier".
@@ -215,6 +257,8 @@ __device__ __forceinline__ unsigned long long make_w(uint32_t key, uint32_t idx)
 
 // Radix word V = key << idx_bits | (idx_mask - idx): larger V ranks earlier and
 // V is unique within a row.
+__device__ __forceinline__ uint32_t mask_bits(int b) { return b >= 32 ? 0xFFFFFFFFu : ((1u << b) - 1u); }
+
 template <int DT>
 __device__ __forceinline__ uint64_t make_v(uint32_t bits, uint32_t idx, int idx_bits,
                                            uint32_t idx_mask) {
@@ -222,8 +266,9 @@ __device__ __forceinline__ uint64_t make_v(uint32_t bits, uint32_t idx, int idx_
 }
 
 struct SelResult {
-  uint64_t prefix;
+  uint64_t prefix;   // the kept candidates are those whose top `depth` bits of V are >= prefix
   int depth;
+  int kept;          // how many they are (over the whole cluster in cluster mode)
 };
 
 // Warp-inclusive scan.
@@ -236,148 +281,216 @@ __device__ __forceinline__ int warp_incl_scan(int x, int lane) {
   return x;
 }
 
-// Block-wide exclusive scan; every thread gets its offset and the total.
-template <int THREADS>
-__device__ __forceinline__ int block_excl_scan(int x, Ctl& ctl, int& total) {
-  constexpr int NW = THREADS / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = warp_incl_scan(x, lane);
-  if (lane == 31) ctl.wsum[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < NW ? ctl.wsum[lane] : 0;
-    int wi = warp_incl_scan(w, lane);
-    if (lane < NW) ctl.wsum[lane] = wi - w;
-    if (lane == 31) ctl.wsum[32] = wi;
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t y = __shfl_xor_sync(0xffffffffu, v, o);
+    v = y > v ? y : v;
   }
-  __syncthreads();
-  int res = ctl.wsum[warp] + incl - x;
-  total = ctl.wsum[32];
-  __syncthreads();
-  return res;
+  return v;
+}
+
+// Sum of per-warp values wc[0..NW) and the exclusive prefix for warp `warp`,
+// computed by every warp on its own (no barrier).
+template <int NW>
+__device__ __forceinline__ int warp_prefix_of(const int* wc, int warp, int lane, int& total) {
+  const int c = lane < NW ? wc[lane] : 0;
+  const int incl = warp_incl_scan(c, lane);
+  total = __shfl_sync(0xffffffffu, incl, 31);
+  const int mine = __shfl_sync(0xffffffffu, incl - c, warp);
+  return mine;
+}
+
+template <bool CLUSTER>
+__device__ __forceinline__ void cta_or_cluster_sync(cg::cluster_group& cluster) {
+  if (CLUSTER) cluster.sync();
+  else __syncthreads();
 }
 
 // --------------------------------------------------------------------------- //
-// MSB-first radix select over V.  Finds (prefix, depth) such that exactly `need`
-// candidates have their top `depth` bits >= prefix.  In cluster mode every CTA
-// holds part of the candidates; histograms are summed over the cluster through
-// distributed shared memory and every CTA takes the same decision.
+// MSB-first radix select over V.  Finds (prefix, depth) such that the candidates
+// whose top `depth` bits are >= prefix number at least `need` and at most
+// need + slack (exactly `need` with slack 0).  All candidates lie in [vlo, vhi],
+// so the bits those two share are skipped.  One barrier per digit: histograms
+// rotate over three buffers (build one, zero the next, the third may still be
+// read), and every warp finds the bucket on its own.  While the digit lies in
+// the key bits the arithmetic is 32-bit.  In cluster mode every CTA holds part
+// of the candidates; histograms are summed over the cluster through distributed
+// shared memory and every CTA takes the same decision.
 // --------------------------------------------------------------------------- //
 template <int DT, int THREADS, bool CLUSTER>
 __device__ SelResult radix_select(const typename Elem<DT>::bits_t* cb, const uint32_t* ci, int cnt,
-                                  int need, int idx_bits, Ctl& ctl, cg::cluster_group& cluster) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int total_bits = Elem<DT>::kKeyBits + idx_bits;
-  const uint32_t idx_mask = idx_bits >= 32 ? 0xFFFFFFFFu : ((1u << idx_bits) - 1u);
-  uint64_t prefix = 0;
-  int depth = 0;
-  int par = 0;
+                                  const int need0, int slack, int idx_bits, uint64_t vlo, uint64_t vhi,
+                                  Ctl& ctl, cg::cluster_group& cluster) {
+  using E = Elem<DT>;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int total_bits = E::kKeyBits + idx_bits;
+  const uint32_t idx_mask = mask_bits(idx_bits);
+  int depth = vlo != vhi ? total_bits - (64 - __clzll(static_cast<long long>(vlo ^ vhi))) : total_bits;
+  uint64_t prefix = depth == 0 ? 0ull : (vhi >> (total_bits - depth));
+  if (depth >= total_bits) return {vhi, total_bits, need0};
+  int need = need0;
+  int hb = ctl.hb;
+  int kept = need0;
   while (true) {
     const int dbits = min(kDigitBits, total_bits - depth);
     const int shift = total_bits - depth - dbits;
     const uint32_t dmask = (1u << dbits) - 1u;
-    int* h = ctl.hist[par];
-    for (int i = tid; i < kBins; i += THREADS) h[i] = 0;
-    __syncthreads();
-    for (int i = tid; i < cnt; i += THREADS) {
-      const uint64_t v = make_v<DT>(cb[i], ci[i], idx_bits, idx_mask);
-      if ((v >> (shift + dbits)) == prefix) atomicAdd(&h[static_cast<uint32_t>(v >> shift) & dmask], 1);
+    int* h = ctl.hist[hb];
+    int* hz = ctl.hist[hb == 2 ? 0 : hb + 1];
+    for (int i = tid; i < kBins; i += THREADS) hz[i] = 0;
+    if (shift >= idx_bits) {   // digit and prefix inside the key bits
+      const int ks = shift - idx_bits;
+      const uint32_t kp = static_cast<uint32_t>(prefix);
+      const int ps = ks + dbits;   // < 32 here
+#pragma unroll 4
+      for (int i = tid; i < cnt; i += THREADS) {
+        const uint32_t key = E::key(cb[i]);
+        if ((ps >= 32 ? 0u : (key >> ps)) == kp) atomicAdd(&h[(key >> ks) & dmask], 1);
+      }
+    } else {
+#pragma unroll 4
+      for (int i = tid; i < cnt; i += THREADS) {
+        const uint64_t v = make_v<DT>(cb[i], ci[i], idx_bits, idx_mask);
+        if ((v >> (shift + dbits)) == prefix) atomicAdd(&h[static_cast<uint32_t>(v >> shift) & dmask], 1);
+      }
     }
     const int* H = h;
+    cta_or_cluster_sync<CLUSTER>(cluster);
     if (CLUSTER) {
-      cluster.sync();
       const int nr = static_cast<int>(cluster.num_blocks());
       for (int b = tid; b < kBins; b += THREADS) {
         int s = 0;
         for (int r = 0; r < nr; ++r) s += cluster.map_shared_rank(h, r)[b];
         ctl.hsum[b] = s;
       }
+      __syncthreads();
       H = ctl.hsum;
     }
-    __syncthreads();
-    if (warp == 0) {
-      int c[kBins / 32];
-      int s = 0;
+    // every warp: bins from the top, 8 per lane, find the bucket holding the need-th
+    int c[kBins / 32];
+    int s = 0;
+#pragma unroll
+    for (int j = 0; j < kBins / 32; ++j) {
+      c[j] = H[kBins - 1 - (lane * (kBins / 32) + j)];
+      s += c[j];
+    }
+    const int incl = warp_incl_scan(s, lane);
+    const int excl = incl - s;
+    const bool mine = excl < need && need <= incl;
+    int digit = 0, above = 0, bucket = 0;
+    if (mine) {
+      int acc = excl;
+      bool done = false;
 #pragma unroll
       for (int j = 0; j < kBins / 32; ++j) {
-        c[j] = H[kBins - 1 - (lane * (kBins / 32) + j)];
-        s += c[j];
-      }
-      const int incl = warp_incl_scan(s, lane);
-      int acc = incl - s;
-      if (acc < need && need <= incl) {
-        bool done = false;
-#pragma unroll
-        for (int j = 0; j < kBins / 32; ++j) {
-          if (!done && acc + c[j] >= need) {
-            ctl.sel_digit = kBins - 1 - (lane * (kBins / 32) + j);
-            ctl.sel_above = acc;
-            ctl.sel_bucket = c[j];
-            done = true;
-          }
-          acc += c[j];
+        if (!done && acc + c[j] >= need) {
+          digit = kBins - 1 - (lane * (kBins / 32) + j);
+          above = acc;
+          bucket = c[j];
+          done = true;
         }
+        acc += c[j];
       }
     }
-    __syncthreads();
-    const int digit = ctl.sel_digit, above = ctl.sel_above, bucket = ctl.sel_bucket;
+    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    bucket = __shfl_sync(0xffffffffu, bucket, src);
     need -= above;
     prefix = (prefix << dbits) | static_cast<uint64_t>(digit);
     depth += dbits;
-    par ^= 1;
-    if (need == bucket || depth == total_bits) break;
+    hb = hb == 2 ? 0 : hb + 1;
+    kept = need0 - need + bucket;
+    if (bucket - need <= slack || depth == total_bits) break;
   }
-  return {prefix, depth};
+  if (tid == 0) ctl.hb = hb;   // read again only after later barriers
+  return {prefix, depth, kept};
 }
 
-// Keep the candidates whose top `depth` bits are >= prefix, preserving their order
-// (each thread owns a contiguous run of EPT slots).  Returns the kept count.
+// Keep the candidates whose top `depth` bits are >= prefix (`kept` of them, or
+// counted here when kept < 0), moving those found past position kept into the
+// holes below it.  Order is not preserved; positions come from per-warp counts
+// (no atomics), each warp owning a contiguous chunk.  Returns the kept count.
 template <int DT, int THREADS>
-__device__ int stable_compact(typename Elem<DT>::bits_t* cb, uint32_t* ci, int cnt, SelResult sel,
-                              int idx_bits, Ctl& ctl) {
-  using bits_t = typename Elem<DT>::bits_t;
-  constexpr int EPT = 8;
-  const int tid = threadIdx.x;
-  const int total_bits = Elem<DT>::kKeyBits + idx_bits;
-  const uint32_t idx_mask = idx_bits >= 32 ? 0xFFFFFFFFu : ((1u << idx_bits) - 1u);
-  const int sh = total_bits - sel.depth;
-  int out = 0;
-  for (int base = 0; base < cnt; base += THREADS * EPT) {
-    bits_t b[EPT];
-    uint32_t ix[EPT];
-    uint32_t km = 0;
-#pragma unroll
-    for (int e = 0; e < EPT; ++e) {
-      const int i = base + tid * EPT + e;
-      b[e] = 0;
-      ix[e] = 0;
-      if (i < cnt) {
-        b[e] = cb[i];
-        ix[e] = ci[i];
-        if ((make_v<DT>(b[e], ix[e], idx_bits, idx_mask) >> sh) >= sel.prefix) km |= 1u << e;
-      }
+__device__ int holes_compact(typename Elem<DT>::bits_t* cb, uint32_t* ci, int cnt, int kept,
+                             SelResult sel, int idx_bits, Ctl& ctl, uint32_t* holes) {
+  constexpr int NW = THREADS / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int sh = Elem<DT>::kKeyBits + idx_bits - sel.depth;
+  const uint32_t idx_mask = mask_bits(idx_bits);
+  auto keep_at = [&](int p) -> bool {
+    return (make_v<DT>(cb[p], ci[p], idx_bits, idx_mask) >> sh) >= sel.prefix;
+  };
+  if (kept < 0) {   // count first
+    const int chunk = ((cnt + NW - 1) / NW + 31) & ~31;
+    const int a = min(cnt, warp * chunk), b = min(cnt, a + chunk);
+    int n = 0;
+    for (int p0 = a; p0 < b; p0 += 32) {
+      const int p = p0 + lane;
+      n += __popc(__ballot_sync(0xffffffffu, p < b && keep_at(p)));
     }
+    if (lane == 0) ctl.wm[warp] = n;
+    __syncthreads();
     int total;
-    int pos = out + block_excl_scan<THREADS>(__popc(km), ctl, total);
-#pragma unroll
-    for (int e = 0; e < EPT; ++e) {
-      if (km & (1u << e)) {
-        cb[pos] = b[e];
-        ci[pos] = ix[e];
-        ++pos;
-      }
-    }
-    out += total;
+    warp_prefix_of<NW>(ctl.wm, warp, lane, total);
+    kept = total;
+    __syncthreads();
+  }
+  // holes live in [0, kept), movers in [kept, cnt)
+  const int hc = ((kept + NW - 1) / NW + 31) & ~31;
+  const int mc = ((cnt - kept + NW - 1) / NW + 31) & ~31;
+  const int ha = min(kept, warp * hc), hbnd = min(kept, ha + hc);
+  const int ma = kept + min(cnt - kept, warp * mc), mbnd = min(cnt, ma + mc);
+  int nh = 0, nm = 0;
+  for (int p0 = ha; p0 < hbnd; p0 += 32) {
+    const int p = p0 + lane;
+    nh += __popc(__ballot_sync(0xffffffffu, p < hbnd && !keep_at(p)));
+  }
+  for (int p0 = ma; p0 < mbnd; p0 += 32) {
+    const int p = p0 + lane;
+    nm += __popc(__ballot_sync(0xffffffffu, p < mbnd && keep_at(p)));
+  }
+  if (lane == 0) {
+    ctl.wc[0][warp] = nh;
+    ctl.wm[warp] = nm;
   }
   __syncthreads();
-  return out;
+  int tot;
+  int hoff = warp_prefix_of<NW>(ctl.wc[0], warp, lane, tot);
+  int moff = warp_prefix_of<NW>(ctl.wm, warp, lane, tot);
+  const uint32_t below = (1u << lane) - 1u;
+  for (int p0 = ha; p0 < hbnd; p0 += 32) {
+    const int p = p0 + lane;
+    const bool hole = p < hbnd && !keep_at(p);
+    const uint32_t bal = __ballot_sync(0xffffffffu, hole);
+    if (hole) holes[hoff + __popc(bal & below)] = static_cast<uint32_t>(p);
+    hoff += __popc(bal);
+  }
+  __syncthreads();
+  for (int p0 = ma; p0 < mbnd; p0 += 32) {
+    const int p = p0 + lane;
+    const bool mover = p < mbnd && keep_at(p);
+    const uint32_t bal = __ballot_sync(0xffffffffu, mover);
+    if (mover) {
+      const uint32_t q = holes[moff + __popc(bal & below)];
+      cb[q] = cb[p];
+      ci[q] = ci[p];
+    }
+    moff += __popc(bal);
+  }
+  __syncthreads();
+  return kept;
 }
 
 // Threshold word for a selection result: the smallest V with that prefix.
+__device__ __forceinline__ uint64_t v_floor(SelResult sel, int total_bits) {
+  return sel.prefix << (total_bits - sel.depth);
+}
+
 __device__ __forceinline__ unsigned long long threshold_of(SelResult sel, int key_bits, int idx_bits) {
-  const int total_bits = key_bits + idx_bits;
-  const uint32_t idx_mask = idx_bits >= 32 ? 0xFFFFFFFFu : ((1u << idx_bits) - 1u);
-  const uint64_t v = sel.prefix << (total_bits - sel.depth);
+  const uint32_t idx_mask = mask_bits(idx_bits);
+  const uint64_t v = v_floor(sel, key_bits + idx_bits);
   const uint32_t key = static_cast<uint32_t>(v >> idx_bits);
   const uint32_t rev = static_cast<uint32_t>(v) & idx_mask;
   return make_w(key, idx_mask - rev);

@@ -40,7 +40,7 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
   dsel_plan_t p{};
   p.threads = kThreads;
   p.block = kBlockElems;
-  p.round = kRoundElems;
+  p.round = round_elems(dtype);
   p.b2 = k <= 1024 ? 1024 : std::min(k, 2048);
   p.capacity = int(round_up(std::max<int64_t>(k + p.b2 + p.round, next_pow2(k)), 32));
   p.idx_bits = ceil_log2_u64(uint64_t(row_stride));
@@ -65,14 +65,14 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
   const int64_t slice = round_up(ceil_div(row_stride, groups * cluster), kStrideReq);
   const int64_t nb_max = ceil_div(slice, p.block);
   const int64_t per_round = p.round / p.block;
-  const int64_t base = stream_smem_bytes(0, p.block, p.capacity, eb) + 256;
+  const int64_t base = stream_layout(0, p.block, p.capacity, int64_t(k) + p.b2, eb).total + 256;
   const int64_t per_stage = int64_t(p.block) * eb + 8 + 4;
   int64_t stages = (int64_t(smem_optin) - base) / per_stage;
   stages = std::min<int64_t>(stages, kMaxStages);
   stages = std::min<int64_t>(stages, std::max<int64_t>(nb_max, per_round));
   stages = std::max<int64_t>(stages, per_round);
   p.stages = int(stages);
-  const int64_t smem = stream_smem_bytes(stages, p.block, p.capacity, eb);
+  const int64_t smem = stream_layout(stages, p.block, p.capacity, int64_t(k) + p.b2, eb).total;
   if (smem > smem_optin) return DSEL_ERR_K;
   p.smem_bytes = int(smem);
 

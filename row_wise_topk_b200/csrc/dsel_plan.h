@@ -10,23 +10,22 @@ namespace dsel {
 // Compile-time CTA shapes.  The streaming kernel is instantiated for exactly
 // these (dtype, threads) pairs; the planner only ever returns one of them.
 constexpr int kThreads = 512;
-constexpr int kVecBytes = 16;                 // one 128-bit load per thread per step
-constexpr int kRoundElems = 4096;             // elements filtered between buffer checks
+constexpr int kVecBytes = 16;                 // one 128-bit shared-memory load per vector
+constexpr int kVecsPerThread = 2;             // vectors each thread screens per round
 constexpr int kBlockElems = 1024;             // B: the pages' setting for k = 512
 constexpr int kStrideReq = 16;                // row_stride multiple (elements)
 constexpr int kMaxStages = 128;               // ring depth cap (one mbarrier per stage)
 constexpr int kMinSliceElems = 8192;          // smallest row share worth its own CTA
-constexpr int kSharedFixedBytes = 4096;       // scalars, histograms, scan scratch
+constexpr int kSharedFixedBytes = 6144;       // control block: scalars, histograms, scan scratch
 constexpr int kMaxK = 4096;
-constexpr int kMaxCluster = 8;               // portable cluster size
+constexpr int kMaxCluster = 8;                // portable cluster size
 constexpr int kMaxGroups = 255;               // clusters per row (merge keeps one prefix per group)
 
 inline int elem_bytes(int dtype) { return dtype == DSEL_BF16 ? 2 : 4; }
 
-// Vectors per thread per round: the round is kRoundElems for both dtypes.
-inline int vectors_per_thread(int dtype) {
-  return kRoundElems / (kThreads * (kVecBytes / elem_bytes(dtype)));
-}
+// Elements a CTA filters between two checks of the candidate buffer.
+constexpr int round_elems_for(int eb) { return kThreads * kVecsPerThread * (kVecBytes / eb); }
+inline int round_elems(int dtype) { return round_elems_for(elem_bytes(dtype)); }
 
 inline int ceil_log2_u64(uint64_t v) {   // smallest b with 2^b >= v (v >= 1)
   int b = 0;
@@ -50,12 +49,49 @@ inline int merge_cluster(const dsel_plan_t& p, int k) {
   return c;
 }
 
-// Shared-memory bytes of the streaming kernel for a plan (upper bound of the
-// device layout: ring, mbarriers, block table, candidate arrays, control block).
-inline int64_t stream_smem_bytes(int64_t stages, int64_t block, int64_t capacity, int eb) {
+// Shared-memory layout of the kernels (byte offsets from the dynamic
+// shared-memory base).  The device code receives these offsets; nothing on the
+// device recomputes them.
+struct SmemLayout {
+  uint32_t bars, blk, cb, ci, holes, ctl, total;
+};
+
+// `holes` = slots of the compaction hole list (k + B2: a compaction keeps at most k + B2/2).
+inline SmemLayout stream_layout(int64_t stages, int64_t block, int64_t capacity, int64_t holes, int eb) {
   auto up = [](int64_t v, int64_t a) { return (v + a - 1) / a * a; };
-  return up(stages * block * eb, 128) + up(stages * 8, 16) + up(stages * 4, 16) +
-         up(capacity * eb, 16) + up(capacity * 4, 16) + kSharedFixedBytes;
+  SmemLayout l{};
+  int64_t off = up(stages * block * eb, 128);
+  l.bars = uint32_t(off);
+  off += up(stages * 8, 16);
+  l.blk = uint32_t(off);
+  off += up(stages * 4, 16);
+  l.cb = uint32_t(off);
+  off += up(capacity * eb, 16);
+  l.ci = uint32_t(off);
+  off += up(capacity * 4, 16);
+  l.holes = uint32_t(off);
+  off += up(holes * 4, 16);
+  l.ctl = uint32_t(off);
+  off += kSharedFixedBytes;
+  l.total = uint32_t(off);
+  return l;
+}
+
+// Merge kernel: candidate arrays, hole list and the control block.
+inline SmemLayout merge_layout(int64_t capacity, int64_t holes, int eb) {
+  auto up = [](int64_t v, int64_t a) { return (v + a - 1) / a * a; };
+  SmemLayout l{};
+  int64_t off = 0;
+  l.cb = 0;
+  off += up(capacity * eb, 16);
+  l.ci = uint32_t(off);
+  off += up(capacity * 4, 16);
+  l.holes = uint32_t(off);
+  off += up(holes * 4, 16);
+  l.ctl = uint32_t(off);
+  off += kSharedFixedBytes;
+  l.total = uint32_t(off);
+  return l;
 }
 
 int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t num_sms,
