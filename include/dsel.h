@@ -108,6 +108,10 @@ extern "C" {
 #define DSEL_ERR_CUDA (-13)        /* a CUDA runtime call failed (launch error forwarded) */
 #define DSEL_ERR_DEVICE_TIMEOUT (-14) /* a kernel gave up a bounded wait (see dsel_device_status) */
 #define DSEL_ERR_UNAVAILABLE (-15) /* the entry point is not part of this build */
+#define DSEL_ERR_SCRATCH_LIMIT (-16) /* dsel_topk_noalloc: the call needs more than its static scratch */
+
+/* Size of the static device scratch behind dsel_topk_noalloc (512 KiB per device). */
+#define DSEL_NOALLOC_SCRATCH_BYTES (512 * 1024)
 
 /* Launch plan chosen for a call (see dsel_plan). */
 typedef struct {
@@ -141,6 +145,35 @@ DSEL_API int dsel_topk(const void* x, int dtype, int64_t rows, int64_t row_strid
                        const int32_t* end, int32_t k, int sorted_index, int return_value,
                        int index_dtype, int nan_mode, void* values_out, void* indices_out,
                        void* stream);
+
+/*
+ * dsel_topk_noalloc -- dsel_topk for callers that cannot let a library allocate
+ * device memory (for example engines that own the device heap through their own
+ * allocator and budget, hosts that forbid side allocations by plug-ins, or
+ * latency-critical loops where cudaMalloc / cudaFree, which may synchronise the
+ * device, are not acceptable).  The pages have no counterpart to this entry
+ * point; it is an interface addition of this library.
+ *
+ * Arguments, layout, results, sentinels and errors are those of dsel_topk.  The
+ * difference is the split-row workspace: instead of a lazily allocated buffer it
+ * uses a static device array of DSEL_NOALLOC_SCRATCH_BYTES that every GPU loading
+ * the library holds until the process exits.  The call never calls cudaMalloc,
+ * cudaFree or any allocating routine.
+ *   - A call whose plan needs more scratch than that returns DSEL_ERR_SCRATCH_LIMIT
+ *     and launches nothing (on a 148-SM B200 this happens only for k >= 3640, on
+ *     at most nine long rows split over several clusters).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) and sets kernel attributes; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents (no slot has to start at zero: each call writes every slot it
+ *     reads).  Calls whose work overlaps on the GPU (different streams, not
+ *     ordered) race on it: order them.
+ */
+DSEL_API int dsel_topk_noalloc(const void* x, int dtype, int64_t rows, int64_t row_stride,
+                               const int32_t* end, int32_t k, int sorted_index, int return_value,
+                               int index_dtype, int nan_mode, void* values_out, void* indices_out,
+                               void* stream);
 
 /* Row-stride requirement in elements for `dtype` (the pages' get_stride_requirement,
  * narracomm paragraph on install and switches): 16 for both dtypes, so every row

@@ -26,6 +26,8 @@ DSEL_NAN_TRAP, DSEL_NAN_FLAG = 0, 1
 DSEL_ORDER_NONE, DSEL_ORDER_INDEX, DSEL_ORDER_VALUE = 0, 1, 2
 DSEL_IDX_PAD, DSEL_IDX_NAN, DSEL_IDX_BAD_END = -1, -2, -3
 DSEL_OK = 0
+DSEL_ERR_SCRATCH_LIMIT = -16
+DSEL_NOALLOC_SCRATCH_BYTES = 512 * 1024
 
 
 class DselPlan(ctypes.Structure):
@@ -63,6 +65,8 @@ def _load() -> ctypes.CDLL:
     lib.dsel_topk.restype = c_int
     lib.dsel_topk.argtypes = [vp, c_int, c_i64, c_i64, vp, ctypes.c_int32, c_int, c_int, c_int, c_int,
                               vp, vp, vp]
+    lib.dsel_topk_noalloc.restype = c_int
+    lib.dsel_topk_noalloc.argtypes = list(lib.dsel_topk.argtypes)
     lib.dsel_stride_requirement.restype = c_i64
     lib.dsel_stride_requirement.argtypes = [c_int]
     lib.dsel_status_string.restype = ctypes.c_char_p
@@ -91,6 +95,17 @@ def dsel_topk(x: int, dtype: int, rows: int, row_stride: int, end: Optional[int]
     """Raw entry point: pointers are integers (device addresses), returns the status."""
     return lib.dsel_topk(x, dtype, rows, row_stride, end, k, sorted_index, return_value,
                          index_dtype, nan_mode, values_out, indices_out, stream)
+
+
+def dsel_topk_noalloc(x: int, dtype: int, rows: int, row_stride: int, end: Optional[int], k: int,
+                      sorted_index: int, return_value: int, index_dtype: int, nan_mode: int,
+                      values_out: Optional[int], indices_out: int, stream: Optional[int]) -> int:
+    """Raw allocation-free entry point (same arguments as dsel_topk): for callers
+    that cannot let the library allocate device memory.  Uses a static per-device
+    scratch of DSEL_NOALLOC_SCRATCH_BYTES; returns DSEL_ERR_SCRATCH_LIMIT when a
+    call needs more, and calls that overlap on the GPU must be ordered."""
+    return lib.dsel_topk_noalloc(x, dtype, rows, row_stride, end, k, sorted_index, return_value,
+                                 index_dtype, nan_mode, values_out, indices_out, stream)
 
 
 def dsel_stride_requirement(dtype: int) -> int:

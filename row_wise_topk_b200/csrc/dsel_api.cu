@@ -161,6 +161,9 @@ DSEL_API const char* dsel_status_string(int status) {
     case DSEL_ERR_CUDA: return "a CUDA runtime call failed";
     case DSEL_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
     case DSEL_ERR_UNAVAILABLE: return "not available in this build";
+    case DSEL_ERR_SCRATCH_LIMIT:
+      return "the split-row scratch this call needs exceeds the static scratch of dsel_topk_noalloc "
+             "(DSEL_NOALLOC_SCRATCH_BYTES per device)";
     default: return "unknown status";
   }
 }
@@ -245,6 +248,90 @@ DSEL_API int dsel_topk(const void* x, int dtype, int64_t rows, int64_t row_strid
     if (st != DSEL_OK) return st;
     kp.ws_pairs = static_cast<uint2*>(ws);
     kp.ws_meta = reinterpret_cast<int2*>(static_cast<char*>(ws) + rows * pl.groups * int64_t(k) * 8);
+  }
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return dtype == DSEL_BF16 ? run<DSEL_BF16>(kp, pl, rows, cs, di) : run<DSEL_F32>(kp, pl, rows, cs, di);
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of dsel_topk.
+//
+// Some callers cannot let a library allocate device memory: engines that own
+// the whole device heap through their own allocator and a fixed memory budget,
+// hosts that forbid side allocations by plug-ins, and latency-critical loops in
+// which a cudaMalloc or cudaFree (either may synchronise the device) is not
+// acceptable.  dsel_topk itself allocates only for split-row plans (one row
+// spread over several thread-block clusters), whose clusters exchange partial
+// results through a workspace.  dsel_topk_noalloc takes that workspace from
+// the static array below instead; it never calls cudaMalloc, cudaFree or any
+// allocating routine.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char dsel_noalloc_scratch[DSEL_NOALLOC_SCRATCH_BYTES];
+
+namespace dsel {
+namespace {
+void* g_noalloc_scratch_addr[64];   // device address of dsel_noalloc_scratch, per device
+}  // namespace
+}  // namespace dsel
+
+DSEL_API int dsel_topk_noalloc(const void* x, int dtype, int64_t rows, int64_t row_stride,
+                               const int32_t* end, int32_t k, int sorted_index, int return_value,
+                               int index_dtype, int nan_mode, void* values_out, void* indices_out,
+                               void* stream) {
+  int st = check_shape(dtype, rows, row_stride, k);
+  if (st != DSEL_OK) return st;
+  if (index_dtype != DSEL_I32 && index_dtype != DSEL_I64) return DSEL_ERR_INDEX_DTYPE;
+  if (nan_mode != DSEL_NAN_TRAP && nan_mode != DSEL_NAN_FLAG) return DSEL_ERR_NAN_MODE;
+  if (sorted_index < DSEL_ORDER_NONE || sorted_index > DSEL_ORDER_VALUE ||
+      (sorted_index == DSEL_ORDER_VALUE && dtype != DSEL_F32))
+    return DSEL_ERR_ORDER;
+  if (return_value != 0 && return_value != 1) return DSEL_ERR_VALUES;
+  if (rows == 0) return DSEL_OK;
+  if (x == nullptr || indices_out == nullptr) return DSEL_ERR_NULL;
+  if ((return_value != 0) != (values_out != nullptr)) return DSEL_ERR_VALUES;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) != 0) return DSEL_ERR_ALIGN;
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSEL_ERR_CUDA;
+  DevInfo* di = nullptr;
+  st = device_info(dev, &di);
+  if (st != DSEL_OK) return st;
+  dsel_plan_t pl;
+  st = make_plan(dtype, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster, &pl);
+  if (st != DSEL_OK) return st;
+
+  KParams kp = {};
+  kp.x = x;
+  kp.end = end;
+  kp.values_out = values_out;
+  kp.indices_out = indices_out;
+  kp.rows = rows;
+  kp.row_stride = row_stride;
+  kp.k = k;
+  kp.groups = pl.groups;
+  kp.b2 = pl.b2;
+  kp.stages = pl.stages;
+  kp.idx_bits = pl.idx_bits;
+  kp.order = sorted_index;
+  kp.return_value = return_value;
+  kp.index_i64 = index_dtype == DSEL_I64;
+  kp.nan_flag = nan_mode == DSEL_NAN_FLAG;
+  if (pl.groups > 1) {
+    if (pl.workspace_bytes > DSEL_NOALLOC_SCRATCH_BYTES) return DSEL_ERR_SCRATCH_LIMIT;
+    // Set-up, once per device, with that device current: host code only knows a
+    // stand-in for the array's name, so ask the runtime for its device address.
+    if (g_noalloc_scratch_addr[dev] == nullptr) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, dsel_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+        return DSEL_ERR_CUDA;
+      g_noalloc_scratch_addr[dev] = ptr;
+    }
+    // Nothing in the scratch has to start at zero: the merge launch reads only the
+    // slots the streaming launch of the same call has just written.
+    char* ws = static_cast<char*>(g_noalloc_scratch_addr[dev]);
+    kp.ws_pairs = reinterpret_cast<uint2*>(ws);
+    kp.ws_meta = reinterpret_cast<int2*>(ws + rows * pl.groups * int64_t(k) * 8);
   }
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   return dtype == DSEL_BF16 ? run<DSEL_BF16>(kp, pl, rows, cs, di) : run<DSEL_F32>(kp, pl, rows, cs, di);

@@ -30,6 +30,7 @@ namespace cg = cooperative_groups;
 namespace dsel {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // bounded waits: 2 s
+constexpr uint32_t kSuspendHintNs = 20000;          // a waiting warp sleeps (woken at completion)
 constexpr int kDigitBits = 8;
 constexpr int kBins = 1 << kDigitBits;
 
@@ -195,10 +196,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0u;
 }

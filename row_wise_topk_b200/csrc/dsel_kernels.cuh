@@ -172,7 +172,7 @@ __device__ __forceinline__ void emit_nan(const KParams& p, int64_t row, int g, b
 //   sort_mode 0: none, 1: ascending index, 2: value descending.
 // ---------------------------------------------------------------------------
 template <int DT, int THREADS>
-__device__ void finalize(const KParams& p, int64_t row, int g, typename Elem<DT>::bits_t* cb,
+__device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, typename Elem<DT>::bits_t* cb,
                          uint32_t* ci, uint32_t* holes, Ctl& ctl, cg::cluster_group& cluster,
                          int cnt, bool nan_local, uint64_t vlo, uint64_t vmax_thread,
                          bool to_workspace, int sort_mode) {
@@ -304,6 +304,156 @@ __device__ void finalize(const KParams& p, int64_t row, int g, typename Elem<DT>
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) off += __shfl_xor_sync(0xffffffffu, off, o);
   emit<DT, THREADS>(p, row, g, to_workspace, off, m, need, crank == 0, cb, ci);
+}
+
+// ---------------------------------------------------------------------------
+// Round-0 threshold seed (cold path, kept out of the per-round loop).  Builds a
+// 2048-bin histogram of the round's keys over the bits where they differ and
+// returns the lower edge of the bin holding the k-th largest: at least k of the
+// round's elements (hence of the slice) are >= it, so it is a valid starting T.
+// voff[v]: byte offset in the ring of this thread's vector v (~0u: none).
+// ---------------------------------------------------------------------------
+struct SeedOut {
+  unsigned long long t;
+  uint64_t vlo;
+  bool ok;
+};
+
+template <int DT, int THREADS, int VPT>
+__device__ __noinline__ SeedOut seed_threshold(const unsigned char* ring, const uint32_t (&voff)[VPT],
+                                               const uint32_t (&eidx)[VPT], uint32_t uhi, int k, int idx_bits,
+                                               Ctl& ctl, int* seed_hist) {
+  using E = Elem<DT>;
+  constexpr int NW = THREADS / 32;
+  constexpr int PV = E::kPerVec;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint4 val[VPT];
+#pragma unroll
+  for (int v = 0; v < VPT; ++v)
+    val[v] = voff[v] != 0xFFFFFFFFu ? *reinterpret_cast<const uint4*>(ring + voff[v]) : make_uint4(0u, 0u, 0u, 0u);
+  int nvalid = 0;
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+  for (int v = 0; v < VPT; ++v) {
+#pragma unroll
+    for (int e = 0; e < PV; ++e) {
+      const uint32_t b = vec_elem<DT>(val[v], e);
+      if (voff[v] != 0xFFFFFFFFu && eidx[v] + e < uhi && !E::is_nan(b)) {
+        const uint32_t kk = E::key(b);
+        kmin = min(kmin, kk);
+        kmax = max(kmax, kk);
+        ++nvalid;
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    nvalid += __shfl_xor_sync(0xffffffffu, nvalid, o);
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    ctl.wc[1][warp] = nvalid;
+    ctl.wv[warp] = (static_cast<unsigned long long>(kmax) << 32) | kmin;
+  }
+  __syncthreads();
+  int tot_valid;
+  warp_prefix_of<NW>(ctl.wc[1], warp, lane, tot_valid);
+  uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
+  if (lane < NW) {
+    gmin = static_cast<uint32_t>(ctl.wv[lane]);
+    gmax = static_cast<uint32_t>(ctl.wv[lane] >> 32);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, o));
+    gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
+  }
+  SeedOut out{0ull, 0ull, false};
+  if (tot_valid <= k || gmin == gmax) return out;   // uniform
+  // window: the kSeedBits bits below the leading bits shared by gmin, gmax
+  const int top = 32 - __clz(gmin ^ gmax);           // low bits in which keys differ
+  const int ws = top > kSeedBits ? top - kSeedBits : 0;
+  const uint32_t kbase = gmin & ~mask_bits(top);
+#pragma unroll
+  for (int v = 0; v < VPT; ++v) {
+#pragma unroll
+    for (int e = 0; e < PV; ++e) {
+      const uint32_t b = vec_elem<DT>(val[v], e);
+      if (voff[v] != 0xFFFFFFFFu && eidx[v] + e < uhi && !E::is_nan(b))
+        atomicAdd(&seed_hist[(E::key(b) - kbase) >> ws], 1);
+    }
+  }
+  __syncthreads();
+  // the bin holding the k-th largest: per-warp slice sums, then the slice
+  constexpr int SLICE = kSeedBins / NW;
+  constexpr int PER_LANE = SLICE / 32;
+  const int sbase = kSeedBins - (warp + 1) * SLICE;  // warp 0 sums the top slice
+  int sl = 0;
+#pragma unroll
+  for (int j = 0; j < PER_LANE; ++j) sl += seed_hist[sbase + lane * PER_LANE + j];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sl += __shfl_xor_sync(0xffffffffu, sl, o);
+  if (lane == 0) ctl.wm[warp] = sl;
+  __syncthreads();
+  const int c = lane < NW ? ctl.wm[lane] : 0;
+  const int incl = warp_incl_scan(c, lane);
+  const bool mine = (incl - c) < k && k <= incl;
+  const int slc = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+  const int need = k - __shfl_sync(0xffffffffu, incl - c, slc);
+  const int b0 = kSeedBins - (slc + 1) * SLICE;
+  int cc[PER_LANE];
+  int sm = 0;
+#pragma unroll
+  for (int j = 0; j < PER_LANE; ++j) {   // bins of that slice from its top
+    cc[j] = seed_hist[b0 + SLICE - 1 - (lane * PER_LANE + j)];
+    sm += cc[j];
+  }
+  const int inc2 = warp_incl_scan(sm, lane);
+  const bool mine2 = (inc2 - sm) < need && need <= inc2;
+  int bin = 0;
+  if (mine2) {
+    int acc = inc2 - sm;
+    bool done = false;
+#pragma unroll
+    for (int j = 0; j < PER_LANE; ++j) {
+      if (!done && acc + cc[j] >= need) {
+        bin = b0 + SLICE - 1 - (lane * PER_LANE + j);
+        done = true;
+      }
+      acc += cc[j];
+    }
+  }
+  bin = __shfl_sync(0xffffffffu, bin, __ffs(__ballot_sync(0xffffffffu, mine2)) - 1);
+  // every key >= the bin's lower edge passes, and at least k elements do
+  const uint32_t key_t = kbase + (static_cast<uint32_t>(bin) << ws);
+  out.t = make_w(key_t, 0xFFFFFFFFu);
+  out.vlo = static_cast<uint64_t>(key_t) << idx_bits;
+  out.ok = true;
+  return out;
+}
+
+// ---------------------------------------------------------------------------
+// Mid-stream compaction (cold path): cut the buffer back to between k and
+// k + slack candidates and return the new count, threshold word and lower bound.
+// ---------------------------------------------------------------------------
+struct CompactOut {
+  int cnt;
+  unsigned long long tw;
+  uint64_t vlo;
+};
+
+template <int DT, int THREADS>
+__device__ __noinline__ CompactOut compact_buffer(typename Elem<DT>::bits_t* cb, uint32_t* ci, uint32_t* holes,
+                                                  Ctl& ctl, cg::cluster_group& cluster, int cnt, int k, int slack,
+                                                  int idx_bits, uint64_t vmax, uint64_t vlo) {
+  const uint64_t vhi = cta_vmax<THREADS>(vmax, ctl);   // barrier: survivors written
+  const SelResult sel = radix_select<DT, THREADS, false>(cb, ci, cnt, k, slack, idx_bits, vlo, vhi, ctl, cluster);
+  CompactOut out;
+  out.cnt = holes_compact<DT, THREADS>(cb, ci, cnt, sel.kept, sel, idx_bits, ctl, holes);
+  out.tw = threshold_of(sel, Elem<DT>::kKeyBits, idx_bits);
+  out.vlo = v_floor(sel, Elem<DT>::kKeyBits + idx_bits);
+  return out;
 }
 
 // ---------------------------------------------------------------------------
@@ -449,9 +599,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
     }
 
     const uint32_t uhi = static_cast<uint32_t>(hi);
-    const int total_bits = E::kKeyBits + p.idx_bits;
     const uint32_t idx_mask = mask_bits(p.idx_bits);
-    const uint32_t below = (1u << lane) - 1u;
     uint64_t vmax = 0;             // largest radix word this thread appended
     uint64_t vlo = 0;              // every candidate's radix word is >= vlo
     unsigned long long t_own = 0;  // this CTA's threshold word
@@ -495,103 +643,17 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
       DSEL_TR(r, 1);
       // ---- 2. round 0: seed T from a histogram of the round's keys ----
       if (r == 0) {
-        int nvalid = 0;
-        uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+        uint32_t voff[VPT];
 #pragma unroll
-        for (int v = 0; v < VPT; ++v) {
-#pragma unroll
-          for (int e = 0; e < PV; ++e) {
-            const uint32_t b = vec_elem<DT>(val[v], e);
-            if (have[v] && eidx[v] + e < uhi && !E::is_nan(b)) {
-              const uint32_t kk = E::key(b);
-              kmin = min(kmin, kk);
-              kmax = max(kmax, kk);
-              ++nvalid;
-            }
-          }
+        for (int v = 0; v < VPT; ++v) {   // where this thread's round-0 vectors sit
+          int s0 = stg[v] - Q;
+          if (s0 < 0) s0 += D;
+          voff[v] = have[v] ? static_cast<uint32_t>(s0 * B * E::kBytes + ov[v] * 16) : 0xFFFFFFFFu;
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          nvalid += __shfl_xor_sync(0xffffffffu, nvalid, o);
-          kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-          kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-        }
-        if (lane == 0) {
-          ctl.wc[1][warp] = nvalid;
-          ctl.wv[warp] = (static_cast<unsigned long long>(kmax) << 32) | kmin;
-        }
-        __syncthreads();
-        int tot_valid;
-        warp_prefix_of<NW>(ctl.wc[1], warp, lane, tot_valid);
-        uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
-        if (lane < NW) {
-          gmin = static_cast<uint32_t>(ctl.wv[lane]);
-          gmax = static_cast<uint32_t>(ctl.wv[lane] >> 32);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, o));
-          gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
-        }
-        if (tot_valid > p.k && gmin != gmax) {   // uniform
-          // window: the kSeedBits bits below the leading bits shared by gmin, gmax
-          const int top = 32 - __clz(gmin ^ gmax);           // low bits in which keys differ
-          const int ws = top > kSeedBits ? top - kSeedBits : 0;
-          const uint32_t kbase = gmin & ~mask_bits(top);
-#pragma unroll
-          for (int v = 0; v < VPT; ++v) {
-#pragma unroll
-            for (int e = 0; e < PV; ++e) {
-              const uint32_t b = vec_elem<DT>(val[v], e);
-              if (have[v] && eidx[v] + e < uhi && !E::is_nan(b))
-                atomicAdd(&seed_hist[(E::key(b) - kbase) >> ws], 1);
-            }
-          }
-          __syncthreads();
-          // the bin holding the k-th largest: per-warp slice sums, then the slice
-          constexpr int SLICE = kSeedBins / NW;
-          constexpr int PER_LANE = SLICE / 32;
-          const int sbase = kSeedBins - (warp + 1) * SLICE;  // warp 0 sums the top slice
-          int sl = 0;
-#pragma unroll
-          for (int j = 0; j < PER_LANE; ++j) sl += seed_hist[sbase + lane * PER_LANE + j];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) sl += __shfl_xor_sync(0xffffffffu, sl, o);
-          if (lane == 0) ctl.wm[warp] = sl;
-          __syncthreads();
-          const int c = lane < NW ? ctl.wm[lane] : 0;
-          const int incl = warp_incl_scan(c, lane);
-          const bool mine = (incl - c) < p.k && p.k <= incl;
-          const int slc = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-          const int need = p.k - __shfl_sync(0xffffffffu, incl - c, slc);
-          const int b0 = kSeedBins - (slc + 1) * SLICE;
-          int cc[PER_LANE];
-          int sm = 0;
-#pragma unroll
-          for (int j = 0; j < PER_LANE; ++j) {   // bins of that slice from its top
-            cc[j] = seed_hist[b0 + SLICE - 1 - (lane * PER_LANE + j)];
-            sm += cc[j];
-          }
-          const int inc2 = warp_incl_scan(sm, lane);
-          const bool mine2 = (inc2 - sm) < need && need <= inc2;
-          int bin = 0;
-          if (mine2) {
-            int acc = inc2 - sm;
-            bool done = false;
-#pragma unroll
-            for (int j = 0; j < PER_LANE; ++j) {
-              if (!done && acc + cc[j] >= need) {
-                bin = b0 + SLICE - 1 - (lane * PER_LANE + j);
-                done = true;
-              }
-              acc += cc[j];
-            }
-          }
-          bin = __shfl_sync(0xffffffffu, bin, __ffs(__ballot_sync(0xffffffffu, mine2)) - 1);
-          // T0: every key >= the bin's lower edge passes, and at least k elements do
-          const uint32_t key_t = kbase + (static_cast<uint32_t>(bin) << ws);
-          t_own = make_w(key_t, 0xFFFFFFFFu);
-          vlo = static_cast<uint64_t>(key_t) << p.idx_bits;
+        const SeedOut so = seed_threshold<DT, THREADS, VPT>(ring, voff, eidx, uhi, p.k, p.idx_bits, ctl, seed_hist);
+        if (so.ok) {
+          t_own = so.t;
+          vlo = so.vlo;
         }
       }
 
@@ -680,13 +742,12 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
 #ifdef DSEL_STATS
         const long long sc0 = clock64();
 #endif
-        const uint64_t vhi = cta_vmax<THREADS>(vmax, ctl);   // barrier: survivors written
-        const SelResult sel = radix_select<DT, THREADS, false>(cb, ci, cnt, p.k, p.b2 / 2, p.idx_bits,
-                                                               vlo, vhi, ctl, cluster);
-        cnt = holes_compact<DT, THREADS>(cb, ci, cnt, sel.kept, sel, p.idx_bits, ctl, holes);
-        const unsigned long long tw = threshold_of(sel, E::kKeyBits, p.idx_bits);
+        const CompactOut co = compact_buffer<DT, THREADS>(cb, ci, holes, ctl, cluster, cnt, p.k, p.b2 / 2,
+                                                          p.idx_bits, vmax, vlo);
+        cnt = co.cnt;
+        const unsigned long long tw = co.tw;
         t_own = tw > t_own ? tw : t_own;
-        vlo = v_floor(sel, total_bits);
+        vlo = co.vlo;
         // any CTA's threshold is a valid bound for the whole row: push it to the peers
         if (C > 1 && warp == 0 && lane < C && lane != crank)
           atomicMax(cluster.map_shared_rank(&ctl.t_w, lane), tw);

@@ -41,7 +41,7 @@ def test_stride_requirement_and_strings():
     assert T.dsel_stride_requirement(T.DSEL_BF16) == 16
     assert T.dsel_stride_requirement(T.DSEL_F32) == 16
     assert T.dsel_stride_requirement(7) == -1
-    for code in range(0, -16, -1):
+    for code in range(0, -17, -1):
         s = T.dsel_status_string(code)
         assert s and s != "unknown status", code
     assert T.dsel_status_string(-99) == "unknown status"
