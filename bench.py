@@ -181,6 +181,12 @@ def max_over_ranks(value: float, pg, device=None) -> float:
     return float(t.item())
 
 
+def whole_job_gbs(bytes_per_step: int, steps: int, elapsed_ms: float, world: int) -> float:
+    """Whole-job effective GB/s: every rank processes its own batch of the workload
+    (weak scaling), and the slowest rank's time counts."""
+    return world * bytes_per_step * steps / (elapsed_ms / 1e3) / 1e9
+
+
 def cpu_oracle_throughput(w: W.Workload, budget_s: float):
     """Times the CPU oracle (as it stands) on whole rows of the workload until the
     budget is spent; returns (GB/s effective, rows/s, rows timed)."""
@@ -341,7 +347,7 @@ def run_ours(args, w, world, rank, local, pg):
     elapsed_ms = max_over_ranks(elapsed_ms, pg, dev)
     ms_per_step = elapsed_ms / args.steps
     eff = w.effective_bytes()
-    value = world * eff * args.steps / (elapsed_ms / 1e3) / 1e9
+    value = whole_job_gbs(eff, args.steps, elapsed_ms, world)
     rows_per_s = world * w.rows * args.steps / (elapsed_ms / 1e3)
 
     # roofline of the streaming kernel: algorithmic bytes per launch / launch time

@@ -242,6 +242,7 @@ DSEL_API int dsel_topk(const void* x, int dtype, int64_t rows, int64_t row_strid
   kp.return_value = return_value;
   kp.index_i64 = index_dtype == DSEL_I64;
   kp.nan_flag = nan_mode == DSEL_NAN_FLAG;
+  kp.capacity = pl.capacity;
   if (pl.groups > 1) {
     void* ws = nullptr;
     st = workspace(dev, stream, size_t(pl.workspace_bytes), &ws);
@@ -317,6 +318,7 @@ DSEL_API int dsel_topk_noalloc(const void* x, int dtype, int64_t rows, int64_t r
   kp.return_value = return_value;
   kp.index_i64 = index_dtype == DSEL_I64;
   kp.nan_flag = nan_mode == DSEL_NAN_FLAG;
+  kp.capacity = pl.capacity;
   if (pl.groups > 1) {
     if (pl.workspace_bytes > DSEL_NOALLOC_SCRATCH_BYTES) return DSEL_ERR_SCRATCH_LIMIT;
     // Set-up, once per device, with that device current: host code only knows a

@@ -110,6 +110,13 @@ __device__ __forceinline__ bool bf16x2_any_geu(uint32_t a, uint32_t t) {
   return r != 0u;
 }
 
+// Non-propagating maxima (a NaN operand loses to a number).
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 __device__ __forceinline__ float f32_max_nan(float a, float b) {
   float d;
   asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
@@ -173,6 +180,10 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void fence_mbar_init() {
@@ -320,7 +331,7 @@ __device__ __forceinline__ void cta_or_cluster_sync(cg::cluster_group& cluster) 
 // shared memory and every CTA takes the same decision.
 // --------------------------------------------------------------------------- //
 template <int DT, int THREADS, bool CLUSTER>
-__device__ SelResult radix_select(const typename Elem<DT>::bits_t* cb, const uint32_t* ci, int cnt,
+__device__ __noinline__ SelResult radix_select(const typename Elem<DT>::bits_t* cb, const uint32_t* ci, int cnt,
                                   const int need0, int slack, int idx_bits, uint64_t vlo, uint64_t vhi,
                                   Ctl& ctl, cg::cluster_group& cluster) {
   using E = Elem<DT>;
@@ -414,7 +425,7 @@ __device__ SelResult radix_select(const typename Elem<DT>::bits_t* cb, const uin
 // holes below it.  Order is not preserved; positions come from per-warp counts
 // (no atomics), each warp owning a contiguous chunk.  Returns the kept count.
 template <int DT, int THREADS>
-__device__ int holes_compact(typename Elem<DT>::bits_t* cb, uint32_t* ci, int cnt, int kept,
+__device__ __noinline__ int holes_compact(typename Elem<DT>::bits_t* cb, uint32_t* ci, int cnt, int kept,
                              SelResult sel, int idx_bits, Ctl& ctl, uint32_t* holes) {
   constexpr int NW = THREADS / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -500,7 +511,7 @@ __device__ __forceinline__ unsigned long long threshold_of(SelResult sel, int ke
 // Bitonic sort of m (<= capacity, padded to a power of two) candidates in shared
 // memory.  BY_VALUE: value descending, then index ascending; else index ascending.
 template <int DT, int THREADS, bool BY_VALUE>
-__device__ void bitonic_sort(typename Elem<DT>::bits_t* cb, uint32_t* ci, int m) {
+__device__ __noinline__ void bitonic_sort(typename Elem<DT>::bits_t* cb, uint32_t* ci, int m) {
   const int tid = threadIdx.x;
   int M = 1;
   while (M < m) M <<= 1;

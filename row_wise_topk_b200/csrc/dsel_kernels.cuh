@@ -27,6 +27,7 @@ struct KParams {
   int32_t index_i64;
   int32_t nan_flag;         // 1: DSEL_NAN_FLAG, 0: DSEL_NAN_TRAP
   int32_t gather;           // final phase gathers the cluster's partial results on rank 0
+  int32_t capacity;         // candidate-buffer slots
   uint32_t off_bars, off_blk, off_cb, off_ci, off_holes, off_ctl;
 };
 
@@ -121,7 +122,7 @@ __device__ __forceinline__ uint64_t cta_vmax(uint64_t vmax, Ctl& ctl) {
 // Exact selection of the `need` best candidates of this CTA's buffer (all in
 // [vlo, vhi]), moved to its front.  Returns the kept count.
 template <int DT, int THREADS>
-__device__ int local_select(typename Elem<DT>::bits_t* cb, uint32_t* ci, int cnt, int need, int idx_bits,
+__device__ __noinline__ int local_select(typename Elem<DT>::bits_t* cb, uint32_t* ci, int cnt, int need, int idx_bits,
                             uint64_t vlo, uint64_t vhi, Ctl& ctl, uint32_t* holes,
                             cg::cluster_group& cluster) {
   if (cnt <= need) return cnt;
@@ -159,6 +160,75 @@ __device__ __forceinline__ void emit_nan(const KParams& p, int64_t row, int g, b
 }
 
 // ---------------------------------------------------------------------------
+// Order the m kept entries and write them at output slots off .. off + m - 1.
+// Ascending index, when the bitmap of the candidates' index span fits in
+// `scratch` (the idle bulk-copy ring): each entry's slot is the number of kept
+// indices below it, from a prefix popcount over the bitmap.  Otherwise (and
+// for value order) a bitonic sort in shared memory, then a plain write.
+// ---------------------------------------------------------------------------
+template <int DT, int THREADS>
+__device__ __noinline__ void finish_sorted(const KParams& p, int64_t row, int g, bool to_workspace,
+                                           typename Elem<DT>::bits_t* cb, uint32_t* ci, int m, int sort_mode,
+                                           Ctl& ctl, unsigned char* scratch, uint32_t scratch_bytes,
+                                           uint32_t span_lo, uint32_t span_len, int off, int total,
+                                           bool write_meta) {
+  using bits_t = typename Elem<DT>::bits_t;
+  constexpr int NW = THREADS / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t words = (span_len + 31u) / 32u;
+  if (sort_mode == 1 && scratch != nullptr && 8ull * words <= scratch_bytes) {
+    uint32_t* bm = reinterpret_cast<uint32_t*>(scratch);
+    uint32_t* wp = bm + words;
+    for (uint32_t i = tid; i < words; i += THREADS) bm[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < m; i += THREADS) {
+      const uint32_t d = ci[i] - span_lo;
+      atomicOr(&bm[d >> 5], 1u << (d & 31u));
+    }
+    __syncthreads();
+    // prefix popcount: warp w walks its contiguous share of words, lanes side by side
+    const uint32_t per = ((words + NW - 1) / NW + 31u) & ~31u;
+    const uint32_t a = min(words, warp * per), b = min(words, a + per);
+    int sum = 0;
+    for (uint32_t w0 = a; w0 < b; w0 += 32) {
+      const uint32_t w = w0 + lane;
+      sum += __popc(w < b ? bm[w] : 0u);
+    }
+    sum = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(sum)));
+    if (lane == 0) ctl.wm[warp] = sum;
+    __syncthreads();
+    int tot;
+    int base = warp_prefix_of<NW>(ctl.wm, warp, lane, tot);
+    for (uint32_t w0 = a; w0 < b; w0 += 32) {
+      const uint32_t w = w0 + lane;
+      const int c = __popc(w < b ? bm[w] : 0u);
+      const int incl = warp_incl_scan(c, lane);
+      if (w < b) wp[w] = static_cast<uint32_t>(base + incl - c);
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    __syncthreads();
+    const int64_t obase = row * p.k + off;
+    uint2* wsd = to_workspace ? p.ws_pairs + (row * p.groups + g) * static_cast<int64_t>(p.k) + off : nullptr;
+    for (int i = tid; i < m; i += THREADS) {
+      const uint32_t idx = ci[i];
+      const uint32_t d = idx - span_lo;
+      const int rank = static_cast<int>(wp[d >> 5]) + __popc(bm[d >> 5] & ((1u << (d & 31u)) - 1u));
+      if (to_workspace) {
+        wsd[rank] = make_uint2(idx, static_cast<uint32_t>(cb[i]));
+      } else {
+        if (p.index_i64) static_cast<int64_t*>(p.indices_out)[obase + rank] = static_cast<int64_t>(idx);
+        else static_cast<int32_t*>(p.indices_out)[obase + rank] = static_cast<int32_t>(idx);
+        if (p.return_value) static_cast<bits_t*>(p.values_out)[obase + rank] = cb[i];
+      }
+    }
+    if (to_workspace && write_meta && tid == 0) p.ws_meta[row * p.groups + g] = make_int2(total, 0);
+    return;
+  }
+  sort_kept<DT, THREADS>(cb, ci, m, sort_mode);
+  emit<DT, THREADS>(p, row, g, to_workspace, off, m, total, write_meta, cb, ci);
+}
+
+// ---------------------------------------------------------------------------
 // Final phase, shared by the streaming and merge kernels.  The cluster's CTAs
 // together hold a superset of the row's (or row part's) best entries; exactly
 // min(k, total) of them are kept, optionally sorted, and written to the output
@@ -175,7 +245,8 @@ template <int DT, int THREADS>
 __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, typename Elem<DT>::bits_t* cb,
                          uint32_t* ci, uint32_t* holes, Ctl& ctl, cg::cluster_group& cluster,
                          int cnt, bool nan_local, uint64_t vlo, uint64_t vmax_thread,
-                         bool to_workspace, int sort_mode) {
+                         bool to_workspace, int sort_mode, unsigned char* ring, uint32_t ring_bytes,
+                         uint32_t span_lo, uint32_t span_len) {
   using bits_t = typename Elem<DT>::bits_t;
   const int C = static_cast<int>(cluster.num_blocks());
   const int crank = static_cast<int>(cluster.block_rank());
@@ -192,50 +263,69 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
       return;
     }
     const int m = local_select<DT, THREADS>(cb, ci, cnt, p.k, p.idx_bits, vlo, vhi, ctl, holes, cluster);
-    sort_kept<DT, THREADS>(cb, ci, m, sort_mode);
-    emit<DT, THREADS>(p, row, g, to_workspace, 0, m, m, true, cb, ci);
+    finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, m, sort_mode, ctl, ring, ring_bytes, span_lo,
+                               span_len, 0, m, true);
     return;
   }
 
   if (p.gather) {
-    const int m =
-        nan_cta ? 0 : local_select<DT, THREADS>(cb, ci, cnt, p.k, p.idx_bits, vlo, vhi, ctl, holes, cluster);
+    // exchange counts, bounds and NaN state
     if (tid == 0) {
-      ctl.x_kept = m;
+      ctl.x_cnt = cnt;
       ctl.x_nan = nan_cta ? 1 : 0;
+      ctl.x_vlo = cnt > 0 ? vlo : ~0ull;
+      ctl.x_vhi = cnt > 0 ? vhi : 0ull;
     }
     cluster.sync();
-    if (crank != 0) return;
-    int nn = lane < C ? cluster.map_shared_rank(&ctl, lane)->x_nan : 0;
-    if (__any_sync(0xffffffffu, nn != 0)) {
-      emit_nan<DT, THREADS>(p, row, g, to_workspace);
+    int tot = 0, nn = 0;
+    unsigned long long lo = ~0ull, hi = 0ull;
+    if (lane < C) {
+      Ctl* pc = cluster.map_shared_rank(&ctl, lane);
+      tot = pc->x_cnt;
+      nn = pc->x_nan;
+      lo = pc->x_vlo;
+      hi = pc->x_vhi;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      tot += __shfl_xor_sync(0xffffffffu, tot, o);
+      nn |= __shfl_xor_sync(0xffffffffu, nn, o);
+      const unsigned long long l2 = __shfl_xor_sync(0xffffffffu, lo, o);
+      const unsigned long long h2 = __shfl_xor_sync(0xffffffffu, hi, o);
+      lo = l2 < lo ? l2 : lo;
+      hi = h2 > hi ? h2 : hi;
+    }
+    if (nn) {
+      if (crank == 0) emit_nan<DT, THREADS>(p, row, g, to_workspace);
       return;
     }
-    // rank 0 appends the peers' lists after its own
-    int off = m;
-    uint64_t vmx = 0;
-    for (int i = tid; i < m; i += THREADS) {
-      const uint64_t v = make_v<DT>(cb[i], ci[i], p.idx_bits, idx_mask);
-      vmx = v > vmx ? v : vmx;
+    // the raw candidates fit rank 0's buffer: gather them as they are; otherwise
+    // every CTA keeps its own best k first
+    const bool direct = tot <= p.capacity;   // uniform over the cluster
+    int m = cnt;
+    if (!direct) {
+      m = local_select<DT, THREADS>(cb, ci, cnt, p.k, p.idx_bits, vlo, vhi, ctl, holes, cluster);
+      if (tid == 0) ctl.x_kept = m;
+      cluster.sync();
+      lo = 0ull;
     }
+    if (crank != 0) return;
+    int off = m;
     for (int r = 1; r < C; ++r) {
-      const int mr = cluster.map_shared_rank(&ctl, r)->x_kept;
+      Ctl* pr = cluster.map_shared_rank(&ctl, r);
+      const int mr = direct ? pr->x_cnt : pr->x_kept;
       const bits_t* rcb = cluster.map_shared_rank(cb, r);
       const uint32_t* rci = cluster.map_shared_rank(ci, r);
       for (int i = tid; i < mr; i += THREADS) {
-        const bits_t b = rcb[i];
-        const uint32_t ix = rci[i];
-        cb[off + i] = b;
-        ci[off + i] = ix;
-        const uint64_t v = make_v<DT>(b, ix, p.idx_bits, idx_mask);
-        vmx = v > vmx ? v : vmx;
+        cb[off + i] = rcb[i];
+        ci[off + i] = rci[i];
       }
       off += mr;
     }
-    const uint64_t ghi = cta_vmax<THREADS>(vmx, ctl);   // barrier: the gathered list is complete
-    const int mm = local_select<DT, THREADS>(cb, ci, off, p.k, p.idx_bits, 0ull, ghi, ctl, holes, cluster);
-    sort_kept<DT, THREADS>(cb, ci, mm, sort_mode);
-    emit<DT, THREADS>(p, row, g, to_workspace, 0, mm, mm, true, cb, ci);
+    __syncthreads();   // the gathered list is complete
+    const int mm = local_select<DT, THREADS>(cb, ci, off, p.k, p.idx_bits, lo, hi, ctl, holes, cluster);
+    finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, mm, sort_mode, ctl, ring, ring_bytes, span_lo,
+                               span_len, 0, mm, true);
     return;
   }
 
@@ -278,7 +368,6 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
         radix_select<DT, THREADS, true>(cb, ci, cnt, need, 0, p.idx_bits, lo, hi, ctl, cluster);
     m = holes_compact<DT, THREADS>(cb, ci, cnt, -1, sel, p.idx_bits, ctl, holes);
   }
-  if (sort_mode == 1) bitonic_sort<DT, THREADS, false>(cb, ci, m);
   if (tid == 0) ctl.x_kept = m;
   cluster.sync();
   if (sort_mode == 2) {   // gather the winners on rank 0 and sort them by value
@@ -295,23 +384,48 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
         off += mr;
       }
       __syncthreads();
-      bitonic_sort<DT, THREADS, true>(cb, ci, off);
-      emit<DT, THREADS>(p, row, g, to_workspace, 0, off, off, true, cb, ci);
+      finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, off, 2, ctl, nullptr, 0u, 0u, 0u, 0, off, true);
     }
     return;
   }
   int off = lane < crank ? cluster.map_shared_rank(&ctl, lane)->x_kept : 0;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) off += __shfl_xor_sync(0xffffffffu, off, o);
-  emit<DT, THREADS>(p, row, g, to_workspace, off, m, need, crank == 0, cb, ci);
+  // each CTA orders its own share (its slice is an index range of its own)
+  finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, m, sort_mode, ctl, ring, ring_bytes, span_lo,
+                             span_len, off, need, crank == 0);
 }
 
 // ---------------------------------------------------------------------------
-// Round-0 threshold seed (cold path, kept out of the per-round loop).  Builds a
-// 2048-bin histogram of the round's keys over the bits where they differ and
-// returns the lower edge of the bin holding the k-th largest: at least k of the
-// round's elements (hence of the slice) are >= it, so it is a valid starting T.
-// voff[v]: byte offset in the ring of this thread's vector v (~0u: none).
+// Where this thread's vectors sit in the current round.  A warp owns whole
+// blocks (BPW <= 2 of them); vector v of lane l is 16-byte slot (v*32 + l) % VPB
+// of owned block (v*32) / VPB.
+// ---------------------------------------------------------------------------
+template <int DT>
+struct WarpRound {
+  int j0, nb, D, s0, lane;
+  uint32_t boff0, boff1;   // first element (in the row) of the warp's owned blocks
+  uint32_t uhi;            // end of this CTA's slice
+  template <int VPB>
+  __device__ __forceinline__ bool locate(int v, uint32_t& voff, uint32_t& eidx) const {
+    const int qb = (v * 32) / VPB;
+    if (j0 + qb >= nb) return false;
+    const int o = (v * 32 + lane) % VPB;
+    eidx = (qb ? boff1 : boff0) + static_cast<uint32_t>(o * Elem<DT>::kPerVec);
+    if (eidx >= uhi) return false;
+    int st = s0 + qb;
+    if (st >= D) st -= D;
+    voff = static_cast<uint32_t>(st * kBlockElems * Elem<DT>::kBytes + o * 16);
+    return true;
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Round-0 threshold seed (cold path, kept out of the per-round loop).  A
+// histogram of the round's keys over the bits where they differ, refined once
+// inside the chosen bin, gives the lower edge of a bin holding the k-th largest
+// key: at least k of the round's elements (hence of the slice) are >= it, so it
+// is a valid starting T.
 // ---------------------------------------------------------------------------
 struct SeedOut {
   unsigned long long t;
@@ -320,25 +434,25 @@ struct SeedOut {
 };
 
 template <int DT, int THREADS, int VPT>
-__device__ __noinline__ SeedOut seed_threshold(const unsigned char* ring, const uint32_t (&voff)[VPT],
-                                               const uint32_t (&eidx)[VPT], uint32_t uhi, int k, int idx_bits,
+__device__ __noinline__ SeedOut seed_threshold(const unsigned char* ring, WarpRound<DT> wr, int k, int idx_bits,
                                                Ctl& ctl, int* seed_hist) {
   using E = Elem<DT>;
   constexpr int NW = THREADS / 32;
   constexpr int PV = E::kPerVec;
+  constexpr int VPB = kBlockElems / PV;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint4 val[VPT];
-#pragma unroll
-  for (int v = 0; v < VPT; ++v)
-    val[v] = voff[v] != 0xFFFFFFFFu ? *reinterpret_cast<const uint4*>(ring + voff[v]) : make_uint4(0u, 0u, 0u, 0u);
+  const uint32_t uhi = wr.uhi;
   int nvalid = 0;
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-#pragma unroll
+#pragma unroll 1
   for (int v = 0; v < VPT; ++v) {
+    uint32_t voff, eidx;
+    if (!wr.template locate<VPB>(v, voff, eidx)) continue;
+    const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
 #pragma unroll
     for (int e = 0; e < PV; ++e) {
-      const uint32_t b = vec_elem<DT>(val[v], e);
-      if (voff[v] != 0xFFFFFFFFu && eidx[v] + e < uhi && !E::is_nan(b)) {
+      const uint32_t b = vec_elem<DT>(val, e);
+      if (eidx + e < uhi && !E::is_nan(b)) {
         const uint32_t kk = E::key(b);
         kmin = min(kmin, kk);
         kmax = max(kmax, kk);
@@ -353,12 +467,12 @@ __device__ __noinline__ SeedOut seed_threshold(const unsigned char* ring, const 
     kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
   }
   if (lane == 0) {
-    ctl.wc[1][warp] = nvalid;
+    ctl.wm[warp] = nvalid;
     ctl.wv[warp] = (static_cast<unsigned long long>(kmax) << 32) | kmin;
   }
   __syncthreads();
   int tot_valid;
-  warp_prefix_of<NW>(ctl.wc[1], warp, lane, tot_valid);
+  warp_prefix_of<NW>(ctl.wm, warp, lane, tot_valid);
   uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
   if (lane < NW) {
     gmin = static_cast<uint32_t>(ctl.wv[lane]);
@@ -371,65 +485,188 @@ __device__ __noinline__ SeedOut seed_threshold(const unsigned char* ring, const 
   }
   SeedOut out{0ull, 0ull, false};
   if (tot_valid <= k || gmin == gmax) return out;   // uniform
-  // window: the kSeedBits bits below the leading bits shared by gmin, gmax
+  // Level 1: the kSeedBits bits below the leading bits shared by gmin and gmax.
+  // Level 2 (when bits remain): the next kSeedBits bits, inside level 1's bin.
   const int top = 32 - __clz(gmin ^ gmax);           // low bits in which keys differ
-  const int ws = top > kSeedBits ? top - kSeedBits : 0;
-  const uint32_t kbase = gmin & ~mask_bits(top);
-#pragma unroll
-  for (int v = 0; v < VPT; ++v) {
-#pragma unroll
-    for (int e = 0; e < PV; ++e) {
-      const uint32_t b = vec_elem<DT>(val[v], e);
-      if (voff[v] != 0xFFFFFFFFu && eidx[v] + e < uhi && !E::is_nan(b))
-        atomicAdd(&seed_hist[(E::key(b) - kbase) >> ws], 1);
-    }
-  }
-  __syncthreads();
-  // the bin holding the k-th largest: per-warp slice sums, then the slice
+  uint32_t kbase = gmin & ~mask_bits(top);            // keys in the current bin share these bits
+  int width = top;                                    // bits below kbase that still vary
+  int need = k;
   constexpr int SLICE = kSeedBins / NW;
   constexpr int PER_LANE = SLICE / 32;
-  const int sbase = kSeedBins - (warp + 1) * SLICE;  // warp 0 sums the top slice
-  int sl = 0;
+  for (int level = 0; level < 2; ++level) {           // uniform
+    int* hist = seed_hist + level * kSeedBins;
+    const int ws = width > kSeedBits ? width - kSeedBits : 0;
+#pragma unroll 1
+    for (int v = 0; v < VPT; ++v) {
+      uint32_t voff, eidx;
+      if (!wr.template locate<VPB>(v, voff, eidx)) continue;
+      const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
 #pragma unroll
-  for (int j = 0; j < PER_LANE; ++j) sl += seed_hist[sbase + lane * PER_LANE + j];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sl += __shfl_xor_sync(0xffffffffu, sl, o);
-  if (lane == 0) ctl.wm[warp] = sl;
-  __syncthreads();
-  const int c = lane < NW ? ctl.wm[lane] : 0;
-  const int incl = warp_incl_scan(c, lane);
-  const bool mine = (incl - c) < k && k <= incl;
-  const int slc = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-  const int need = k - __shfl_sync(0xffffffffu, incl - c, slc);
-  const int b0 = kSeedBins - (slc + 1) * SLICE;
-  int cc[PER_LANE];
-  int sm = 0;
-#pragma unroll
-  for (int j = 0; j < PER_LANE; ++j) {   // bins of that slice from its top
-    cc[j] = seed_hist[b0 + SLICE - 1 - (lane * PER_LANE + j)];
-    sm += cc[j];
-  }
-  const int inc2 = warp_incl_scan(sm, lane);
-  const bool mine2 = (inc2 - sm) < need && need <= inc2;
-  int bin = 0;
-  if (mine2) {
-    int acc = inc2 - sm;
-    bool done = false;
-#pragma unroll
-    for (int j = 0; j < PER_LANE; ++j) {
-      if (!done && acc + cc[j] >= need) {
-        bin = b0 + SLICE - 1 - (lane * PER_LANE + j);
-        done = true;
+      for (int e = 0; e < PV; ++e) {
+        const uint32_t b = vec_elem<DT>(val, e);
+        if (eidx + e < uhi && !E::is_nan(b)) {
+          const uint32_t d = E::key(b) - kbase;
+          if ((width >= 32) || d < (1u << width)) atomicAdd(&hist[d >> ws], 1);
+        }
       }
-      acc += cc[j];
+    }
+    __syncthreads();   // histogram complete; every warp is past its reads of wm
+    // the bin holding the need-th largest: per-warp slice sums, then the slice
+    const int sbase = kSeedBins - (warp + 1) * SLICE;  // warp 0 sums the top slice
+    int sl = 0;
+#pragma unroll
+    for (int j = 0; j < PER_LANE; ++j) sl += hist[sbase + lane * PER_LANE + j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sl += __shfl_xor_sync(0xffffffffu, sl, o);
+    if (lane == 0) ctl.wm[warp] = sl;
+    __syncthreads();
+    const int c = lane < NW ? ctl.wm[lane] : 0;
+    const int incl = warp_incl_scan(c, lane);
+    const bool mine = (incl - c) < need && need <= incl;
+    const int slc = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    need -= __shfl_sync(0xffffffffu, incl - c, slc);
+    const int b0 = kSeedBins - (slc + 1) * SLICE;
+    int cc[PER_LANE];
+    int sm = 0;
+#pragma unroll
+    for (int j = 0; j < PER_LANE; ++j) {   // bins of that slice from its top
+      cc[j] = hist[b0 + SLICE - 1 - (lane * PER_LANE + j)];
+      sm += cc[j];
+    }
+    const int inc2 = warp_incl_scan(sm, lane);
+    const bool mine2 = (inc2 - sm) < need && need <= inc2;
+    int bin = 0, above = 0;
+    if (mine2) {
+      int acc = inc2 - sm;
+      bool done = false;
+#pragma unroll
+      for (int j = 0; j < PER_LANE; ++j) {
+        if (!done && acc + cc[j] >= need) {
+          bin = b0 + SLICE - 1 - (lane * PER_LANE + j);
+          above = acc;
+          done = true;
+        }
+        acc += cc[j];
+      }
+    }
+    const int src2 = __ffs(__ballot_sync(0xffffffffu, mine2)) - 1;
+    bin = __shfl_sync(0xffffffffu, bin, src2);
+    need -= __shfl_sync(0xffffffffu, above, src2);
+    kbase += static_cast<uint32_t>(bin) << ws;
+    width = ws;
+    if (ws == 0) break;
+    __syncthreads();   // all warps have read wm before the next level writes it
+  }
+  // every key >= the final bin's lower edge passes, and at least k elements do
+  out.t = make_w(kbase, 0xFFFFFFFFu);
+  out.vlo = static_cast<uint64_t>(kbase) << idx_bits;
+  out.ok = true;
+  return out;
+}
+
+// ---------------------------------------------------------------------------
+// Cheap round-0 seed for k <= 4 * THREADS: the maximum of every full 16-byte
+// vector of the round (NaN-ignoring), then the k-th largest of those maxima by
+// a radix select over their keys.  Each maximum is a real element, so at least
+// k elements are >= the result: a valid starting T.  A vector that is partial
+// (past the slice end) or whose maximum is NaN counts as empty (key 0, below
+// every number).
+// ---------------------------------------------------------------------------
+template <int DT, int THREADS, int VPT>
+__device__ __noinline__ SeedOut seed_by_vector_max(const unsigned char* ring, WarpRound<DT> wr, int k, int idx_bits,
+                                                   Ctl& ctl) {
+  using E = Elem<DT>;
+  constexpr int NW = THREADS / 32;
+  constexpr int PV = E::kPerVec;
+  constexpr int VPB = kBlockElems / PV;
+  const int tid = threadIdx.x, lane = tid & 31;
+  uint32_t gk[VPT];
+#pragma unroll
+  for (int v = 0; v < VPT; ++v) {
+    gk[v] = 0u;
+    uint32_t voff, eidx;
+    if (wr.template locate<VPB>(v, voff, eidx) && eidx + PV <= wr.uhi) {
+      const uint4 x = *reinterpret_cast<const uint4*>(ring + voff);
+      uint32_t mb;
+      if (DT == DSEL_BF16) {
+        const uint32_t m2 = bf16x2_max(bf16x2_max(x.x, x.y), bf16x2_max(x.z, x.w));
+        const uint32_t lo = m2 & 0xFFFFu, hi = m2 >> 16;
+        const uint32_t klo = E::is_nan(lo) ? 0u : E::key(lo), khi = E::is_nan(hi) ? 0u : E::key(hi);
+        gk[v] = klo > khi ? klo : khi;
+        (void)mb;
+      } else {
+        const float m = fmaxf(fmaxf(__uint_as_float(x.x), __uint_as_float(x.y)),
+                              fmaxf(__uint_as_float(x.z), __uint_as_float(x.w)));
+        mb = __float_as_uint(m);
+        gk[v] = E::is_nan(mb) ? 0u : E::key(mb);
+      }
     }
   }
-  bin = __shfl_sync(0xffffffffu, bin, __ffs(__ballot_sync(0xffffffffu, mine2)) - 1);
-  // every key >= the bin's lower edge passes, and at least k elements do
-  const uint32_t key_t = kbase + (static_cast<uint32_t>(bin) << ws);
-  out.t = make_w(key_t, 0xFFFFFFFFu);
+  // k-th largest of the THREADS * VPT maxima: 8-bit digits from the top of the key
+  int need = k;
+  uint32_t prefix = 0;
+  int depth = 0;
+  int* h = ctl.hist[0];
+  for (int i = tid; i < kBins; i += THREADS) h[i] = 0;
+  __syncthreads();
+  while (true) {   // uniform
+    const int sh = E::kKeyBits - depth - kDigitBits;
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) {
+      const uint32_t top = (depth == 0) ? 0u : (gk[v] >> (sh + kDigitBits));
+      if (top == prefix) atomicAdd(&h[(gk[v] >> sh) & (kBins - 1)], 1);
+    }
+    __syncthreads();
+    int c[kBins / 32];
+    int s = 0;
+#pragma unroll
+    for (int j = 0; j < kBins / 32; ++j) {
+      c[j] = h[kBins - 1 - (lane * (kBins / 32) + j)];
+      s += c[j];
+    }
+    const int incl = warp_incl_scan(s, lane);
+    const bool mine = (incl - s) < need && need <= incl;
+    const unsigned bal = __ballot_sync(0xffffffffu, mine);
+    int digit = 0, above = 0, bucket = 0;
+    if (mine) {
+      int acc = incl - s;
+      bool done = false;
+#pragma unroll
+      for (int j = 0; j < kBins / 32; ++j) {
+        if (!done && acc + c[j] >= need) {
+          digit = kBins - 1 - (lane * (kBins / 32) + j);
+          above = acc;
+          bucket = c[j];
+          done = true;
+        }
+        acc += c[j];
+      }
+    }
+    __syncthreads();   // every warp has read the histogram
+    if (bal == 0u) {   // fewer than k maxima (uniform); leave the histogram zeroed
+      for (int i = tid; i < kBins; i += THREADS) h[i] = 0;
+      return SeedOut{0ull, 0ull, false};
+    }
+    const int src = __ffs(bal) - 1;
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    bucket = __shfl_sync(0xffffffffu, bucket, src);
+    need -= above;
+    prefix = (prefix << kDigitBits) | static_cast<uint32_t>(digit);
+    depth += kDigitBits;
+    if (need == bucket || depth == E::kKeyBits) break;
+    for (int i = tid; i < kBins; i += THREADS) h[i] = 0;
+    __syncthreads();
+  }
+  const uint32_t key_t = depth >= E::kKeyBits ? prefix : (prefix << (E::kKeyBits - depth));
+  if (key_t == 0u) return SeedOut{0ull, 0ull, false};   // the k-th maximum is an empty vector
+  for (int i = tid; i < kBins; i += THREADS) h[i] = 0;   // the histograms start zeroed elsewhere
+  __syncthreads();
+  SeedOut out;
+  out.t = make_w(key_t, 0xFFFFFFFFu);   // passes every key >= key_t
   out.vlo = static_cast<uint64_t>(key_t) << idx_bits;
   out.ok = true;
+  (void)NW;
   return out;
 }
 
@@ -478,7 +715,10 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
   constexpr int VPT = R / (THREADS * PV);              // vectors per thread per round
   static_assert(VPB % 32 == 0, "a warp must stay inside one block");
   static_assert(VPT >= 1 && VPT * THREADS * PV == R && Q * B == R, "round shape");
-  static_assert(Q <= NW, "one refill per warp");
+  constexpr int VPW = 32 * VPT;                        // vectors per warp per round
+  static_assert(VPW % VPB == 0 || VPB % VPW == 0, "warps own whole blocks or whole warps share one");
+  static_assert(VPW >= VPB, "a warp owns whole blocks, so only it reads and refills their stages");
+  constexpr int BPW = VPW / VPB;                       // blocks owned by a warp per round
   static_assert(kSeedBins % (NW * 32) == 0, "seed histogram split");
 
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -517,7 +757,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
   const int64_t n = row_length(p, row, &bad_end);
 
   for (int i = tid; i < 3 * kBins; i += THREADS) (&ctl.hist[0][0])[i] = 0;
-  for (int i = tid; i < kSeedBins; i += THREADS) seed_hist[i] = 0;
+  for (int i = tid; i < 2 * kSeedBins; i += THREADS) seed_hist[i] = 0;   // two histogram levels
   if (tid == 0) {
     ctl.t_w = 0ull;
     ctl.nan_found = 0;
@@ -586,171 +826,219 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
     }
     DSEL_EV(1);
 
-    // per-slot state: which block of the round, which vector in it, ring stage/phase
-    int qv[VPT], ov[VPT], stg[VPT];
-    uint32_t phs[VPT];
-#pragma unroll
-    for (int v = 0; v < VPT; ++v) {
-      const int u = v * THREADS + tid;
-      qv[v] = u / VPB;
-      ov[v] = u % VPB;
-      stg[v] = qv[v];   // q < Q <= D
-      phs[v] = 0;
-    }
-
     const uint32_t uhi = static_cast<uint32_t>(hi);
     const uint32_t idx_mask = mask_bits(p.idx_bits);
-    uint64_t vmax = 0;             // largest radix word this thread appended
+    const int cap = p.capacity;
+    uint64_t vmax = 0;             // largest radix word this thread kept
     uint64_t vlo = 0;              // every candidate's radix word is >= vlo
     unsigned long long t_own = 0;  // this CTA's threshold word
     int cnt = 0;                   // candidates in the buffer (same value in every thread)
+    int par = 0;                   // which of the two per-warp count arrays is next
     bool nan_thread = false;
+    // cut the buffer back to k..k+slack, raise T and tell the peers (all threads)
+    auto compact = [&](int slack) {
+      const CompactOut co = compact_buffer<DT, THREADS>(cb, ci, holes, ctl, cluster, cnt, p.k, slack, p.idx_bits,
+                                                        vmax, vlo);
+      cnt = co.cnt;
+      t_own = co.tw > t_own ? co.tw : t_own;
+      vlo = co.vlo;
+      // any CTA's threshold is a valid bound for the whole row: push it to the peers
+      if (C > 1 && warp == 0 && lane < C && lane != crank) atomicMax(cluster.map_shared_rank(&ctl.t_w, lane), co.tw);
+    };
+    static_assert(VPT * PV <= 64, "keep bits fit one 64-bit word");
     const int rounds = (nb + Q - 1) / Q;
     for (int r = 0; r < rounds; ++r) {
       DSEL_TR(r, 0);
-      // ---- 1. wait for and load this round's vectors ----
-      uint4 val[VPT];
-      uint32_t eidx[VPT];
-      bool have[VPT];
+      WarpRound<DT> wr;
+      wr.j0 = r * Q + (warp * VPW) / VPB;              // first block this warp owns in the round
+      wr.nb = nb;
+      wr.D = D;
+      wr.s0 = wr.j0 % D;
+      wr.lane = lane;
+      wr.uhi = uhi;
+      wr.boff0 = wr.boff1 = 0;
+      const int j0 = wr.j0;
+      // ---- 1. wait for the owned blocks, then load and screen every vector ----
 #pragma unroll
-      for (int v = 0; v < VPT; ++v) {
-        const int j = r * Q + qv[v];
-        val[v] = make_uint4(0u, 0u, 0u, 0u);
-        eidx[v] = 0;
-        have[v] = false;
-        if (j < nb) {   // warp-uniform
-          const int s = stg[v];
+      for (int qb = 0; qb < BPW; ++qb) {
+        if (j0 + qb < nb) {   // warp-uniform
+          int st = wr.s0 + qb;
+          if (st >= D) st -= D;
 #ifdef DSEL_STATS
           const long long w0 = clock64();
 #endif
-          if (!mbar_wait(smem_u32(&bars[s]), phs[v])) ctl.abort = 1;
+          if (!mbar_wait(smem_u32(&bars[st]), static_cast<uint32_t>(((j0 + qb) / D) & 1))) ctl.abort = 1;
 #ifdef DSEL_STATS
           st_wait += clock64() - w0;
 #endif
-          eidx[v] = blk_off[s] + static_cast<uint32_t>(ov[v] * PV);
-          if (eidx[v] < uhi) {
-            have[v] = true;
-            val[v] = *reinterpret_cast<const uint4*>(ring + static_cast<size_t>(s) * B * E::kBytes + ov[v] * 16);
-          }
-        }
-        stg[v] += Q;
-        if (stg[v] >= D) {
-          stg[v] -= D;
-          phs[v] ^= 1u;
+          if (qb == 0) wr.boff0 = blk_off[st];
+          else wr.boff1 = blk_off[st];
         }
       }
-
+      unsigned long long w = *reinterpret_cast<volatile unsigned long long*>(&ctl.t_w);
+      w = w > t_own ? w : t_own;   // a peer may have raised it
+      uint32_t tk = static_cast<uint32_t>(w >> 32);
+      uint32_t ti = ~static_cast<uint32_t>(w);
+      uint32_t tv = E::bits_of_key(tk);
+      if (DT == DSEL_BF16) tv |= tv << 16;
+      uint32_t maybe_mask = 0;
+#pragma unroll
+      for (int v = 0; v < VPT; ++v) {
+        uint32_t voff, eidx;
+        if (wr.template locate<VPB>(v, voff, eidx)) {
+          const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
+          if ((eidx + PV > uhi) || screen<DT>(val, tv)) maybe_mask |= 1u << v;
+        }
+      }
       DSEL_TR(r, 1);
+
       // ---- 2. round 0: seed T from a histogram of the round's keys ----
       if (r == 0) {
-        uint32_t voff[VPT];
-#pragma unroll
-        for (int v = 0; v < VPT; ++v) {   // where this thread's round-0 vectors sit
-          int s0 = stg[v] - Q;
-          if (s0 < 0) s0 += D;
-          voff[v] = have[v] ? static_cast<uint32_t>(s0 * B * E::kBytes + ov[v] * 16) : 0xFFFFFFFFu;
-        }
-        const SeedOut so = seed_threshold<DT, THREADS, VPT>(ring, voff, eidx, uhi, p.k, p.idx_bits, ctl, seed_hist);
+        const SeedOut so = p.k <= 4 * THREADS
+                               ? seed_by_vector_max<DT, THREADS, VPT>(ring, wr, p.k, p.idx_bits, ctl)
+                               : seed_threshold<DT, THREADS, VPT>(ring, wr, p.k, p.idx_bits, ctl, seed_hist);
         if (so.ok) {
           t_own = so.t;
           vlo = so.vlo;
+          if (so.t > w) {   // re-screen against the seeded T (flags only shrink)
+            w = so.t;
+            tk = static_cast<uint32_t>(w >> 32);
+            ti = ~static_cast<uint32_t>(w);
+            tv = E::bits_of_key(tk);
+            if (DT == DSEL_BF16) tv |= tv << 16;
+            uint32_t mm = maybe_mask, kept_flags = 0;
+            while (mm) {
+              const int v = __ffs(mm) - 1;
+              mm &= mm - 1u;
+              uint32_t voff, eidx;
+              wr.template locate<VPB>(v, voff, eidx);
+              const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
+              if ((eidx + PV > uhi) || screen<DT>(val, tv)) kept_flags |= 1u << v;
+            }
+            maybe_mask = kept_flags;
+          }
         }
       }
 
-      // ---- 3. screen + exact test against T; per-warp survivor counts ----
-      const unsigned long long tp = *reinterpret_cast<volatile unsigned long long*>(&ctl.t_w);
-      const unsigned long long w = tp > t_own ? tp : t_own;   // a peer may have raised it
-      const uint32_t tk = static_cast<uint32_t>(w >> 32);
-      const uint32_t ti = ~static_cast<uint32_t>(w);
-      uint32_t tv = E::bits_of_key(tk);
-      if (DT == DSEL_BF16) tv |= tv << 16;
-      uint32_t keep[VPT];
-      int mine = 0;   // survivors of this thread in this round
-#pragma unroll
-      for (int v = 0; v < VPT; ++v) {
-        keep[v] = 0;
-        const bool tail = have[v] && (eidx[v] + PV > uhi);
-        const bool maybe = have[v] && (tail || screen<DT>(val[v], tv));
-        if (__any_sync(0xffffffffu, maybe)) {   // warp-uniform
+      // ---- 3. exact test of the flagged vectors (rare once T has settled) ----
+      uint64_t keepbits = 0;   // bit v*PV + e: element e of vector v survives
+      if (__any_sync(0xffffffffu, maybe_mask != 0u)) {
 #ifdef DSEL_STATS
-          if (lane == 0) atomicAdd(&ctl.st_slow_vectors, 1);
+        if (lane == 0) atomicAdd(&ctl.st_slow_vectors, __popc(maybe_mask));
 #endif
-          uint32_t cm = maybe ? candidate_mask<DT>(val[v], tv) : 0u;
-          if (tail) cm &= (1u << (uhi - eidx[v])) - 1u;   // elements at or past hi are not this row's
-          while (cm) {   // exact test, only for the elements the float compare let through
+        uint32_t mm = maybe_mask;
+        while (mm) {
+          const int v = __ffs(mm) - 1;
+          mm &= mm - 1u;
+          uint32_t voff, eidx;
+          wr.template locate<VPB>(v, voff, eidx);
+          const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
+          uint32_t cm = candidate_mask<DT>(val, tv);
+          if (eidx + PV > uhi) cm &= (1u << (uhi - eidx)) - 1u;   // past hi: not this row's
+          while (cm) {
             const int e = __ffs(cm) - 1;
             cm &= cm - 1u;
-            const uint32_t b = vec_elem_dyn<DT>(val[v], e);
-            const uint32_t idx = eidx[v] + e;
+            const uint32_t b = vec_elem_dyn<DT>(val, e);
+            const uint32_t idx = eidx + e;
             if (E::is_nan(b)) {
               if (!p.nan_flag) nan_trap();   // the pages' default policy: abort on NaN
               nan_thread = true;
             } else {
               const uint32_t kk = E::key(b);
               if (kk > tk || (kk == tk && idx < ti)) {
-                keep[v] |= 1u << e;
+                keepbits |= 1ull << (v * PV + e);
                 const uint64_t vv = (static_cast<uint64_t>(kk) << p.idx_bits) | (idx_mask - idx);
                 vmax = vv > vmax ? vv : vmax;
               }
             }
           }
-          mine += __popc(keep[v]);
         }
       }
-      const int wcount = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(mine)));
-      if (lane == 0) ctl.wc[r & 1][warp] = wcount;
+      int mine = __popcll(keepbits);   // survivors of this thread not yet in the buffer
       if (r == 0) DSEL_EV(2);
       DSEL_TR(r, 2);
-      __syncthreads();
-      DSEL_TR(r, 3);
-      if (r == 0) DSEL_EV(3);
-      // refill the stages this round consumed: warp q issues block r*Q + q + D
-      if (warp < Q && lane == 0) {
-        const int j = r * Q + warp + D;
-        if (j < nb) issue(j);
-      }
-      // ---- 4. write survivors at offsets from the per-warp counts ----
-      int total;
-      const int woff = cnt + warp_prefix_of<NW>(ctl.wc[r & 1], warp, lane, total);
-      DSEL_TR(r, 6);
-#ifdef DSEL_STATS
-      if (tr_w >= 0 && r < kTraceRounds) g_trace[(tr_w * kTraceRounds + r) * kTraceEvents + 7] = wcount;
-#endif
-      if (wcount != 0) {   // warp-uniform
-        const int incl = warp_incl_scan(mine, lane);
-        int pos = woff + incl - mine;
-#pragma unroll
-        for (int v = 0; v < VPT; ++v) {
-          uint32_t km = keep[v];
-          while (km) {
-            const int e = __ffs(km) - 1;
-            km &= km - 1u;
-            cb[pos] = static_cast<bits_t>(vec_elem_dyn<DT>(val[v], e));
-            ci[pos] = eidx[v] + e;
-            ++pos;
+
+      // ---- 4. append at offsets from per-warp counts; what does not fit waits ----
+      bool first = true;
+      while (true) {   // uniform: every thread takes the same path
+        const int wcount = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(mine)));
+        if (lane == 0) ctl.wc[par][warp] = wcount;
+        __syncthreads();
+        if (first) {
+          DSEL_TR(r, 3);
+          if (r == 0) DSEL_EV(3);
+          first = false;
+        }
+        int total;
+        const int woff = warp_prefix_of<NW>(ctl.wc[par], warp, lane, total);
+        par ^= 1;
+        const int space = cap - cnt;
+        DSEL_TR(r, 6);
+        if (wcount != 0) {   // warp-uniform
+          int rank = woff + warp_incl_scan(mine, lane) - mine;
+          uint64_t kb = keepbits;
+          while (kb) {
+            const int bit = __ffsll(static_cast<long long>(kb)) - 1;
+            kb &= kb - 1ull;
+            if (rank < space) {
+              const int v = bit / PV, e = bit % PV;
+              uint32_t voff, eidx;
+              wr.template locate<VPB>(v, voff, eidx);
+              const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
+              cb[cnt + rank] = static_cast<bits_t>(vec_elem_dyn<DT>(val, e));
+              ci[cnt + rank] = eidx + e;
+              keepbits &= ~(1ull << bit);
+            }
+            ++rank;
           }
         }
-      }
-      cnt += total;
-      DSEL_TR(r, 4);
 #ifdef DSEL_STATS
-      if (tid == 0) ctl.st_appended += total;
+        if (tid == 0) ctl.st_appended += min(total, space);
+#endif
+        if (total <= space) {
+          cnt += total;
+          break;
+        }
+        // buffer full: compact it, raise T, and re-test the survivors still waiting
+        cnt = cap;
+        compact(p.b2 / 2);
+        w = *reinterpret_cast<volatile unsigned long long*>(&ctl.t_w);
+        w = w > t_own ? w : t_own;
+        tk = static_cast<uint32_t>(w >> 32);
+        ti = ~static_cast<uint32_t>(w);
+        uint64_t kb = keepbits;
+        while (kb) {
+          const int bit = __ffsll(static_cast<long long>(kb)) - 1;
+          kb &= kb - 1ull;
+          const int v = bit / PV, e = bit % PV;
+          uint32_t voff, eidx;
+          wr.template locate<VPB>(v, voff, eidx);
+          const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
+          const uint32_t kk = E::key(vec_elem_dyn<DT>(val, e));
+          if (!(kk > tk || (kk == tk && eidx + e < ti))) keepbits &= ~(1ull << bit);
+        }
+        mine = __popcll(keepbits);
+      }
+      DSEL_TR(r, 4);
+      // ---- 5. refill this warp's stages: no other warp reads them ----
+      __syncwarp();
+      if (lane == 0) {
+        fence_proxy_async();   // our reads of the stages come before the copies that overwrite them
+#pragma unroll
+        for (int qb = 0; qb < BPW; ++qb) {
+          const int j = j0 + qb + D;
+          if (j < nb) issue(j);
+        }
+      }
+#ifdef DSEL_STATS
       ++st_rounds;
 #endif
-      // ---- 5. cut the buffer back when it holds k + B2 ----
+      // ---- 6. cut the buffer back when it holds k + B2 ----
       if (cnt >= p.k + p.b2) {   // uniform: cnt is the same register value everywhere
 #ifdef DSEL_STATS
         const long long sc0 = clock64();
 #endif
-        const CompactOut co = compact_buffer<DT, THREADS>(cb, ci, holes, ctl, cluster, cnt, p.k, p.b2 / 2,
-                                                          p.idx_bits, vmax, vlo);
-        cnt = co.cnt;
-        const unsigned long long tw = co.tw;
-        t_own = tw > t_own ? tw : t_own;
-        vlo = co.vlo;
-        // any CTA's threshold is a valid bound for the whole row: push it to the peers
-        if (C > 1 && warp == 0 && lane < C && lane != crank)
-          atomicMax(cluster.map_shared_rank(&ctl.t_w, lane), tw);
+        compact(p.b2 / 2);
 #ifdef DSEL_STATS
         if (tid == 0) {
           ctl.st_compactions += 1;
@@ -774,8 +1062,14 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
 
     const bool to_ws = p.groups > 1;
     const int sort_mode = to_ws ? (p.order == DSEL_ORDER_INDEX ? 1 : 0) : p.order;
-    finalize<DT, THREADS>(p, row, g, cb, ci, holes, ctl, cluster, cnt, nan_thread, vlo, vmax, to_ws,
-                          sort_mode);
+    // index span of the candidates this CTA orders: its slice, or the cluster's
+    // slices when rank 0 gathers them
+    const bool cl_span = C > 1 && p.gather;
+    const int64_t span_a = cl_span ? min(n, static_cast<int64_t>(g * C) * slice) : lo;
+    const int64_t span_b = cl_span ? min(n, static_cast<int64_t>(g * C + C) * slice) : hi;
+    finalize<DT, THREADS>(p, row, g, cb, ci, holes, ctl, cluster, cnt, nan_thread, vlo, vmax, to_ws, sort_mode,
+                          ring, static_cast<uint32_t>(D * B * E::kBytes), static_cast<uint32_t>(span_a),
+                          static_cast<uint32_t>(span_b - span_a));
   }
 #ifdef DSEL_STATS
   if (tid == 0 && blockIdx.x < kStatsCtas) {
@@ -877,7 +1171,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_merge_kernel(const __grid_con
     }
     __syncthreads();   // pref (histogram scratch) is dead from here on
     finalize<DT, THREADS>(p, row, 0, cb, ci, holes, ctl, cluster, nan ? 0 : (b - a), nan, 0ull, vmx, false,
-                          p.order);
+                          p.order, nullptr, 0u, 0u, 0u);
   }
   if (C > 1) cluster.sync();
 }

@@ -42,7 +42,9 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
   p.block = kBlockElems;
   p.round = round_elems(dtype);
   p.b2 = k <= 1024 ? 1024 : std::min(k, 2048);
-  p.capacity = int(round_up(std::max<int64_t>(k + p.b2 + p.round, next_pow2(k)), 32));
+  // k + B2 + slack; a round's survivors beyond that wait in registers until a
+  // compaction makes room, so the round may be larger than the slack
+  p.capacity = int(round_up(std::max<int64_t>(k + p.b2 + append_slack(k), next_pow2(k)), 32));
   p.idx_bits = ceil_log2_u64(uint64_t(row_stride));
 
   // Row split.
@@ -69,8 +71,12 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
   const int64_t per_stage = int64_t(p.block) * eb + 8 + 4;
   int64_t stages = (int64_t(smem_optin) - base) / per_stage;
   stages = std::min<int64_t>(stages, kMaxStages);
-  stages = std::min<int64_t>(stages, std::max<int64_t>(nb_max, per_round));
-  stages = std::max<int64_t>(stages, per_round);
+  if (nb_max <= stages) {
+    stages = nb_max;                         // the whole slice in flight at once, no refills
+  } else {
+    stages = stages / per_round * per_round; // refills go to the warp that owns the stage
+  }
+  stages = std::max<int64_t>(stages, std::min<int64_t>(per_round, nb_max));
   p.stages = int(stages);
   const int64_t smem = stream_layout(stages, p.block, p.capacity, int64_t(k) + p.b2, eb).total;
   if (smem > smem_optin) return DSEL_ERR_K;

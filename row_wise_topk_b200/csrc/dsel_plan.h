@@ -11,7 +11,11 @@ namespace dsel {
 // these (dtype, threads) pairs; the planner only ever returns one of them.
 constexpr int kThreads = 512;
 constexpr int kVecBytes = 16;                 // one 128-bit shared-memory load per vector
-constexpr int kVecsPerThread = 2;             // vectors each thread screens per round
+constexpr int kVecsPerThread = 8;             // vectors each thread screens per round (whole blocks per warp)
+
+// Candidate-buffer slots beyond k + B2.  A round's survivors that do not fit
+// wait until a compaction makes room, so this need not cover a whole round.
+inline int append_slack(int k) { return k <= 1024 ? 4096 : 2048; }
 constexpr int kBlockElems = 1024;             // B: the pages' setting for k = 512
 constexpr int kStrideReq = 16;                // row_stride multiple (elements)
 constexpr int kMaxStages = 128;               // ring depth cap (one mbarrier per stage)

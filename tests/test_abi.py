@@ -100,9 +100,12 @@ def test_plan_invariants(dtype, rows, stride, k):
     assert st == 0
     eb = 2 if dtype == T.DSEL_BF16 else 4
     assert p["smem_bytes"] <= PEAK["smem_optin"]
-    assert p["capacity"] >= k + p["b2"] + p["round"]
+    assert p["capacity"] >= k + p["b2"] + (4096 if k <= 1024 else 2048)
     assert p["capacity"] >= 1 << (k - 1).bit_length()          # room for the bitonic padding
-    assert p["stages"] >= p["round"] // p["block"]
+    q = p["round"] // p["block"]
+    slice_ = -(-(-(-stride // (p["cluster"] * p["groups"]))) // 16) * 16
+    nb_max = -(-slice_ // p["block"])
+    assert p["stages"] == nb_max or (p["stages"] % q == 0 and p["stages"] < nb_max)
     assert p["round"] % p["block"] == 0 and (p["block"] * eb) % 16 == 0
     assert 1 <= p["cluster"] <= PEAK["max_cluster"]
     assert p["groups"] >= 1 and p["groups"] * k <= 8 * p["capacity"]
