@@ -115,13 +115,15 @@ extern "C" {
 
 /* Launch plan chosen for a call (see dsel_plan). */
 typedef struct {
-  int32_t threads;       /* threads per CTA */
+  int32_t threads;       /* threads per CTA: 512 (one CTA per SM), or 128 when there are at least
+                            as many rows as SMs and rows are short (several CTAs per SM) */
   int32_t cluster;       /* CTAs per thread-block cluster working on one row */
   int32_t groups;        /* clusters per row (> 1: split-row plan with a merge launch) */
   int32_t block;         /* B: elements per contiguous block visited in random order */
   int32_t b2;            /* B2: the buffer is cut back to k when it holds k + B2 */
   int32_t round;         /* elements the CTA filters between two buffer checks */
-  int32_t capacity;      /* candidate-buffer slots per CTA (k + B2 + 4096, or + 2048 for k > 1024) */
+  int32_t capacity;      /* candidate-buffer slots per CTA: k + B2 + slack (512 threads: 4096, or
+                            2048 for k > 1024; 128 threads: 1024), at least next_pow2(k) */
   int32_t stages;        /* blocks kept in flight per CTA (shared-memory ring) */
   int32_t idx_bits;      /* bits of the in-row index used to break ties */
   int32_t smem_bytes;    /* dynamic shared memory per CTA */
@@ -204,6 +206,10 @@ DSEL_API int dsel_device_status(int* status_out, void* stream);
  * then cycle times (from kernel start, thread 0) of: set-up done, prologue
  * issued, first round filtered, first round barrier, first compaction done,
  * stream done; then thread 0's cycles waiting for blocks, and total cycles.
+ * With n_ctas == -1, host_out instead receives the per-round timeline of CTA 0:
+ * 16 warps x 12 rounds x 10 int64 cycle times from kernel start (round start,
+ * screened, counted, append barrier, written, after compaction, prefixed,
+ * seeded, blocks arrived, seed returned; 0 = not reached).
  * Synchronises `stream`. */
 DSEL_API int dsel_debug_stats(uint64_t* host_out, int64_t n_ctas, void* stream);
 

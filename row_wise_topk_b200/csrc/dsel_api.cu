@@ -18,7 +18,7 @@ struct DevInfo {
   int sms = 0;
   int smem_optin = 0;
   int major = 0;
-  bool attrs_set[2] = {false, false};
+  bool attrs_set[2][2] = {{false, false}, {false, false}};   // [dtype][short shape]
 };
 
 std::mutex g_mu;
@@ -76,11 +76,11 @@ int workspace(int dev, void* stream, size_t bytes, void** out) {
 }
 
 template <typename Kern>
-cudaError_t launch_cluster(Kern kern, unsigned grid, int cluster, uint32_t smem, cudaStream_t st,
+cudaError_t launch_cluster(Kern kern, unsigned grid, int threads, int cluster, uint32_t smem, cudaStream_t st,
                            const KParams& kp) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -93,17 +93,18 @@ cudaError_t launch_cluster(Kern kern, unsigned grid, int cluster, uint32_t smem,
   return cudaLaunchKernelEx(&cfg, kern, kp);
 }
 
-template <int DT>
-int run(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
-  auto sk = topk_stream_kernel<DT, kThreads>;
+template <int DT, int THREADS>
+int run_shape(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
+  auto sk = topk_stream_kernel<DT, THREADS>;
   auto mk = topk_merge_kernel<DT, kThreads>;
-  if (!di->attrs_set[DT]) {
+  constexpr int shp = THREADS == kThreads ? 0 : 1;
+  if (!di->attrs_set[DT][shp]) {
     if (cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) != cudaSuccess ||
         cudaFuncSetAttribute(sk, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
         cudaFuncSetAttribute(mk, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) != cudaSuccess ||
         cudaFuncSetAttribute(mk, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
       return DSEL_ERR_CUDA;
-    di->attrs_set[DT] = true;
+    di->attrs_set[DT][shp] = true;
   }
   const int eb = elem_bytes(DT);
   const SmemLayout sl = stream_layout(pl.stages, pl.block, pl.capacity, int64_t(base.k) + pl.b2, eb);
@@ -117,7 +118,7 @@ int run(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t s
   kp.gather = int64_t(pl.cluster) * base.k <= pl.capacity;
   const int64_t grid = rows * pl.groups * pl.cluster;
   if (grid > 0x7FFFFFFF) return DSEL_ERR_ROWS;
-  if (launch_cluster(sk, unsigned(grid), pl.cluster, sl.total, st, kp) != cudaSuccess) return DSEL_ERR_CUDA;
+  if (launch_cluster(sk, unsigned(grid), THREADS, pl.cluster, sl.total, st, kp) != cudaSuccess) return DSEL_ERR_CUDA;
   if (pl.groups > 1) {
     const SmemLayout ml = merge_layout(pl.capacity, int64_t(base.k) + pl.b2, eb);
     KParams mp = kp;
@@ -127,9 +128,17 @@ int run(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t s
     mp.off_ctl = ml.ctl;
     const int mc = merge_cluster(pl, base.k);
     mp.gather = int64_t(mc) * base.k <= pl.capacity;
-    if (launch_cluster(mk, unsigned(rows * mc), mc, ml.total, st, mp) != cudaSuccess) return DSEL_ERR_CUDA;
+    if (launch_cluster(mk, unsigned(rows * mc), kThreads, mc, ml.total, st, mp) != cudaSuccess) return DSEL_ERR_CUDA;
   }
   return DSEL_OK;
+}
+
+// The planner returns split-row plans (groups > 1) only with the 512-thread shape.
+template <int DT>
+int run(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
+  if (pl.threads == kThreadsShort) return run_shape<DT, kThreadsShort>(base, pl, rows, st, di);
+  if (pl.threads == kThreads) return run_shape<DT, kThreads>(base, pl, rows, st, di);
+  return DSEL_ERR_DEVICE;
 }
 
 }  // namespace
@@ -174,7 +183,7 @@ DSEL_API int dsel_debug_stats(uint64_t* host_out, int64_t n_ctas, void* stream) 
   const int64_t n = n_ctas < kStatsCtas ? n_ctas : kStatsCtas;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (n_ctas == -1) {   // the per-round timeline instead (4 x 64 x 6 values)
-    if (cudaMemcpyFromSymbolAsync(host_out, g_trace, sizeof(long long) * 4 * kTraceRounds * kTraceEvents, 0,
+    if (cudaMemcpyFromSymbolAsync(host_out, g_trace, sizeof(long long) * kTraceSize, 0,
                                   cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
         cudaStreamSynchronize(cs) != cudaSuccess)
       return DSEL_ERR_CUDA;

@@ -350,6 +350,7 @@ __device__ __noinline__ SelResult radix_select(const typename Elem<DT>::bits_t* 
     const uint32_t dmask = (1u << dbits) - 1u;
     int* h = ctl.hist[hb];
     int* hz = ctl.hist[hb == 2 ? 0 : hb + 1];
+#pragma unroll 1
     for (int i = tid; i < kBins; i += THREADS) hz[i] = 0;
     if (shift >= idx_bits) {   // digit and prefix inside the key bits
       const int ks = shift - idx_bits;
@@ -371,8 +372,10 @@ __device__ __noinline__ SelResult radix_select(const typename Elem<DT>::bits_t* 
     cta_or_cluster_sync<CLUSTER>(cluster);
     if (CLUSTER) {
       const int nr = static_cast<int>(cluster.num_blocks());
+#pragma unroll 1
       for (int b = tid; b < kBins; b += THREADS) {
         int s = 0;
+#pragma unroll 1
         for (int r = 0; r < nr; ++r) s += cluster.map_shared_rank(h, r)[b];
         ctl.hsum[b] = s;
       }
@@ -438,6 +441,7 @@ __device__ __noinline__ int holes_compact(typename Elem<DT>::bits_t* cb, uint32_
     const int chunk = ((cnt + NW - 1) / NW + 31) & ~31;
     const int a = min(cnt, warp * chunk), b = min(cnt, a + chunk);
     int n = 0;
+#pragma unroll 1
     for (int p0 = a; p0 < b; p0 += 32) {
       const int p = p0 + lane;
       n += __popc(__ballot_sync(0xffffffffu, p < b && keep_at(p)));
@@ -455,10 +459,12 @@ __device__ __noinline__ int holes_compact(typename Elem<DT>::bits_t* cb, uint32_
   const int ha = min(kept, warp * hc), hbnd = min(kept, ha + hc);
   const int ma = kept + min(cnt - kept, warp * mc), mbnd = min(cnt, ma + mc);
   int nh = 0, nm = 0;
+#pragma unroll 1
   for (int p0 = ha; p0 < hbnd; p0 += 32) {
     const int p = p0 + lane;
     nh += __popc(__ballot_sync(0xffffffffu, p < hbnd && !keep_at(p)));
   }
+#pragma unroll 1
   for (int p0 = ma; p0 < mbnd; p0 += 32) {
     const int p = p0 + lane;
     nm += __popc(__ballot_sync(0xffffffffu, p < mbnd && keep_at(p)));
@@ -472,6 +478,7 @@ __device__ __noinline__ int holes_compact(typename Elem<DT>::bits_t* cb, uint32_
   int hoff = warp_prefix_of<NW>(ctl.wc[0], warp, lane, tot);
   int moff = warp_prefix_of<NW>(ctl.wm, warp, lane, tot);
   const uint32_t below = (1u << lane) - 1u;
+#pragma unroll 1
   for (int p0 = ha; p0 < hbnd; p0 += 32) {
     const int p = p0 + lane;
     const bool hole = p < hbnd && !keep_at(p);
@@ -480,6 +487,7 @@ __device__ __noinline__ int holes_compact(typename Elem<DT>::bits_t* cb, uint32_
     hoff += __popc(bal);
   }
   __syncthreads();
+#pragma unroll 1
   for (int p0 = ma; p0 < mbnd; p0 += 32) {
     const int p = p0 + lane;
     const bool mover = p < mbnd && keep_at(p);
@@ -515,13 +523,17 @@ __device__ __noinline__ void bitonic_sort(typename Elem<DT>::bits_t* cb, uint32_
   const int tid = threadIdx.x;
   int M = 1;
   while (M < m) M <<= 1;
+#pragma unroll 1
   for (int i = m + tid; i < M; i += THREADS) {
     ci[i] = 0xFFFFFFFFu;
     cb[i] = static_cast<typename Elem<DT>::bits_t>(Elem<DT>::kNegInf);
   }
   __syncthreads();
+#pragma unroll 1
   for (int size = 2; size <= M; size <<= 1) {
+#pragma unroll 1
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll 1
       for (int t = tid; t < (M >> 1); t += THREADS) {
         const int lo = 2 * t - (t & (stride - 1));
         const int hi = lo + stride;

@@ -35,11 +35,24 @@ struct KParams {
 constexpr int kStatsCtas = 8192;
 constexpr int kStatsFields = 16;
 __device__ unsigned long long g_stats[kStatsCtas * kStatsFields];
-// per-round timeline of CTA 0 for warps 0, 5, 10, 15 (lane 0): [warp][round][event]
-constexpr int kTraceRounds = 64;
-constexpr int kTraceEvents = 8;
-__device__ long long g_trace[4 * kTraceRounds * kTraceEvents];
+// per-round timeline of CTA 0 (lane 0 of every warp): [warp][round][event]
+constexpr int kTraceWarps = 16;
+constexpr int kTraceRounds = 12;
+constexpr int kTraceEvents = 10;
+constexpr int kTraceSize = kTraceWarps * kTraceRounds * kTraceEvents;
+__device__ long long g_trace[kTraceSize];
 #endif
+
+// Final-phase timeline of CTA 0 (thread 0), stats builds only: absolute clocks
+// in trace row kTraceRounds - 1 of warp 0; slot kTraceEvents - 1 holds the
+// kernel-start clock.
+__device__ __forceinline__ void trace_final(int e) {
+#ifdef DSEL_STATS
+  if (blockIdx.x == 0 && threadIdx.x == 0) g_trace[(kTraceRounds - 1) * kTraceEvents + e] = clock64();
+#else
+  (void)e;
+#endif
+}
 
 constexpr int kSeedBits = 11;                 // round-0 histogram: 2048 bins
 constexpr int kSeedBins = 1 << kSeedBits;
@@ -52,6 +65,7 @@ __device__ void write_rows_out(const KParams& p, int64_t row, int off, int m,
                                const typename Elem<DT>::bits_t* cb, const uint32_t* ci) {
   using bits_t = typename Elem<DT>::bits_t;
   const int64_t base = row * p.k + off;
+#pragma unroll 1
   for (int i = threadIdx.x; i < m; i += THREADS) {
     const uint32_t idx = ci[i];
     if (p.index_i64) static_cast<int64_t*>(p.indices_out)[base + i] = static_cast<int64_t>(idx);
@@ -64,13 +78,15 @@ template <int DT, int THREADS>
 __device__ void write_ws(const KParams& p, int64_t row, int g, int off, int m,
                          const typename Elem<DT>::bits_t* cb, const uint32_t* ci) {
   uint2* dst = p.ws_pairs + (row * p.groups + g) * static_cast<int64_t>(p.k) + off;
+#pragma unroll 1
   for (int i = threadIdx.x; i < m; i += THREADS) dst[i] = make_uint2(ci[i], static_cast<uint32_t>(cb[i]));
 }
 
 template <int DT, int THREADS>
-__device__ void write_sentinel_row(const KParams& p, int64_t row, int32_t code) {
+__device__ __noinline__ void write_sentinel_row(const KParams& p, int64_t row, int32_t code) {
   using bits_t = typename Elem<DT>::bits_t;
   const int64_t base = row * p.k;
+#pragma unroll 1
   for (int i = threadIdx.x; i < p.k; i += THREADS) {
     if (p.index_i64) static_cast<int64_t*>(p.indices_out)[base + i] = code;
     else static_cast<int32_t*>(p.indices_out)[base + i] = code;
@@ -80,10 +96,11 @@ __device__ void write_sentinel_row(const KParams& p, int64_t row, int32_t code) 
 
 // Rows no longer than k: every entry, in index order, then padding.  No NaN check.
 template <int DT, int THREADS>
-__device__ void write_short_row(const KParams& p, int64_t row, int64_t n) {
+__device__ __noinline__ void write_short_row(const KParams& p, int64_t row, int64_t n) {
   using bits_t = typename Elem<DT>::bits_t;
   const bits_t* xr = static_cast<const bits_t*>(p.x) + row * p.row_stride;
   const int64_t base = row * p.k;
+#pragma unroll 1
   for (int i = threadIdx.x; i < p.k; i += THREADS) {
     const bool in = i < n;
     const int32_t idx = in ? i : DSEL_IDX_PAD;
@@ -128,6 +145,7 @@ __device__ __noinline__ int local_select(typename Elem<DT>::bits_t* cb, uint32_t
   if (cnt <= need) return cnt;
   const SelResult sel =
       radix_select<DT, THREADS, false>(cb, ci, cnt, need, 0, idx_bits, vlo, vhi, ctl, cluster);
+  trace_final(4);
   return holes_compact<DT, THREADS>(cb, ci, cnt, sel.kept, sel, idx_bits, ctl, holes);
 }
 
@@ -179,8 +197,10 @@ __device__ __noinline__ void finish_sorted(const KParams& p, int64_t row, int g,
   if (sort_mode == 1 && scratch != nullptr && 8ull * words <= scratch_bytes) {
     uint32_t* bm = reinterpret_cast<uint32_t*>(scratch);
     uint32_t* wp = bm + words;
+#pragma unroll 1
     for (uint32_t i = tid; i < words; i += THREADS) bm[i] = 0u;
     __syncthreads();
+#pragma unroll 1
     for (int i = tid; i < m; i += THREADS) {
       const uint32_t d = ci[i] - span_lo;
       atomicOr(&bm[d >> 5], 1u << (d & 31u));
@@ -190,6 +210,7 @@ __device__ __noinline__ void finish_sorted(const KParams& p, int64_t row, int g,
     const uint32_t per = ((words + NW - 1) / NW + 31u) & ~31u;
     const uint32_t a = min(words, warp * per), b = min(words, a + per);
     int sum = 0;
+#pragma unroll 1
     for (uint32_t w0 = a; w0 < b; w0 += 32) {
       const uint32_t w = w0 + lane;
       sum += __popc(w < b ? bm[w] : 0u);
@@ -199,6 +220,7 @@ __device__ __noinline__ void finish_sorted(const KParams& p, int64_t row, int g,
     __syncthreads();
     int tot;
     int base = warp_prefix_of<NW>(ctl.wm, warp, lane, tot);
+#pragma unroll 1
     for (uint32_t w0 = a; w0 < b; w0 += 32) {
       const uint32_t w = w0 + lane;
       const int c = __popc(w < b ? bm[w] : 0u);
@@ -209,6 +231,7 @@ __device__ __noinline__ void finish_sorted(const KParams& p, int64_t row, int g,
     __syncthreads();
     const int64_t obase = row * p.k + off;
     uint2* wsd = to_workspace ? p.ws_pairs + (row * p.groups + g) * static_cast<int64_t>(p.k) + off : nullptr;
+#pragma unroll 1
     for (int i = tid; i < m; i += THREADS) {
       const uint32_t idx = ci[i];
       const uint32_t d = idx - span_lo;
@@ -253,9 +276,11 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
   const int tid = threadIdx.x, lane = tid & 31;
   const uint32_t idx_mask = mask_bits(p.idx_bits);
 
+  trace_final(0);
   if (nan_local) ctl.nan_found = 1;
   const uint64_t vhi = cta_vmax<THREADS>(vmax_thread, ctl);   // barrier: nan_found visible
   const bool nan_cta = ctl.nan_found != 0;
+  trace_final(1);
 
   if (C == 1) {
     if (nan_cta) {
@@ -263,8 +288,10 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
       return;
     }
     const int m = local_select<DT, THREADS>(cb, ci, cnt, p.k, p.idx_bits, vlo, vhi, ctl, holes, cluster);
+    trace_final(5);
     finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, m, sort_mode, ctl, ring, ring_bytes, span_lo,
                                span_len, 0, m, true);
+    trace_final(6);
     return;
   }
 
@@ -277,6 +304,7 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
       ctl.x_vhi = cnt > 0 ? vhi : 0ull;
     }
     cluster.sync();
+    trace_final(2);
     int tot = 0, nn = 0;
     unsigned long long lo = ~0ull, hi = 0ull;
     if (lane < C) {
@@ -311,11 +339,13 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
     }
     if (crank != 0) return;
     int off = m;
+#pragma unroll 1
     for (int r = 1; r < C; ++r) {
       Ctl* pr = cluster.map_shared_rank(&ctl, r);
       const int mr = direct ? pr->x_cnt : pr->x_kept;
       const bits_t* rcb = cluster.map_shared_rank(cb, r);
       const uint32_t* rci = cluster.map_shared_rank(ci, r);
+#pragma unroll 1
       for (int i = tid; i < mr; i += THREADS) {
         cb[off + i] = rcb[i];
         ci[off + i] = rci[i];
@@ -323,13 +353,17 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
       off += mr;
     }
     __syncthreads();   // the gathered list is complete
+    trace_final(3);
     const int mm = local_select<DT, THREADS>(cb, ci, off, p.k, p.idx_bits, lo, hi, ctl, holes, cluster);
+    trace_final(5);
     finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, mm, sort_mode, ctl, ring, ring_bytes, span_lo,
                                span_len, 0, mm, true);
+    trace_final(6);
     return;
   }
 
   // ---- distributed select over the cluster ----
+#pragma unroll 1
   for (int i = tid; i < 3 * kBins; i += THREADS) (&ctl.hist[0][0])[i] = 0;
   if (tid == 0) {
     ctl.hb = 0;
@@ -373,10 +407,12 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
   if (sort_mode == 2) {   // gather the winners on rank 0 and sort them by value
     if (crank == 0) {
       int off = m;
+#pragma unroll 1
       for (int r = 1; r < C; ++r) {
         const int mr = cluster.map_shared_rank(&ctl, r)->x_kept;
         const bits_t* rcb = cluster.map_shared_rank(cb, r);
         const uint32_t* rci = cluster.map_shared_rank(ci, r);
+#pragma unroll 1
         for (int i = tid; i < mr; i += THREADS) {
           cb[off + i] = rcb[i];
           ci[off + i] = rci[i];
@@ -396,29 +432,132 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
                              span_len, off, need, crank == 0);
 }
 
+// Survivor bits of one thread in one round (up to 128 elements), kept in two
+// registers; bit positions are run-time values, so no array indexing.
+struct Keep128 {
+  uint64_t w[2];
+  __device__ __forceinline__ void set(int b) {
+    if (b < 64) w[0] |= 1ull << b;
+    else w[1] |= 1ull << (b - 64);
+  }
+  __device__ __forceinline__ void clr(int b) {
+    if (b < 64) w[0] &= ~(1ull << b);
+    else w[1] &= ~(1ull << (b - 64));
+  }
+  __device__ __forceinline__ int count() const { return __popcll(w[0]) + __popcll(w[1]); }
+};
+
 // ---------------------------------------------------------------------------
-// Where this thread's vectors sit in the current round.  A warp owns whole
-// blocks (BPW <= 2 of them); vector v of lane l is 16-byte slot (v*32 + l) % VPB
-// of owned block (v*32) / VPB.
+// Where this thread's vectors sit in the current round.  A warp owns one whole
+// block per round (B = 32 lanes x VPT vectors); vector v of a lane is 16-byte
+// slot v * 32 + lane of that block, at ring byte offset sb + v * 512, starting
+// at row element eb + v * 32 * PV.
 // ---------------------------------------------------------------------------
 template <int DT>
 struct WarpRound {
-  int j0, nb, D, s0, lane;
-  uint32_t boff0, boff1;   // first element (in the row) of the warp's owned blocks
-  uint32_t uhi;            // end of this CTA's slice
-  template <int VPB>
+  static constexpr int PV = Elem<DT>::kPerVec;
+  uint32_t sb;   // ring byte offset of the lane's first vector
+  uint32_t eb;   // row element of the lane's first vector
+  int j0;        // the owned block (visit order)
+  bool owns;     // the block exists this round (warp-uniform)
+  uint32_t uhi;  // end of this CTA's slice
+  // Ring byte offset and first row element of vector v; false when the vector
+  // lies past the slice end or the warp owns no block this round.
   __device__ __forceinline__ bool locate(int v, uint32_t& voff, uint32_t& eidx) const {
-    const int qb = (v * 32) / VPB;
-    if (j0 + qb >= nb) return false;
-    const int o = (v * 32 + lane) % VPB;
-    eidx = (qb ? boff1 : boff0) + static_cast<uint32_t>(o * Elem<DT>::kPerVec);
+    if (!owns) return false;
+    eidx = eb + static_cast<uint32_t>(v * 32 * PV);
     if (eidx >= uhi) return false;
-    int st = s0 + qb;
-    if (st >= D) st -= D;
-    voff = static_cast<uint32_t>(st * kBlockElems * Elem<DT>::kBytes + o * 16);
+    voff = sb + static_cast<uint32_t>(v * 512);
     return true;
   }
 };
+
+// Key of the largest element of a 16-byte vector; true (key unset) when the
+// vector holds a NaN.
+template <int DT>
+__device__ __forceinline__ bool vec_max_key(const uint4 x, uint32_t& key) {
+  using E = Elem<DT>;
+  if (DT == DSEL_BF16) {
+    const uint32_t m2 = bf16x2_max_nan(bf16x2_max_nan(x.x, x.y), bf16x2_max_nan(x.z, x.w));
+    const uint32_t lo = m2 & 0xFFFFu, hi = m2 >> 16;
+    if (E::is_nan(lo) || E::is_nan(hi)) return true;
+    const uint32_t klo = E::key(lo), khi = E::key(hi);
+    key = klo > khi ? klo : khi;
+    return false;
+  } else {
+    const float a = __uint_as_float(x.x), b = __uint_as_float(x.y), c = __uint_as_float(x.z), d = __uint_as_float(x.w);
+    if (a != a || b != b || c != c || d != d) return true;
+    key = E::key(__float_as_uint(fmaxf(fmaxf(a, b), fmaxf(c, d))));
+    return false;
+  }
+}
+
+// Largest key t such that at least k of the CTA's non-empty group maxima
+// (gm != 0) are >= t, or 0 when the CTA holds fewer than k of them.  Bisection
+// over the bits below the common prefix of the smallest and largest maximum,
+// three bits per step: every warp counts its maxima at the seven candidate
+// thresholds, the per-warp counts meet in `scratch` (2 x NW x 8 ints, double
+// buffered so that one barrier per step suffices), and every warp takes the
+// same decision.
+template <int THREADS, int G>
+__device__ __forceinline__ uint32_t cta_kth_largest(const uint32_t (&gm)[G], int k, Ctl& ctl, int* scratch) {
+  constexpr int NW = THREADS / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int nz = 0;
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    if (gm[g] != 0u) {
+      ++nz;
+      kmin = min(kmin, gm[g]);
+      kmax = max(kmax, gm[g]);
+    }
+  }
+  nz = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(nz)));
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) {
+    ctl.wm[warp] = nz;
+    ctl.wv[warp] = (static_cast<unsigned long long>(kmax) << 32) | kmin;
+  }
+  __syncthreads();   // ctl.wm / wv are written again only after later barriers
+  nz = static_cast<int>(__reduce_add_sync(0xffffffffu, lane < NW ? static_cast<unsigned>(ctl.wm[lane]) : 0u));
+  if (nz < k) return 0u;   // uniform
+  const unsigned long long wv = lane < NW ? ctl.wv[lane] : 0xFFFFFFFFull;
+  kmin = __reduce_min_sync(0xffffffffu, static_cast<uint32_t>(wv));
+  kmax = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(wv >> 32));
+  int b = 32 - __clz(kmin ^ kmax);   // bits below the common prefix
+  uint32_t pre = kmax & ~mask_bits(b);
+  int par = 0;
+#pragma unroll 1
+  while (b > 0) {   // uniform
+    const int sb = b >= 3 ? 3 : b;
+    b -= sb;
+    int* sc = scratch + par * (NW * 8);
+    par ^= 1;
+    // counts at thresholds pre | t << b, t = 1 .. 7 (those with t >= 2^sb stay 0)
+#pragma unroll
+    for (int t = 1; t < 8; ++t) {
+      int c = 0;
+      if (t < (1 << sb)) {
+        const uint32_t cand = pre | (static_cast<uint32_t>(t) << b);
+#pragma unroll
+        for (int g = 0; g < G; ++g) c += gm[g] >= cand ? 1 : 0;
+      }
+      c = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c)));
+      if (lane == 0) sc[warp * 8 + t] = c;
+    }
+    __syncthreads();
+    int best = 0;
+#pragma unroll
+    for (int t = 1; t < 8; ++t) {
+      const int tot = static_cast<int>(__reduce_add_sync(0xffffffffu, lane < NW ? static_cast<unsigned>(sc[lane * 8 + t]) : 0u));
+      if (t < (1 << sb) && tot >= k) best = t;
+    }
+    pre |= static_cast<uint32_t>(best) << b;
+  }
+  return pre;
+}
 
 // ---------------------------------------------------------------------------
 // Round-0 threshold seed (cold path, kept out of the per-round loop).  A
@@ -439,7 +578,6 @@ __device__ __noinline__ SeedOut seed_threshold(const unsigned char* ring, WarpRo
   using E = Elem<DT>;
   constexpr int NW = THREADS / 32;
   constexpr int PV = E::kPerVec;
-  constexpr int VPB = kBlockElems / PV;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t uhi = wr.uhi;
   int nvalid = 0;
@@ -447,7 +585,7 @@ __device__ __noinline__ SeedOut seed_threshold(const unsigned char* ring, WarpRo
 #pragma unroll 1
   for (int v = 0; v < VPT; ++v) {
     uint32_t voff, eidx;
-    if (!wr.template locate<VPB>(v, voff, eidx)) continue;
+    if (!wr.locate(v, voff, eidx)) continue;
     const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
 #pragma unroll
     for (int e = 0; e < PV; ++e) {
@@ -493,13 +631,14 @@ __device__ __noinline__ SeedOut seed_threshold(const unsigned char* ring, WarpRo
   int need = k;
   constexpr int SLICE = kSeedBins / NW;
   constexpr int PER_LANE = SLICE / 32;
+#pragma unroll 1
   for (int level = 0; level < 2; ++level) {           // uniform
     int* hist = seed_hist + level * kSeedBins;
     const int ws = width > kSeedBits ? width - kSeedBits : 0;
 #pragma unroll 1
     for (int v = 0; v < VPT; ++v) {
       uint32_t voff, eidx;
-      if (!wr.template locate<VPB>(v, voff, eidx)) continue;
+      if (!wr.locate(v, voff, eidx)) continue;
       const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
 #pragma unroll
       for (int e = 0; e < PV; ++e) {
@@ -565,109 +704,25 @@ __device__ __noinline__ SeedOut seed_threshold(const unsigned char* ring, WarpRo
 }
 
 // ---------------------------------------------------------------------------
-// Cheap round-0 seed for k <= 4 * THREADS: the maximum of every full 16-byte
-// vector of the round (NaN-ignoring), then the k-th largest of those maxima by
-// a radix select over their keys.  Each maximum is a real element, so at least
-// k elements are >= the result: a valid starting T.  A vector that is partial
-// (past the slice end) or whose maximum is NaN counts as empty (key 0, below
-// every number).
+// Bulk copy of the j-th block in visiting order, (pa * j + pc) mod nb, of the
+// slice [lo, hi) into ring stage j mod D.  Out of line: it is called from the
+// prologue and from every refill, and inlining would repeat its 64-bit modulo.
 // ---------------------------------------------------------------------------
-template <int DT, int THREADS, int VPT>
-__device__ __noinline__ SeedOut seed_by_vector_max(const unsigned char* ring, WarpRound<DT> wr, int k, int idx_bits,
-                                                   Ctl& ctl) {
+template <int DT>
+__device__ __noinline__ void issue_block(int j, uint32_t pa, uint32_t pc, int nb, int64_t lo, int64_t hi, int D,
+                                         const char* rowp, unsigned char* ring, uint64_t* bars, uint32_t* blk_off) {
   using E = Elem<DT>;
-  constexpr int NW = THREADS / 32;
-  constexpr int PV = E::kPerVec;
-  constexpr int VPB = kBlockElems / PV;
-  const int tid = threadIdx.x, lane = tid & 31;
-  uint32_t gk[VPT];
-#pragma unroll
-  for (int v = 0; v < VPT; ++v) {
-    gk[v] = 0u;
-    uint32_t voff, eidx;
-    if (wr.template locate<VPB>(v, voff, eidx) && eidx + PV <= wr.uhi) {
-      const uint4 x = *reinterpret_cast<const uint4*>(ring + voff);
-      uint32_t mb;
-      if (DT == DSEL_BF16) {
-        const uint32_t m2 = bf16x2_max(bf16x2_max(x.x, x.y), bf16x2_max(x.z, x.w));
-        const uint32_t lo = m2 & 0xFFFFu, hi = m2 >> 16;
-        const uint32_t klo = E::is_nan(lo) ? 0u : E::key(lo), khi = E::is_nan(hi) ? 0u : E::key(hi);
-        gk[v] = klo > khi ? klo : khi;
-        (void)mb;
-      } else {
-        const float m = fmaxf(fmaxf(__uint_as_float(x.x), __uint_as_float(x.y)),
-                              fmaxf(__uint_as_float(x.z), __uint_as_float(x.w)));
-        mb = __float_as_uint(m);
-        gk[v] = E::is_nan(mb) ? 0u : E::key(mb);
-      }
-    }
-  }
-  // k-th largest of the THREADS * VPT maxima: 8-bit digits from the top of the key
-  int need = k;
-  uint32_t prefix = 0;
-  int depth = 0;
-  int* h = ctl.hist[0];
-  for (int i = tid; i < kBins; i += THREADS) h[i] = 0;
-  __syncthreads();
-  while (true) {   // uniform
-    const int sh = E::kKeyBits - depth - kDigitBits;
-#pragma unroll
-    for (int v = 0; v < VPT; ++v) {
-      const uint32_t top = (depth == 0) ? 0u : (gk[v] >> (sh + kDigitBits));
-      if (top == prefix) atomicAdd(&h[(gk[v] >> sh) & (kBins - 1)], 1);
-    }
-    __syncthreads();
-    int c[kBins / 32];
-    int s = 0;
-#pragma unroll
-    for (int j = 0; j < kBins / 32; ++j) {
-      c[j] = h[kBins - 1 - (lane * (kBins / 32) + j)];
-      s += c[j];
-    }
-    const int incl = warp_incl_scan(s, lane);
-    const bool mine = (incl - s) < need && need <= incl;
-    const unsigned bal = __ballot_sync(0xffffffffu, mine);
-    int digit = 0, above = 0, bucket = 0;
-    if (mine) {
-      int acc = incl - s;
-      bool done = false;
-#pragma unroll
-      for (int j = 0; j < kBins / 32; ++j) {
-        if (!done && acc + c[j] >= need) {
-          digit = kBins - 1 - (lane * (kBins / 32) + j);
-          above = acc;
-          bucket = c[j];
-          done = true;
-        }
-        acc += c[j];
-      }
-    }
-    __syncthreads();   // every warp has read the histogram
-    if (bal == 0u) {   // fewer than k maxima (uniform); leave the histogram zeroed
-      for (int i = tid; i < kBins; i += THREADS) h[i] = 0;
-      return SeedOut{0ull, 0ull, false};
-    }
-    const int src = __ffs(bal) - 1;
-    digit = __shfl_sync(0xffffffffu, digit, src);
-    above = __shfl_sync(0xffffffffu, above, src);
-    bucket = __shfl_sync(0xffffffffu, bucket, src);
-    need -= above;
-    prefix = (prefix << kDigitBits) | static_cast<uint32_t>(digit);
-    depth += kDigitBits;
-    if (need == bucket || depth == E::kKeyBits) break;
-    for (int i = tid; i < kBins; i += THREADS) h[i] = 0;
-    __syncthreads();
-  }
-  const uint32_t key_t = depth >= E::kKeyBits ? prefix : (prefix << (E::kKeyBits - depth));
-  if (key_t == 0u) return SeedOut{0ull, 0ull, false};   // the k-th maximum is an empty vector
-  for (int i = tid; i < kBins; i += THREADS) h[i] = 0;   // the histograms start zeroed elsewhere
-  __syncthreads();
-  SeedOut out;
-  out.t = make_w(key_t, 0xFFFFFFFFu);   // passes every key >= key_t
-  out.vlo = static_cast<uint64_t>(key_t) << idx_bits;
-  out.ok = true;
-  (void)NW;
-  return out;
+  constexpr int B = block_elems_for(E::kBytes);
+  const uint32_t m = static_cast<uint32_t>((static_cast<uint64_t>(pa) * static_cast<uint32_t>(j) + pc) %
+                                           static_cast<uint32_t>(nb));
+  const int64_t e0 = lo + static_cast<int64_t>(m) * B;
+  const int64_t ce = min(static_cast<int64_t>(B), hi - e0);
+  const uint32_t bytes = static_cast<uint32_t>((ce * E::kBytes + 15) & ~static_cast<int64_t>(15));
+  const int s = j % D;
+  blk_off[s] = static_cast<uint32_t>(e0);
+  const uint32_t bar = smem_u32(&bars[s]);
+  mbar_expect_tx(bar, bytes);
+  bulk_g2s(smem_u32(ring + static_cast<size_t>(s) * B * E::kBytes), rowp + e0 * E::kBytes, bytes, bar);
 }
 
 // ---------------------------------------------------------------------------
@@ -703,22 +758,21 @@ __device__ __noinline__ CompactOut compact_buffer(typename Elem<DT>::bits_t* cb,
 // that T starts near the k-th value instead of at -inf.
 // ---------------------------------------------------------------------------
 template <int DT, int THREADS>
-__global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_constant__ KParams p) {
+__global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kernel(const __grid_constant__ KParams p) {
   using E = Elem<DT>;
   using bits_t = typename E::bits_t;
   constexpr int NW = THREADS / 32;
   constexpr int PV = E::kPerVec;
-  constexpr int B = kBlockElems;
-  constexpr int VPB = B / PV;                          // 16-byte vectors per block
-  constexpr int R = round_elems_for(E::kBytes);       // elements per round
-  constexpr int Q = R / B;                             // blocks per round
+  constexpr int B = block_elems_for(E::kBytes);       // elements per block: one warp's share of a round
+  constexpr int R = round_elems_for(E::kBytes, THREADS);   // elements per round
+  constexpr int Q = R / B;                             // blocks per round: one per warp
   constexpr int VPT = R / (THREADS * PV);              // vectors per thread per round
-  static_assert(VPB % 32 == 0, "a warp must stay inside one block");
-  static_assert(VPT >= 1 && VPT * THREADS * PV == R && Q * B == R, "round shape");
-  constexpr int VPW = 32 * VPT;                        // vectors per warp per round
-  static_assert(VPW % VPB == 0 || VPB % VPW == 0, "warps own whole blocks or whole warps share one");
-  static_assert(VPW >= VPB, "a warp owns whole blocks, so only it reads and refills their stages");
-  constexpr int BPW = VPW / VPB;                       // blocks owned by a warp per round
+  static_assert(Q == NW && VPT * 32 * PV == B && VPT * THREADS * PV == R, "round shape");
+  static_assert(VPT <= 32, "screen flags fit one 32-bit mask");
+  constexpr int SG = THREADS == kThreads ? 4 : 8;      // round-0 seed: group maxima per thread
+  constexpr int VPG = VPT / SG;                        // vectors per group
+  static_assert(VPG * SG == VPT, "seed groups");
+  static_assert(VPT * PV <= 128, "keep bits fit two 64-bit words");
   static_assert(kSeedBins % (NW * 32) == 0, "seed histogram split");
 
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -740,13 +794,14 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
   const int D = p.stages;
 #ifdef DSEL_STATS
   const long long st_t0 = clock64();
+  if (blockIdx.x == 0 && threadIdx.x == 0) g_trace[(kTraceRounds - 1) * kTraceEvents + kTraceEvents - 1] = st_t0;
   long long st_t1 = st_t0;
   int st_rounds = 0;
   long long st_ev[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   long long st_wait = 0;
 #define DSEL_EV(i) do { if (tid == 0) st_ev[i] = clock64() - st_t0; } while (0)
-  const int tr_w = (blockIdx.x == 0 && lane == 0 && warp % 5 == 0) ? warp / 5 : -1;
-#define DSEL_TR(r, e) do { if (tr_w >= 0 && (r) < kTraceRounds) \
+  const int tr_w = (blockIdx.x == 0 && lane == 0 && warp < kTraceWarps) ? warp : -1;
+#define DSEL_TR(r, e) do { if (tr_w >= 0 && (r) < kTraceRounds - 1) \
     g_trace[(tr_w * kTraceRounds + (r)) * kTraceEvents + (e)] = clock64() - st_t0; } while (0)
 #else
 #define DSEL_EV(i) do { } while (0)
@@ -756,7 +811,9 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
   bool bad_end;
   const int64_t n = row_length(p, row, &bad_end);
 
+#pragma unroll 1
   for (int i = tid; i < 3 * kBins; i += THREADS) (&ctl.hist[0][0])[i] = 0;
+#pragma unroll 1
   for (int i = tid; i < 2 * kSeedBins; i += THREADS) seed_hist[i] = 0;   // two histogram levels
   if (tid == 0) {
     ctl.t_w = 0ull;
@@ -769,7 +826,10 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
     ctl.st_appended = 0;
     ctl.st_slow_vectors = 0;
 #endif
-    for (int s = 0; s < D; ++s) mbar_init(smem_u32(&bars[s]), 1);
+  }
+#pragma unroll 1
+  for (int s = tid; s < D; s += THREADS) {   // each thread fences the barriers it initialised
+    mbar_init(smem_u32(&bars[s]), 1);
     fence_mbar_init();
   }
   if (C > 1) cluster.sync();   // peers' control blocks are ready before anyone touches them remotely
@@ -797,6 +857,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
     if (nb > 1) {
       const uint32_t unb = static_cast<uint32_t>(nb);
       pa = static_cast<uint32_t>((static_cast<uint64_t>(unb) * 618u + 500u) / 1000u) | 1u;
+#pragma unroll 1
       for (;;) {
         uint32_t a = pa, b = unb;
         while (b) { const uint32_t t = a % b; a = b; b = t; }
@@ -809,20 +870,14 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
       pc = static_cast<uint32_t>((h >> 29) % unb);
     }
     auto issue = [&](int j) {
-      const uint32_t m = static_cast<uint32_t>((static_cast<uint64_t>(pa) * static_cast<uint32_t>(j) + pc) %
-                                               static_cast<uint32_t>(nb));
-      const int64_t e0 = lo + static_cast<int64_t>(m) * B;
-      const int64_t ce = min(static_cast<int64_t>(B), hi - e0);
-      const uint32_t bytes = static_cast<uint32_t>((ce * E::kBytes + 15) & ~static_cast<int64_t>(15));
-      const int s = j % D;
-      blk_off[s] = static_cast<uint32_t>(e0);
-      const uint32_t bar = smem_u32(&bars[s]);
-      mbar_expect_tx(bar, bytes);
-      bulk_g2s(smem_u32(ring + static_cast<size_t>(s) * B * E::kBytes), rowp + e0 * E::kBytes, bytes, bar);
+      issue_block<DT>(j, pa, pc, nb, lo, hi, D, rowp, ring, bars, blk_off);
     };
-    {   // prologue: the first D blocks, one per thread
+    {   // prologue: the first D blocks, each issued by lane 0 of the warp that owns its stage
       const int first = min(D, nb);
-      for (int j = tid; j < first; j += THREADS) issue(j);
+#pragma unroll 1
+      for (int j = warp; j < first; j += Q) {
+        if (lane == 0) issue(j);
+      }
     }
     DSEL_EV(1);
 
@@ -845,83 +900,110 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
       // any CTA's threshold is a valid bound for the whole row: push it to the peers
       if (C > 1 && warp == 0 && lane < C && lane != crank) atomicMax(cluster.map_shared_rank(&ctl.t_w, lane), co.tw);
     };
-    static_assert(VPT * PV <= 64, "keep bits fit one 64-bit word");
     const int rounds = (nb + Q - 1) / Q;
+#pragma unroll 1
     for (int r = 0; r < rounds; ++r) {
       DSEL_TR(r, 0);
       WarpRound<DT> wr;
-      wr.j0 = r * Q + (warp * VPW) / VPB;              // first block this warp owns in the round
-      wr.nb = nb;
-      wr.D = D;
-      wr.s0 = wr.j0 % D;
-      wr.lane = lane;
+      wr.j0 = r * Q + warp;                            // the block this warp owns in the round
+      wr.owns = wr.j0 < nb;
       wr.uhi = uhi;
-      wr.boff0 = wr.boff1 = 0;
+      wr.sb = 0u;
+      wr.eb = 0u;
       const int j0 = wr.j0;
-      // ---- 1. wait for the owned blocks, then load and screen every vector ----
-#pragma unroll
-      for (int qb = 0; qb < BPW; ++qb) {
-        if (j0 + qb < nb) {   // warp-uniform
-          int st = wr.s0 + qb;
-          if (st >= D) st -= D;
+      // ---- 1. wait for the owned block ----
+      if (wr.owns) {   // warp-uniform
+        const int st = j0 % D;
 #ifdef DSEL_STATS
-          const long long w0 = clock64();
+        const long long w0 = clock64();
 #endif
-          if (!mbar_wait(smem_u32(&bars[st]), static_cast<uint32_t>(((j0 + qb) / D) & 1))) ctl.abort = 1;
+        if (!mbar_wait(smem_u32(&bars[st]), static_cast<uint32_t>((j0 / D) & 1))) ctl.abort = 1;
 #ifdef DSEL_STATS
-          st_wait += clock64() - w0;
+        st_wait += clock64() - w0;
 #endif
-          if (qb == 0) wr.boff0 = blk_off[st];
-          else wr.boff1 = blk_off[st];
-        }
+        wr.sb = static_cast<uint32_t>(st * B * E::kBytes + lane * 16);
+        wr.eb = blk_off[st] + static_cast<uint32_t>(lane * PV);
       }
+      DSEL_TR(r, 8);
       unsigned long long w = *reinterpret_cast<volatile unsigned long long*>(&ctl.t_w);
       w = w > t_own ? w : t_own;   // a peer may have raised it
-      uint32_t tk = static_cast<uint32_t>(w >> 32);
-      uint32_t ti = ~static_cast<uint32_t>(w);
-      uint32_t tv = E::bits_of_key(tk);
-      if (DT == DSEL_BF16) tv |= tv << 16;
-      uint32_t maybe_mask = 0;
-#pragma unroll
-      for (int v = 0; v < VPT; ++v) {
-        uint32_t voff, eidx;
-        if (wr.template locate<VPB>(v, voff, eidx)) {
-          const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
-          if ((eidx + PV > uhi) || screen<DT>(val, tv)) maybe_mask |= 1u << v;
-        }
-      }
-      DSEL_TR(r, 1);
-
-      // ---- 2. round 0: seed T from a histogram of the round's keys ----
+      uint32_t tk, ti;
+      uint32_t maybe_mask = 0;     // bit v: vector v may hold a survivor (or a NaN)
       if (r == 0) {
-        const SeedOut so = p.k <= 4 * THREADS
-                               ? seed_by_vector_max<DT, THREADS, VPT>(ring, wr, p.k, p.idx_bits, ctl)
-                               : seed_threshold<DT, THREADS, VPT>(ring, wr, p.k, p.idx_bits, ctl, seed_hist);
+        // ---- 2a. round 0: one pass for each vector's largest key, seed T from
+        //      those maxima, and screen with them (no second read) ----
+        // group g holds vectors g*VPG .. g*VPG + VPG - 1; gm[g] = its largest key
+        // (0 = empty: partial and NaN vectors are left out and always tested exactly)
+        uint32_t gm[SG];
+        uint32_t forced = 0u, valid = 0u;
+#pragma unroll
+        for (int g = 0; g < SG; ++g) {
+          uint32_t m = 0u;
+#pragma unroll 1
+          for (int i = 0; i < VPG; ++i) {
+            const int v = g * VPG + i;
+            const uint32_t eidx = wr.eb + static_cast<uint32_t>(v * 32 * PV);
+            if (wr.owns && eidx < uhi) {
+              valid |= 1u << v;
+              const uint4 val = *reinterpret_cast<const uint4*>(ring + wr.sb + v * 512);
+              uint32_t kx = 0u;
+              if (vec_max_key<DT>(val, kx) || eidx + PV > uhi) forced |= 1u << v;
+              else m = kx > m ? kx : m;
+            }
+          }
+          gm[g] = m;
+        }
+        DSEL_TR(r, 1);
+        SeedOut so{0ull, 0ull, false};
+        if (2 * p.k <= SG * THREADS) {
+          // the k-th largest group maximum: k distinct elements are at or above it
+          const uint32_t tkey = cta_kth_largest<THREADS, SG>(gm, p.k, ctl, seed_hist);
+          if (tkey != 0u) {   // uniform
+            so.t = make_w(tkey, 0xFFFFFFFFu);     // passes every key >= tkey
+            so.vlo = static_cast<uint64_t>(tkey) << p.idx_bits;
+            so.ok = true;
+          }
+        } else {
+          so = seed_threshold<DT, THREADS, VPT>(ring, wr, p.k, p.idx_bits, ctl, seed_hist);
+        }
+        DSEL_TR(r, 9);
         if (so.ok) {
           t_own = so.t;
           vlo = so.vlo;
-          if (so.t > w) {   // re-screen against the seeded T (flags only shrink)
-            w = so.t;
-            tk = static_cast<uint32_t>(w >> 32);
-            ti = ~static_cast<uint32_t>(w);
-            tv = E::bits_of_key(tk);
-            if (DT == DSEL_BF16) tv |= tv << 16;
-            uint32_t mm = maybe_mask, kept_flags = 0;
-            while (mm) {
-              const int v = __ffs(mm) - 1;
-              mm &= mm - 1u;
-              uint32_t voff, eidx;
-              wr.template locate<VPB>(v, voff, eidx);
-              const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
-              if ((eidx + PV > uhi) || screen<DT>(val, tv)) kept_flags |= 1u << v;
-            }
-            maybe_mask = kept_flags;
+          w = so.t > w ? so.t : w;
+        }
+        tk = static_cast<uint32_t>(w >> 32);
+        ti = ~static_cast<uint32_t>(w);
+        // a group whose largest key is below T's key holds no survivor
+        maybe_mask = forced;
+#pragma unroll
+        for (int g = 0; g < SG; ++g) {
+          if (gm[g] >= tk) maybe_mask |= (((1u << VPG) - 1u) << (g * VPG)) & valid;
+        }
+      } else {
+        // ---- 2b. later rounds: screen every vector against T ----
+        tk = static_cast<uint32_t>(w >> 32);
+        ti = ~static_cast<uint32_t>(w);
+        uint32_t tv = E::bits_of_key(tk);
+        if (DT == DSEL_BF16) tv |= tv << 16;
+#pragma unroll 2
+        for (int v = 0; v < VPT; ++v) {
+          const uint32_t eidx = wr.eb + static_cast<uint32_t>(v * 32 * PV);
+          if (wr.owns && eidx < uhi) {
+            const uint4 val = *reinterpret_cast<const uint4*>(ring + wr.sb + v * 512);
+            if ((eidx + PV > uhi) || screen<DT>(val, tv)) maybe_mask |= 1u << v;
           }
         }
+        DSEL_TR(r, 1);
       }
+      uint32_t tv = E::bits_of_key(tk);
+      if (DT == DSEL_BF16) tv |= tv << 16;
+
+      DSEL_TR(r, 7);
 
       // ---- 3. exact test of the flagged vectors (rare once T has settled) ----
-      uint64_t keepbits = 0;   // bit v*PV + e: element e of vector v survives
+      Keep128 keep;            // bit v*PV + e: element e of vector v survives
+      keep.w[0] = keep.w[1] = 0ull;
       if (__any_sync(0xffffffffu, maybe_mask != 0u)) {
 #ifdef DSEL_STATS
         if (lane == 0) atomicAdd(&ctl.st_slow_vectors, __popc(maybe_mask));
@@ -931,7 +1013,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
           const int v = __ffs(mm) - 1;
           mm &= mm - 1u;
           uint32_t voff, eidx;
-          wr.template locate<VPB>(v, voff, eidx);
+          wr.locate(v, voff, eidx);
           const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
           uint32_t cm = candidate_mask<DT>(val, tv);
           if (eidx + PV > uhi) cm &= (1u << (uhi - eidx)) - 1u;   // past hi: not this row's
@@ -946,7 +1028,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
             } else {
               const uint32_t kk = E::key(b);
               if (kk > tk || (kk == tk && idx < ti)) {
-                keepbits |= 1ull << (v * PV + e);
+                keep.set(v * PV + e);
                 const uint64_t vv = (static_cast<uint64_t>(kk) << p.idx_bits) | (idx_mask - idx);
                 vmax = vv > vmax ? vv : vmax;
               }
@@ -954,7 +1036,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
           }
         }
       }
-      int mine = __popcll(keepbits);   // survivors of this thread not yet in the buffer
+      int mine = keep.count();   // survivors of this thread not yet in the buffer
       if (r == 0) DSEL_EV(2);
       DSEL_TR(r, 2);
 
@@ -976,20 +1058,23 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
         DSEL_TR(r, 6);
         if (wcount != 0) {   // warp-uniform
           int rank = woff + warp_incl_scan(mine, lane) - mine;
-          uint64_t kb = keepbits;
-          while (kb) {
-            const int bit = __ffsll(static_cast<long long>(kb)) - 1;
-            kb &= kb - 1ull;
-            if (rank < space) {
-              const int v = bit / PV, e = bit % PV;
-              uint32_t voff, eidx;
-              wr.template locate<VPB>(v, voff, eidx);
-              const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
-              cb[cnt + rank] = static_cast<bits_t>(vec_elem_dyn<DT>(val, e));
-              ci[cnt + rank] = eidx + e;
-              keepbits &= ~(1ull << bit);
+#pragma unroll
+          for (int wi = 0; wi < 2; ++wi) {
+            uint64_t kb = keep.w[wi];
+            while (kb) {
+              const int bit = wi * 64 + __ffsll(static_cast<long long>(kb)) - 1;
+              kb &= kb - 1ull;
+              if (rank < space) {
+                const int v = bit / PV, e = bit % PV;
+                uint32_t voff, eidx;
+                wr.locate(v, voff, eidx);
+                const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
+                cb[cnt + rank] = static_cast<bits_t>(vec_elem_dyn<DT>(val, e));
+                ci[cnt + rank] = eidx + e;
+                keep.clr(bit);
+              }
+              ++rank;
             }
-            ++rank;
           }
         }
 #ifdef DSEL_STATS
@@ -1006,29 +1091,28 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
         w = w > t_own ? w : t_own;
         tk = static_cast<uint32_t>(w >> 32);
         ti = ~static_cast<uint32_t>(w);
-        uint64_t kb = keepbits;
-        while (kb) {
-          const int bit = __ffsll(static_cast<long long>(kb)) - 1;
-          kb &= kb - 1ull;
-          const int v = bit / PV, e = bit % PV;
-          uint32_t voff, eidx;
-          wr.template locate<VPB>(v, voff, eidx);
-          const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
-          const uint32_t kk = E::key(vec_elem_dyn<DT>(val, e));
-          if (!(kk > tk || (kk == tk && eidx + e < ti))) keepbits &= ~(1ull << bit);
+#pragma unroll
+        for (int wi = 0; wi < 2; ++wi) {
+          uint64_t kb = keep.w[wi];
+          while (kb) {
+            const int bit = wi * 64 + __ffsll(static_cast<long long>(kb)) - 1;
+            kb &= kb - 1ull;
+            const int v = bit / PV, e = bit % PV;
+            uint32_t voff, eidx;
+            wr.locate(v, voff, eidx);
+            const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
+            const uint32_t kk = E::key(vec_elem_dyn<DT>(val, e));
+            if (!(kk > tk || (kk == tk && eidx + e < ti))) keep.clr(bit);
+          }
         }
-        mine = __popcll(keepbits);
+        mine = keep.count();
       }
       DSEL_TR(r, 4);
-      // ---- 5. refill this warp's stages: no other warp reads them ----
+      // ---- 5. refill this warp's stage: no other warp reads it ----
       __syncwarp();
       if (lane == 0) {
         fence_proxy_async();   // our reads of the stages come before the copies that overwrite them
-#pragma unroll
-        for (int qb = 0; qb < BPW; ++qb) {
-          const int j = j0 + qb + D;
-          if (j < nb) issue(j);
-        }
+        if (j0 + D < nb) issue(j0 + D);
       }
 #ifdef DSEL_STATS
       ++st_rounds;
@@ -1053,6 +1137,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
     // this CTA's shared memory can go away.
     __syncthreads();
     if (ctl.abort && tid == 0) {
+#pragma unroll 1
       for (int j = max(0, nb - D); j < nb; ++j) mbar_wait(smem_u32(&bars[j % D]), (j / D) & 1);
     }
 #ifdef DSEL_STATS
@@ -1082,6 +1167,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_stream_kernel(const __grid_co
     st[5] = static_cast<unsigned long long>(ctl.st_slow_vectors);
     st[6] = static_cast<unsigned long long>(st_rounds);
     st[7] = 0;
+#pragma unroll 1
     for (int i = 0; i < 6; ++i) st[8 + i] = static_cast<unsigned long long>(st_ev[i]);
     st[14] = static_cast<unsigned long long>(st_wait);
     st[15] = static_cast<unsigned long long>(clock64() - st_t0);
@@ -1117,6 +1203,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_merge_kernel(const __grid_con
 
   bool bad_end;
   const int64_t n = row_length(p, row, &bad_end);
+#pragma unroll 1
   for (int i = tid; i < 3 * kBins; i += THREADS) (&ctl.hist[0][0])[i] = 0;
   if (tid == 0) {
     ctl.t_w = 0ull;
@@ -1137,6 +1224,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_merge_kernel(const __grid_con
     const int2* meta = p.ws_meta + row * p.groups;
     if (tid == 0) {
       int acc = 0, nan = 0;
+#pragma unroll 1
       for (int gg = 0; gg < p.groups; ++gg) {
         const int2 mt = meta[gg];
         pref[gg] = acc;
@@ -1155,6 +1243,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_merge_kernel(const __grid_con
     if (!nan) {
       const uint2* src = p.ws_pairs + row * p.groups * static_cast<int64_t>(p.k);
       const uint32_t idx_mask = mask_bits(p.idx_bits);
+#pragma unroll 1
       for (int i = a + tid; i < b; i += THREADS) {
         int lo = 0, hi = p.groups - 1;   // last group whose prefix <= i
         while (lo < hi) {

@@ -2,9 +2,12 @@
 //
 // The pages fix only B = B2 = 1024 for k = 512 ("DeepSeek releases DeepSelect, a
 // TopK kernel for sparse attention and sampling", method paragraph) and say both
-// should sit "on the order of k"; everything else here is this library's choice
-// for a 148-SM B200:
-//   * one CTA per row while there are at least as many rows as SMs;
+// should sit "on the order of k"; B2 follows them, B is one warp's share of a
+// round (4096 bf16 / 1024 f32 elements, see block_elems_for), and everything
+// else here is this library's choice for a 148-SM B200:
+//   * one CTA per row while there are at least as many rows as SMs; when rows
+//     are also short (at most two 128-thread rounds), a 128-thread CTA, several
+//     per SM, each with at most one round of blocks in flight;
 //   * otherwise each row is cut into S contiguous slices, one CTA each, grouped in
 //     thread-block clusters of C CTAs that share the threshold and merge through
 //     distributed shared memory; rows too long for one cluster (S > max_cluster)
@@ -38,13 +41,14 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
 
   const int eb = elem_bytes(dtype);
   dsel_plan_t p{};
-  p.threads = kThreads;
-  p.block = kBlockElems;
-  p.round = round_elems(dtype);
+  const bool short_rows = rows >= num_sms && row_stride <= 2 * int64_t(round_elems(dtype, kThreadsShort));
+  p.threads = short_rows ? kThreadsShort : kThreads;
+  p.block = block_elems(dtype);
+  p.round = round_elems(dtype, p.threads);
   p.b2 = k <= 1024 ? 1024 : std::min(k, 2048);
   // k + B2 + slack; a round's survivors beyond that wait in registers until a
   // compaction makes room, so the round may be larger than the slack
-  p.capacity = int(round_up(std::max<int64_t>(k + p.b2 + append_slack(k), next_pow2(k)), 32));
+  p.capacity = int(round_up(std::max<int64_t>(k + p.b2 + append_slack(k, p.threads), next_pow2(k)), 32));
   p.idx_bits = ceil_log2_u64(uint64_t(row_stride));
 
   // Row split.
@@ -71,7 +75,9 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
   const int64_t per_stage = int64_t(p.block) * eb + 8 + 4;
   int64_t stages = (int64_t(smem_optin) - base) / per_stage;
   stages = std::min<int64_t>(stages, kMaxStages);
-  if (nb_max <= stages) {
+  if (short_rows) {
+    stages = std::min(nb_max, per_round);    // one round in flight: keeps several CTAs per SM
+  } else if (nb_max <= stages) {
     stages = nb_max;                         // the whole slice in flight at once, no refills
   } else {
     stages = stages / per_round * per_round; // refills go to the warp that owns the stage

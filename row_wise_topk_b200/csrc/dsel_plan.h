@@ -8,15 +8,24 @@
 namespace dsel {
 
 // Compile-time CTA shapes.  The streaming kernel is instantiated for exactly
-// these (dtype, threads) pairs; the planner only ever returns one of them.
+// these (dtype, threads) pairs; the planner only ever returns one of them:
+// 512 threads, one CTA per SM, for long rows and split rows; 128 threads for
+// many short rows, so that several rows share an SM and one CTA's loads overlap
+// another's selection.
 constexpr int kThreads = 512;
+constexpr int kThreadsShort = 128;
 constexpr int kVecBytes = 16;                 // one 128-bit shared-memory load per vector
-constexpr int kVecsPerThread = 8;             // vectors each thread screens per round (whole blocks per warp)
+// Vectors each thread screens per round (a warp owns whole blocks): 16 for bf16
+// (a 64K-element round, the whole slice of a 131,072-position row split in two),
+// 8 for f32 (16K elements, so that two rounds fit the ring for double buffering).
+constexpr int vecs_per_thread_for(int eb) { return eb == 2 ? 16 : 8; }
 
 // Candidate-buffer slots beyond k + B2.  A round's survivors that do not fit
 // wait until a compaction makes room, so this need not cover a whole round.
-inline int append_slack(int k) { return k <= 1024 ? 4096 : 2048; }
-constexpr int kBlockElems = 1024;             // B: the pages' setting for k = 512
+inline int append_slack(int k, int threads) {
+  if (threads == kThreadsShort) return 1024;
+  return k <= 1024 ? 4096 : 2048;
+}
 constexpr int kStrideReq = 16;                // row_stride multiple (elements)
 constexpr int kMaxStages = 128;               // ring depth cap (one mbarrier per stage)
 constexpr int kMinSliceElems = 8192;          // smallest row share worth its own CTA
@@ -28,8 +37,16 @@ constexpr int kMaxGroups = 255;               // clusters per row (merge keeps o
 inline int elem_bytes(int dtype) { return dtype == DSEL_BF16 ? 2 : 4; }
 
 // Elements a CTA filters between two checks of the candidate buffer.
-constexpr int round_elems_for(int eb) { return kThreads * kVecsPerThread * (kVecBytes / eb); }
-inline int round_elems(int dtype) { return round_elems_for(elem_bytes(dtype)); }
+constexpr int round_elems_for(int eb, int threads) { return threads * vecs_per_thread_for(eb) * (kVecBytes / eb); }
+inline int round_elems(int dtype, int threads) { return round_elems_for(elem_bytes(dtype), threads); }
+
+// B, elements per contiguous block (the unit of the random visiting order and of
+// one bulk copy): one warp's share of a round, 32 lanes x vectors per thread, so
+// each warp issues, and waits on, exactly one copy per round.  4096 for bf16
+// (8 KB), 1024 for f32 (4 KB).  The pages set B = 1024 for k = 512; bf16 takes
+// the larger block so that a CTA issues a quarter as many copies.
+constexpr int block_elems_for(int eb) { return 32 * vecs_per_thread_for(eb) * (kVecBytes / eb); }
+inline int block_elems(int dtype) { return block_elems_for(elem_bytes(dtype)); }
 
 inline int ceil_log2_u64(uint64_t v) {   // smallest b with 2^b >= v (v >= 1)
   int b = 0;

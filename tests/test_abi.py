@@ -100,12 +100,19 @@ def test_plan_invariants(dtype, rows, stride, k):
     assert st == 0
     eb = 2 if dtype == T.DSEL_BF16 else 4
     assert p["smem_bytes"] <= PEAK["smem_optin"]
-    assert p["capacity"] >= k + p["b2"] + (4096 if k <= 1024 else 2048)
+    slack = 1024 if p["threads"] == 128 else (4096 if k <= 1024 else 2048)
+    assert p["capacity"] >= k + p["b2"] + slack
     assert p["capacity"] >= 1 << (k - 1).bit_length()          # room for the bitonic padding
     q = p["round"] // p["block"]
     slice_ = -(-(-(-stride // (p["cluster"] * p["groups"]))) // 16) * 16
     nb_max = -(-slice_ // p["block"])
     assert p["stages"] == nb_max or (p["stages"] % q == 0 and p["stages"] < nb_max)
+    assert p["threads"] in (128, 512)
+    assert p["round"] == p["threads"] * (16 if dtype == T.DSEL_BF16 else 8) * (16 // eb)
+    if p["threads"] == 128:   # short rows: one CTA per row, one round in flight, several CTAs per SM
+        assert rows >= PEAK["num_sms"] and stride <= 2 * p["round"]
+        assert (p["cluster"], p["groups"]) == (1, 1) and p["stages"] <= q
+        assert p["smem_bytes"] <= 232448 // 2
     assert p["round"] % p["block"] == 0 and (p["block"] * eb) % 16 == 0
     assert 1 <= p["cluster"] <= PEAK["max_cluster"]
     assert p["groups"] >= 1 and p["groups"] * k <= 8 * p["capacity"]
@@ -120,8 +127,10 @@ def test_plan_invariants(dtype, rows, stride, k):
 
 
 def test_plan_splits():
-    # many rows: one CTA per row
-    assert T.dsel_plan(T.DSEL_BF16, 4096, 16384, 512, **PEAK)[1]["cluster"] == 1
+    # many rows: one CTA per row; short ones get the 128-thread shape
+    p = T.dsel_plan(T.DSEL_BF16, 4096, 16384, 512, **PEAK)[1]
+    assert p["cluster"] == 1 and p["threads"] == 128
+    assert T.dsel_plan(T.DSEL_F32, 256, 129280, 4096, **PEAK)[1]["threads"] == 512
     # 64 indexer rows: two CTAs per row
     p = T.dsel_plan(T.DSEL_BF16, 64, 131072, 512, **PEAK)[1]
     assert (p["cluster"], p["groups"]) == (2, 1)

@@ -147,6 +147,32 @@ def test_torch_wrapper_bf16():
 # --------------------------------------------------------------------------- #
 # the workload families at full size (the bench's launch configuration)
 # --------------------------------------------------------------------------- #
+# --------------------------------------------------------------------------- #
+# the 128-thread shape: at least as many rows as SMs, rows of one or two rounds
+# --------------------------------------------------------------------------- #
+SHORT = [
+    # (seed, dtype, rows, stride, k, dist, order)
+    (301, "bf16", 160, 32768, 1, "normal", 1),
+    (302, "bf16", 160, 32768, 512, "ties", 0),
+    (303, "bf16", 150, 16384, 4096, "normal", 1),
+    (304, "bf16", 300, 2048, 512, "ties", 1),
+    (305, "f32", 150, 8192, 64, "normal", 2),
+    (306, "f32", 160, 8192, 2000, "ties", 1),
+    (307, "f32", 200, 4096, 4096, "normal", 0),
+    (308, "f32", 149, 6144, 700, "ascending", 1),
+]
+
+
+@pytest.mark.parametrize("seed,dtype,rows,stride,k,dist,order", SHORT)
+def test_short_row_shape(seed, dtype, rows, stride, k, dist, order):
+    st, plan = T.dsel_plan(T.DSEL_BF16 if dtype == "bf16" else T.DSEL_F32, rows, stride, k,
+                           num_sms=torch.cuda.get_device_properties(0).multi_processor_count)
+    assert st == 0 and plan["threads"] == 128, "the case must use the 128-thread shape"
+    w = W.random_small(seed, dtype, rows, stride, k, dist=dist, with_end=(seed % 2 == 0),
+                       end_lo=0, sorted_index=1, return_value=1, index_dtype="i64")
+    check(w, order=order)
+
+
 def test_pr1_duplicates_full():
     check(W.pr1_duplicates())
 
