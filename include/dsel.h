@@ -123,7 +123,7 @@ typedef struct {
   int32_t b2;            /* B2: the buffer is cut back to k when it holds k + B2 */
   int32_t round;         /* elements the CTA filters between two buffer checks */
   int32_t capacity;      /* candidate-buffer slots per CTA: k + B2 + slack (512 threads: 4096, or
-                            2048 for k > 1024; 128 threads: 1024), at least next_pow2(k) */
+                            2048 for k > 1024; 128 threads: 1024), at least next_pow2(k) and 4096 */
   int32_t stages;        /* blocks kept in flight per CTA (shared-memory ring) */
   int32_t idx_bits;      /* bits of the in-row index used to break ties */
   int32_t smem_bytes;    /* dynamic shared memory per CTA */

@@ -21,6 +21,7 @@
 
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "../../include/dsel.h"
@@ -32,6 +33,7 @@ namespace dsel {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // bounded waits: 2 s
 constexpr uint32_t kSuspendHintNs = 20000;          // a waiting warp sleeps (woken at completion)
 constexpr int kDigitBits = 8;
+constexpr int kTieMax = 128;                  // radix select: largest bucket finished by direct ranking
 constexpr int kBins = 1 << kDigitBits;
 
 __device__ int g_device_status;                    // DSEL_ERR_DEVICE_TIMEOUT when a wait gave up
@@ -250,6 +252,8 @@ struct __align__(16) Ctl {
   int hb;                       // index of a histogram that is all zero
   int x_cnt, x_nan, x_kept;     // exchanged with peers in the final phase
   int sel_flag;
+  int tie_n;                    // radix select: members of a small bucket gathered so far
+  unsigned long long tie_v;     // radix select: the selected radix word of that bucket
   int wc[2][kWarpsMax];         // per-warp counts, by round parity
   int wm[kWarpsMax];            // per-warp counts (compaction movers)
   int hist[3][kBins];
@@ -261,6 +265,10 @@ struct __align__(16) Ctl {
   int st_slow_vectors;
 #endif
 };
+
+static_assert(offsetof(Ctl, hsum) % 16 == 0 && sizeof(Ctl::hsum) >= kTieMax * 8,
+              "the radix select's small-bucket list fits hsum");
+static_assert(offsetof(Ctl, hist) % 16 == 0 && (kBins * 4) % 16 == 0, "histograms are read as int4");
 
 // Composite threshold word: larger means "ranks earlier".
 __device__ __forceinline__ unsigned long long make_w(uint32_t key, uint32_t idx) {
@@ -313,6 +321,23 @@ __device__ __forceinline__ int warp_prefix_of(const int* wc, int warp, int lane,
   return mine;
 }
 
+// Sum of lane `lane`'s contiguous chunk of N4 int4s, h4[base4 + lane * N4 ..
+// + N4), read in a rotated order: with chunks of 2^m int4s the plain order puts
+// up to 32 lanes on the same banks, the rotation keeps 8 lanes per wavefront
+// (the minimum for 128-bit loads).  h4 must be 16-byte aligned.
+template <int N4>
+__device__ __forceinline__ int chunk_sum4(const int4* h4, int base4, int lane) {
+  static_assert(N4 == 1 || N4 == 2 || N4 == 4 || N4 == 8, "chunk of 1, 2, 4 or 8 int4s");
+  const int rot = (lane / (8 / N4)) % N4;
+  int s = 0;
+#pragma unroll
+  for (int j = 0; j < N4; ++j) {
+    const int4 q = h4[base4 + lane * N4 + ((j + rot) % N4)];
+    s += q.x + q.y + q.z + q.w;
+  }
+  return s;
+}
+
 template <bool CLUSTER>
 __device__ __forceinline__ void cta_or_cluster_sync(cg::cluster_group& cluster) {
   if (CLUSTER) cluster.sync();
@@ -344,6 +369,7 @@ __device__ __noinline__ SelResult radix_select(const typename Elem<DT>::bits_t* 
   int need = need0;
   int hb = ctl.hb;
   int kept = need0;
+  if (!CLUSTER && tid == 0) ctl.tie_n = 0;   // ordered before any use by the first pass's barrier
   while (true) {
     const int dbits = min(kDigitBits, total_bits - depth);
     const int shift = total_bits - depth - dbits;
@@ -383,13 +409,22 @@ __device__ __noinline__ SelResult radix_select(const typename Elem<DT>::bits_t* 
       H = ctl.hsum;
     }
     // every warp: bins from the top, 8 per lane, find the bucket holding the need-th
-    int c[kBins / 32];
+    // lane l holds bins kBins-1-8l down to kBins-8-8l (c[0] the highest), read as
+    // two int4s whose order alternates between lane groups (no bank conflicts)
+    static_assert(kBins == 256, "two int4s of bins per lane");
+    int c[8];
+    {
+      const int4* H4 = reinterpret_cast<const int4*>(H);
+      const int sw = (lane >> 2) & 1;
+      const int4 qa = H4[62 - 2 * lane + sw];
+      const int4 qb = H4[63 - 2 * lane - sw];
+      const int4 lo = sw ? qb : qa, hi = sw ? qa : qb;   // bins 248-8l.. and 252-8l..
+      c[0] = hi.w; c[1] = hi.z; c[2] = hi.y; c[3] = hi.x;
+      c[4] = lo.w; c[5] = lo.z; c[6] = lo.y; c[7] = lo.x;
+    }
     int s = 0;
 #pragma unroll
-    for (int j = 0; j < kBins / 32; ++j) {
-      c[j] = H[kBins - 1 - (lane * (kBins / 32) + j)];
-      s += c[j];
-    }
+    for (int j = 0; j < 8; ++j) s += c[j];
     const int incl = warp_incl_scan(s, lane);
     const int excl = incl - s;
     const bool mine = excl < need && need <= incl;
@@ -418,6 +453,40 @@ __device__ __noinline__ SelResult radix_select(const typename Elem<DT>::bits_t* 
     hb = hb == 2 ? 0 : hb + 1;
     kept = need0 - need + bucket;
     if (bucket - need <= slack || depth == total_bits) break;
+    if (!CLUSTER && slack == 0 && bucket <= kTieMax) {
+      // Small bucket (typically equal keys at the boundary): rank its members by
+      // their whole radix word, which is unique, instead of more digit passes.
+      unsigned long long* lst = reinterpret_cast<unsigned long long*>(ctl.hsum);
+      const int sh = total_bits - depth;
+#pragma unroll 1
+      for (int i0 = 0; i0 < cnt; i0 += THREADS) {   // same trip count in every thread
+        const int i = i0 + tid;
+        uint64_t v = 0;
+        bool in = false;
+        if (i < cnt) {
+          v = make_v<DT>(cb[i], ci[i], idx_bits, idx_mask);
+          in = (v >> sh) == prefix;
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, in);
+        int base = 0;
+        if (lane == 0 && bal != 0u) base = atomicAdd(&ctl.tie_n, __popc(bal));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (in) lst[base + __popc(bal & ((1u << lane) - 1u))] = v;
+      }
+      __syncthreads();
+      if (tid < bucket) {   // the member with need - 1 larger words is the need-th
+        const unsigned long long vj = lst[tid];
+        int r = 0;
+#pragma unroll 4
+        for (int i = 0; i < bucket; ++i) r += lst[i] > vj ? 1 : 0;
+        if (r == need - 1) ctl.tie_v = vj;
+      }
+      __syncthreads();
+      prefix = ctl.tie_v;
+      depth = total_bits;
+      kept = need0;
+      break;
+    }
   }
   if (tid == 0) ctl.hb = hb;   // read again only after later barriers
   return {prefix, depth, kept};

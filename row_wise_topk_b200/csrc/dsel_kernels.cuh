@@ -43,6 +43,17 @@ constexpr int kTraceSize = kTraceWarps * kTraceRounds * kTraceEvents;
 __device__ long long g_trace[kTraceSize];
 #endif
 
+// Per-warp marks inside a phase (CTA 0, lane 0 of each warp), stats builds
+// only: absolute clocks in trace row kTraceRounds - 2.
+__device__ __forceinline__ void trace_mark(int e) {
+#ifdef DSEL_STATS
+  if (blockIdx.x == 0 && (threadIdx.x & 31) == 0 && (threadIdx.x >> 5) < kTraceWarps)
+    g_trace[((threadIdx.x >> 5) * kTraceRounds + kTraceRounds - 2) * kTraceEvents + e] = clock64();
+#else
+  (void)e;
+#endif
+}
+
 // Final-phase timeline of CTA 0 (thread 0), stats builds only: absolute clocks
 // in trace row kTraceRounds - 1 of warp 0; slot kTraceEvents - 1 holds the
 // kernel-start clock.
@@ -178,21 +189,59 @@ __device__ __forceinline__ void emit_nan(const KParams& p, int64_t row, int g, b
 }
 
 // ---------------------------------------------------------------------------
-// Order the m kept entries and write them at output slots off .. off + m - 1.
-// Ascending index, when the bitmap of the candidates' index span fits in
-// `scratch` (the idle bulk-copy ring): each entry's slot is the number of kept
-// indices below it, from a prefix popcount over the bitmap.  Otherwise (and
-// for value order) a bitonic sort in shared memory, then a plain write.
+// Write the kept entries of the list cb/ci[0, n) at output slots off ..
+// off + m - 1.  The kept ones are those whose radix word has top sel.depth bits
+// >= sel.prefix (all of them when sel.depth is 0); there are m = sel.kept.
+//   * any order: each warp takes slots for its kept entries with one shared
+//     atomic per 32 entries;
+//   * ascending index, when the bitmap of the candidates' index span fits in
+//     `scratch` (the idle bulk-copy ring): each entry's slot is the number of
+//     kept indices below it, from a prefix popcount over the bitmap;
+//   * otherwise (and for value order) the kept entries are compacted to the
+//     front, sorted by a bitonic network and written in order.
 // ---------------------------------------------------------------------------
 template <int DT, int THREADS>
 __device__ __noinline__ void finish_sorted(const KParams& p, int64_t row, int g, bool to_workspace,
-                                           typename Elem<DT>::bits_t* cb, uint32_t* ci, int m, int sort_mode,
-                                           Ctl& ctl, unsigned char* scratch, uint32_t scratch_bytes,
-                                           uint32_t span_lo, uint32_t span_len, int off, int total,
-                                           bool write_meta) {
+                                           typename Elem<DT>::bits_t* cb, uint32_t* ci, int n, SelResult sel,
+                                           int sort_mode, Ctl& ctl, uint32_t* holes, unsigned char* scratch,
+                                           uint32_t scratch_bytes, uint32_t span_lo, uint32_t span_len, int off,
+                                           int total, bool write_meta) {
   using bits_t = typename Elem<DT>::bits_t;
   constexpr int NW = THREADS / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t idx_mask = mask_bits(p.idx_bits);
+  const int shv = Elem<DT>::kKeyBits + p.idx_bits - sel.depth;   // < 64
+  auto keep = [&](int i) -> bool {
+    return (make_v<DT>(cb[i], ci[i], p.idx_bits, idx_mask) >> shv) >= sel.prefix;
+  };
+  const int64_t obase = row * p.k + off;
+  uint2* wsd = to_workspace ? p.ws_pairs + (row * p.groups + g) * static_cast<int64_t>(p.k) + off : nullptr;
+  auto put = [&](int slot, int i) {
+    if (to_workspace) {
+      wsd[slot] = make_uint2(ci[i], static_cast<uint32_t>(cb[i]));
+    } else {
+      if (p.index_i64) static_cast<int64_t*>(p.indices_out)[obase + slot] = static_cast<int64_t>(ci[i]);
+      else static_cast<int32_t*>(p.indices_out)[obase + slot] = static_cast<int32_t>(ci[i]);
+      if (p.return_value) static_cast<bits_t*>(p.values_out)[obase + slot] = cb[i];
+    }
+  };
+  if (sort_mode == 0) {
+    if (tid == 0) ctl.sel_flag = 0;   // next free slot
+    __syncthreads();
+    const uint32_t below = (1u << lane) - 1u;
+#pragma unroll 1
+    for (int i0 = 0; i0 < n; i0 += THREADS) {   // same trip count in every thread
+      const int i = i0 + tid;
+      const bool kp = i < n && keep(i);
+      const unsigned bal = __ballot_sync(0xffffffffu, kp);
+      int base = 0;
+      if (lane == 0 && bal != 0u) base = atomicAdd(&ctl.sel_flag, __popc(bal));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (kp) put(base + __popc(bal & below), i);
+    }
+    if (to_workspace && write_meta && tid == 0) p.ws_meta[row * p.groups + g] = make_int2(total, 0);
+    return;
+  }
   const uint32_t words = (span_len + 31u) / 32u;
   if (sort_mode == 1 && scratch != nullptr && 8ull * words <= scratch_bytes) {
     uint32_t* bm = reinterpret_cast<uint32_t*>(scratch);
@@ -201,9 +250,11 @@ __device__ __noinline__ void finish_sorted(const KParams& p, int64_t row, int g,
     for (uint32_t i = tid; i < words; i += THREADS) bm[i] = 0u;
     __syncthreads();
 #pragma unroll 1
-    for (int i = tid; i < m; i += THREADS) {
-      const uint32_t d = ci[i] - span_lo;
-      atomicOr(&bm[d >> 5], 1u << (d & 31u));
+    for (int i = tid; i < n; i += THREADS) {
+      if (keep(i)) {
+        const uint32_t d = ci[i] - span_lo;
+        atomicOr(&bm[d >> 5], 1u << (d & 31u));
+      }
     }
     __syncthreads();
     // prefix popcount: warp w walks its contiguous share of words, lanes side by side
@@ -229,41 +280,30 @@ __device__ __noinline__ void finish_sorted(const KParams& p, int64_t row, int g,
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
     __syncthreads();
-    const int64_t obase = row * p.k + off;
-    uint2* wsd = to_workspace ? p.ws_pairs + (row * p.groups + g) * static_cast<int64_t>(p.k) + off : nullptr;
 #pragma unroll 1
-    for (int i = tid; i < m; i += THREADS) {
-      const uint32_t idx = ci[i];
-      const uint32_t d = idx - span_lo;
-      const int rank = static_cast<int>(wp[d >> 5]) + __popc(bm[d >> 5] & ((1u << (d & 31u)) - 1u));
-      if (to_workspace) {
-        wsd[rank] = make_uint2(idx, static_cast<uint32_t>(cb[i]));
-      } else {
-        if (p.index_i64) static_cast<int64_t*>(p.indices_out)[obase + rank] = static_cast<int64_t>(idx);
-        else static_cast<int32_t*>(p.indices_out)[obase + rank] = static_cast<int32_t>(idx);
-        if (p.return_value) static_cast<bits_t*>(p.values_out)[obase + rank] = cb[i];
+    for (int i = tid; i < n; i += THREADS) {
+      if (keep(i)) {
+        const uint32_t d = ci[i] - span_lo;
+        put(static_cast<int>(wp[d >> 5]) + __popc(bm[d >> 5] & ((1u << (d & 31u)) - 1u)), i);
       }
     }
     if (to_workspace && write_meta && tid == 0) p.ws_meta[row * p.groups + g] = make_int2(total, 0);
     return;
   }
+  const int m = sel.depth == 0 ? n : holes_compact<DT, THREADS>(cb, ci, n, sel.kept, sel, p.idx_bits, ctl, holes);
   sort_kept<DT, THREADS>(cb, ci, m, sort_mode);
   emit<DT, THREADS>(p, row, g, to_workspace, off, m, total, write_meta, cb, ci);
 }
 
-// ---------------------------------------------------------------------------
-// Final phase, shared by the streaming and merge kernels.  The cluster's CTAs
-// together hold a superset of the row's (or row part's) best entries; exactly
-// min(k, total) of them are kept, optionally sorted, and written to the output
-// (or, for a split row, to the workspace).
-//   * one CTA: local exact select;
-//   * gather (cluster * k fits one buffer): each CTA keeps its own best k, rank 0
-//     copies the peers' lists over distributed shared memory and selects again;
-//   * otherwise: a cluster-wide radix select on summed histograms, each CTA
-//     writing its share (slices are in index order, so per-CTA index sorts
-//     concatenate into a sorted row); value order gathers on rank 0 at the end.
-//   sort_mode 0: none, 1: ascending index, 2: value descending.
-// ---------------------------------------------------------------------------
+// The best min(k, n) entries of cb/ci[0, n) (all within [vlo, vhi]), as a
+// selection result for finish_sorted (depth 0: all of them).
+template <int DT, int THREADS>
+__device__ __forceinline__ SelResult select_best(const KParams& p, typename Elem<DT>::bits_t* cb, uint32_t* ci, int n,
+                                                 uint64_t vlo, uint64_t vhi, Ctl& ctl, cg::cluster_group& cluster) {
+  if (n <= p.k) return SelResult{0ull, 0, n};
+  return radix_select<DT, THREADS, false>(cb, ci, n, p.k, 0, p.idx_bits, vlo, vhi, ctl, cluster);
+}
+
 template <int DT, int THREADS>
 __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, typename Elem<DT>::bits_t* cb,
                          uint32_t* ci, uint32_t* holes, Ctl& ctl, cg::cluster_group& cluster,
@@ -287,10 +327,10 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
       emit_nan<DT, THREADS>(p, row, g, to_workspace);
       return;
     }
-    const int m = local_select<DT, THREADS>(cb, ci, cnt, p.k, p.idx_bits, vlo, vhi, ctl, holes, cluster);
+    const SelResult sel = select_best<DT, THREADS>(p, cb, ci, cnt, vlo, vhi, ctl, cluster);
     trace_final(5);
-    finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, m, sort_mode, ctl, ring, ring_bytes, span_lo,
-                               span_len, 0, m, true);
+    finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, cnt, sel, sort_mode, ctl, holes, ring, ring_bytes,
+                               span_lo, span_len, 0, sel.kept, true);
     trace_final(6);
     return;
   }
@@ -354,10 +394,10 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
     }
     __syncthreads();   // the gathered list is complete
     trace_final(3);
-    const int mm = local_select<DT, THREADS>(cb, ci, off, p.k, p.idx_bits, lo, hi, ctl, holes, cluster);
+    const SelResult sel = select_best<DT, THREADS>(p, cb, ci, off, lo, hi, ctl, cluster);
     trace_final(5);
-    finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, mm, sort_mode, ctl, ring, ring_bytes, span_lo,
-                               span_len, 0, mm, true);
+    finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, off, sel, sort_mode, ctl, holes, ring, ring_bytes,
+                               span_lo, span_len, 0, sel.kept, true);
     trace_final(6);
     return;
   }
@@ -420,7 +460,8 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
         off += mr;
       }
       __syncthreads();
-      finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, off, 2, ctl, nullptr, 0u, 0u, 0u, 0, off, true);
+      finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, off, SelResult{0ull, 0, off}, 2, ctl, holes, nullptr,
+                                 0u, 0u, 0u, 0, off, true);
     }
     return;
   }
@@ -428,8 +469,8 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) off += __shfl_xor_sync(0xffffffffu, off, o);
   // each CTA orders its own share (its slice is an index range of its own)
-  finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, m, sort_mode, ctl, ring, ring_bytes, span_lo,
-                             span_len, off, need, crank == 0);
+  finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, m, SelResult{0ull, 0, m}, sort_mode, ctl, holes, ring,
+                             ring_bytes, span_lo, span_len, off, need, crank == 0);
 }
 
 // Survivor bits of one thread in one round (up to 128 elements), kept in two
@@ -492,17 +533,17 @@ __device__ __forceinline__ bool vec_max_key(const uint4 x, uint32_t& key) {
   }
 }
 
-// Largest key t such that at least k of the CTA's non-empty group maxima
-// (gm != 0) are >= t, or 0 when the CTA holds fewer than k of them.  Bisection
-// over the bits below the common prefix of the smallest and largest maximum,
-// three bits per step: every warp counts its maxima at the seven candidate
-// thresholds, the per-warp counts meet in `scratch` (2 x NW x 8 ints, double
-// buffered so that one barrier per step suffices), and every warp takes the
-// same decision.
+// A key t such that at least k of the CTA's non-empty group maxima (gm != 0)
+// are >= t, close below the k-th largest of them; 0 when the CTA holds fewer
+// than k.  One histogram pass: the maxima fall into 1024 bins spread evenly
+// over [kmin, kmax] (bins of 2^sh keys, sh = 0 when the span is below 1024),
+// and t is the lower edge of the bin that holds the k-th largest.  `hist` has
+// 1024 zeroed ints, 16-byte aligned.  Two barriers; no warp reduction in a loop.
 template <int THREADS, int G>
-__device__ __forceinline__ uint32_t cta_kth_largest(const uint32_t (&gm)[G], int k, Ctl& ctl, int* scratch) {
+__device__ __forceinline__ uint32_t cta_kth_largest(const uint32_t (&gm)[G], int k, Ctl& ctl, int* hist) {
   constexpr int NW = THREADS / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  trace_mark(0);
   int nz = 0;
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll
@@ -521,42 +562,54 @@ __device__ __forceinline__ uint32_t cta_kth_largest(const uint32_t (&gm)[G], int
     ctl.wv[warp] = (static_cast<unsigned long long>(kmax) << 32) | kmin;
   }
   __syncthreads();   // ctl.wm / wv are written again only after later barriers
-  nz = static_cast<int>(__reduce_add_sync(0xffffffffu, lane < NW ? static_cast<unsigned>(ctl.wm[lane]) : 0u));
-  if (nz < k) return 0u;   // uniform
-  const unsigned long long wv = lane < NW ? ctl.wv[lane] : 0xFFFFFFFFull;
-  kmin = __reduce_min_sync(0xffffffffu, static_cast<uint32_t>(wv));
-  kmax = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(wv >> 32));
-  int b = 32 - __clz(kmin ^ kmax);   // bits below the common prefix
-  uint32_t pre = kmax & ~mask_bits(b);
-  int par = 0;
-#pragma unroll 1
-  while (b > 0) {   // uniform
-    const int sb = b >= 3 ? 3 : b;
-    b -= sb;
-    int* sc = scratch + par * (NW * 8);
-    par ^= 1;
-    // counts at thresholds pre | t << b, t = 1 .. 7 (those with t >= 2^sb stay 0)
+  trace_mark(1);
+  nz = 0;
+  kmin = 0xFFFFFFFFu;
+  kmax = 0u;
 #pragma unroll
-    for (int t = 1; t < 8; ++t) {
-      int c = 0;
-      if (t < (1 << sb)) {
-        const uint32_t cand = pre | (static_cast<uint32_t>(t) << b);
-#pragma unroll
-        for (int g = 0; g < G; ++g) c += gm[g] >= cand ? 1 : 0;
-      }
-      c = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c)));
-      if (lane == 0) sc[warp * 8 + t] = c;
-    }
-    __syncthreads();
-    int best = 0;
-#pragma unroll
-    for (int t = 1; t < 8; ++t) {
-      const int tot = static_cast<int>(__reduce_add_sync(0xffffffffu, lane < NW ? static_cast<unsigned>(sc[lane * 8 + t]) : 0u));
-      if (t < (1 << sb) && tot >= k) best = t;
-    }
-    pre |= static_cast<uint32_t>(best) << b;
+  for (int w = 0; w < NW; ++w) {   // every thread: the same loads
+    nz += ctl.wm[w];
+    const unsigned long long wv = ctl.wv[w];
+    kmin = min(kmin, static_cast<uint32_t>(wv));
+    kmax = max(kmax, static_cast<uint32_t>(wv >> 32));
   }
-  return pre;
+  trace_mark(2);
+  if (nz < k) return 0u;   // uniform
+  constexpr int NB = 1024;                  // bins
+  constexpr int PER_LANE = NB / 32;
+  const uint32_t span = kmax - kmin;
+  const int sh = max(0, (32 - __clz(span)) - 10);   // (span >> sh) < NB
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    if (gm[g] != 0u) atomicAdd(&hist[(gm[g] - kmin) >> sh], 1);
+  }
+  trace_mark(3);
+  __syncthreads();
+  trace_mark(4);
+  // every warp: lane l sums the PER_LANE consecutive bins below NB - 1 - l * PER_LANE
+  const int top = NB - 1 - lane * PER_LANE;
+  // lane l's bins are NB-32-32l .. NB-1-32l, int4s 8(31-l) .. 8(31-l)+7
+  const int sum = chunk_sum4<PER_LANE / 4>(reinterpret_cast<const int4*>(hist), 0, 31 - lane);
+  trace_mark(5);
+  const int incl = warp_incl_scan(sum, lane);
+  const bool mine = incl - sum < k && k <= incl;   // this lane's bins hold the k-th largest
+  int bin = 0;
+  if (mine) {   // walk down the lane's bins, four at a time
+    int acc = incl - sum;
+#pragma unroll 1
+    for (int j = 0; j < PER_LANE; j += 4) {
+      const int4 q = *reinterpret_cast<const int4*>(hist + top - j - 3);
+      if (acc + q.w >= k) { bin = top - j; break; }
+      if (acc + q.w + q.z >= k) { bin = top - j - 1; break; }
+      if (acc + q.w + q.z + q.y >= k) { bin = top - j - 2; break; }
+      acc += q.w + q.z + q.y + q.x;
+      if (acc >= k) { bin = top - j - 3; break; }
+    }
+  }
+  const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+  bin = __shfl_sync(0xffffffffu, bin, src);
+  trace_mark(6);
+  return kmin + (static_cast<uint32_t>(bin) << sh);
 }
 
 // ---------------------------------------------------------------------------
@@ -652,9 +705,9 @@ __device__ __noinline__ SeedOut seed_threshold(const unsigned char* ring, WarpRo
     __syncthreads();   // histogram complete; every warp is past its reads of wm
     // the bin holding the need-th largest: per-warp slice sums, then the slice
     const int sbase = kSeedBins - (warp + 1) * SLICE;  // warp 0 sums the top slice
-    int sl = 0;
-#pragma unroll
-    for (int j = 0; j < PER_LANE; ++j) sl += hist[sbase + lane * PER_LANE + j];
+    static_assert(PER_LANE % 4 == 0 && SLICE % 4 == 0, "slices are read as int4s");
+    const int4* hist4 = reinterpret_cast<const int4*>(hist);
+    int sl = chunk_sum4<PER_LANE / 4>(hist4, sbase / 4, lane);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sl += __shfl_xor_sync(0xffffffffu, sl, o);
     if (lane == 0) ctl.wm[warp] = sl;
@@ -665,27 +718,23 @@ __device__ __noinline__ SeedOut seed_threshold(const unsigned char* ring, WarpRo
     const int slc = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
     need -= __shfl_sync(0xffffffffu, incl - c, slc);
     const int b0 = kSeedBins - (slc + 1) * SLICE;
-    int cc[PER_LANE];
-    int sm = 0;
-#pragma unroll
-    for (int j = 0; j < PER_LANE; ++j) {   // bins of that slice from its top
-      cc[j] = hist[b0 + SLICE - 1 - (lane * PER_LANE + j)];
-      sm += cc[j];
-    }
+    // lane l: the PER_LANE bins below b0 + SLICE - 1 - l * PER_LANE (chunk 31 - l)
+    const int sm = chunk_sum4<PER_LANE / 4>(hist4, b0 / 4, 31 - lane);
     const int inc2 = warp_incl_scan(sm, lane);
     const bool mine2 = (inc2 - sm) < need && need <= inc2;
     int bin = 0, above = 0;
-    if (mine2) {
+    if (mine2) {   // one lane walks its bins from the top
       int acc = inc2 - sm;
-      bool done = false;
-#pragma unroll
+#pragma unroll 1
       for (int j = 0; j < PER_LANE; ++j) {
-        if (!done && acc + cc[j] >= need) {
-          bin = b0 + SLICE - 1 - (lane * PER_LANE + j);
+        const int bj = b0 + SLICE - 1 - (lane * PER_LANE + j);
+        const int cj = hist[bj];
+        if (acc + cj >= need) {
+          bin = bj;
           above = acc;
-          done = true;
+          break;
         }
-        acc += cc[j];
+        acc += cj;
       }
     }
     const int src2 = __ffs(__ballot_sync(0xffffffffu, mine2)) - 1;
@@ -772,7 +821,7 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
   constexpr int SG = THREADS == kThreads ? 4 : 8;      // round-0 seed: group maxima per thread
   constexpr int VPG = VPT / SG;                        // vectors per group
   static_assert(VPG * SG == VPT, "seed groups");
-  static_assert(VPT * PV <= 128, "keep bits fit two 64-bit words");
+  static_assert(VPT * PV <= 128 && 64 % PV == 0, "keep bits fit two 64-bit words, vectors not straddling");
   static_assert(kSeedBins % (NW * 32) == 0, "seed histogram split");
 
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -801,7 +850,7 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
   long long st_wait = 0;
 #define DSEL_EV(i) do { if (tid == 0) st_ev[i] = clock64() - st_t0; } while (0)
   const int tr_w = (blockIdx.x == 0 && lane == 0 && warp < kTraceWarps) ? warp : -1;
-#define DSEL_TR(r, e) do { if (tr_w >= 0 && (r) < kTraceRounds - 1) \
+#define DSEL_TR(r, e) do { if (tr_w >= 0 && (r) < kTraceRounds - 2) \
     g_trace[(tr_w * kTraceRounds + (r)) * kTraceEvents + (e)] = clock64() - st_t0; } while (0)
 #else
 #define DSEL_EV(i) do { } while (0)
@@ -814,7 +863,11 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
 #pragma unroll 1
   for (int i = tid; i < 3 * kBins; i += THREADS) (&ctl.hist[0][0])[i] = 0;
 #pragma unroll 1
-  for (int i = tid; i < 2 * kSeedBins; i += THREADS) seed_hist[i] = 0;   // two histogram levels
+  {   // round-0 seed histograms: two levels of kSeedBins for large k, else 1024 bins
+    static_assert(2 * kSeedBins <= kSeedSlots, "seed histograms fit the index array");
+    const int nz = 2 * p.k > SG * THREADS ? 2 * kSeedBins : 1024;
+    for (int i = tid; i < nz; i += THREADS) seed_hist[i] = 0;
+  }
   if (tid == 0) {
     ctl.t_w = 0ull;
     ctl.nan_found = 0;
@@ -932,25 +985,27 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
       if (r == 0) {
         // ---- 2a. round 0: one pass for each vector's largest key, seed T from
         //      those maxima, and screen with them (no second read) ----
-        // group g holds vectors g*VPG .. g*VPG + VPG - 1; gm[g] = its largest key
-        // (0 = empty: partial and NaN vectors are left out and always tested exactly)
-        uint32_t gm[SG];
+        // gk[v]: largest key of vector v (0 = none: partial and NaN vectors are
+        // left out and always tested exactly); gm[g]: largest of group g's keys
+        uint32_t gk[VPT], gm[SG];
         uint32_t forced = 0u, valid = 0u;
+#pragma unroll
+        for (int v = 0; v < VPT; ++v) {
+          gk[v] = 0u;
+          const uint32_t eidx = wr.eb + static_cast<uint32_t>(v * 32 * PV);
+          if (wr.owns && eidx < uhi) {
+            valid |= 1u << v;
+            const uint4 val = *reinterpret_cast<const uint4*>(ring + wr.sb + v * 512);
+            uint32_t kx = 0u;
+            if (vec_max_key<DT>(val, kx) || eidx + PV > uhi) forced |= 1u << v;
+            else gk[v] = kx;
+          }
+        }
 #pragma unroll
         for (int g = 0; g < SG; ++g) {
           uint32_t m = 0u;
-#pragma unroll 1
-          for (int i = 0; i < VPG; ++i) {
-            const int v = g * VPG + i;
-            const uint32_t eidx = wr.eb + static_cast<uint32_t>(v * 32 * PV);
-            if (wr.owns && eidx < uhi) {
-              valid |= 1u << v;
-              const uint4 val = *reinterpret_cast<const uint4*>(ring + wr.sb + v * 512);
-              uint32_t kx = 0u;
-              if (vec_max_key<DT>(val, kx) || eidx + PV > uhi) forced |= 1u << v;
-              else m = kx > m ? kx : m;
-            }
-          }
+#pragma unroll
+          for (int i = 0; i < VPG; ++i) m = max(m, gk[g * VPG + i]);
           gm[g] = m;
         }
         DSEL_TR(r, 1);
@@ -974,11 +1029,11 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
         }
         tk = static_cast<uint32_t>(w >> 32);
         ti = ~static_cast<uint32_t>(w);
-        // a group whose largest key is below T's key holds no survivor
+        // a vector whose largest key is below T's key holds no survivor
         maybe_mask = forced;
 #pragma unroll
-        for (int g = 0; g < SG; ++g) {
-          if (gm[g] >= tk) maybe_mask |= (((1u << VPG) - 1u) << (g * VPG)) & valid;
+        for (int v = 0; v < VPT; ++v) {
+          if (gk[v] >= tk && gk[v] != 0u) maybe_mask |= 1u << v;
         }
       } else {
         // ---- 2b. later rounds: screen every vector against T ----
@@ -1008,32 +1063,33 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
 #ifdef DSEL_STATS
         if (lane == 0) atomicAdd(&ctl.st_slow_vectors, __popc(maybe_mask));
 #endif
-        uint32_t mm = maybe_mask;
+        uint32_t mm = maybe_mask;   // flagged vectors lie inside the slice
+#pragma unroll 1
         while (mm) {
           const int v = __ffs(mm) - 1;
           mm &= mm - 1u;
-          uint32_t voff, eidx;
-          wr.locate(v, voff, eidx);
-          const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
-          uint32_t cm = candidate_mask<DT>(val, tv);
-          if (eidx + PV > uhi) cm &= (1u << (uhi - eidx)) - 1u;   // past hi: not this row's
-          while (cm) {
-            const int e = __ffs(cm) - 1;
-            cm &= cm - 1u;
-            const uint32_t b = vec_elem_dyn<DT>(val, e);
-            const uint32_t idx = eidx + e;
-            if (E::is_nan(b)) {
-              if (!p.nan_flag) nan_trap();   // the pages' default policy: abort on NaN
-              nan_thread = true;
-            } else {
-              const uint32_t kk = E::key(b);
-              if (kk > tk || (kk == tk && idx < ti)) {
-                keep.set(v * PV + e);
-                const uint64_t vv = (static_cast<uint64_t>(kk) << p.idx_bits) | (idx_mask - idx);
-                vmax = vv > vmax ? vv : vmax;
-              }
-            }
+          const uint32_t eidx = wr.eb + static_cast<uint32_t>(v * 32 * PV);
+          const uint4 val = *reinterpret_cast<const uint4*>(ring + wr.sb + v * 512);
+          const uint32_t lim = uhi - eidx;   // elements of the vector inside the slice
+          uint32_t kb = 0u;
+          bool nanv = false;
+#pragma unroll
+          for (int e = 0; e < PV; ++e) {   // straight-line: no per-element loop
+            const uint32_t b = vec_elem<DT>(val, e);
+            const bool in = static_cast<uint32_t>(e) < lim;
+            const bool isn = E::is_nan(b);
+            const uint32_t kk = E::key(b);
+            const bool pass = kk > tk || (kk == tk && eidx + e < ti);
+            kb |= (in && !isn && pass) ? (1u << e) : 0u;
+            nanv |= in && isn;
           }
+          if (nanv) {
+            if (!p.nan_flag) nan_trap();   // the pages' default policy: abort on NaN
+            nan_thread = true;
+          }
+          const int bit = v * PV;          // a vector's bits never straddle the two words
+          if (bit < 64) keep.w[0] |= static_cast<uint64_t>(kb) << bit;
+          else keep.w[1] |= static_cast<uint64_t>(kb) << (bit - 64);
         }
       }
       int mine = keep.count();   // survivors of this thread not yet in the buffer
@@ -1069,8 +1125,11 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
                 uint32_t voff, eidx;
                 wr.locate(v, voff, eidx);
                 const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
-                cb[cnt + rank] = static_cast<bits_t>(vec_elem_dyn<DT>(val, e));
+                const uint32_t bv = vec_elem_dyn<DT>(val, e);
+                cb[cnt + rank] = static_cast<bits_t>(bv);
                 ci[cnt + rank] = eidx + e;
+                const uint64_t vv = (static_cast<uint64_t>(E::key(bv)) << p.idx_bits) | (idx_mask - (eidx + e));
+                vmax = vv > vmax ? vv : vmax;   // largest radix word this thread wrote
                 keep.clr(bit);
               }
               ++rank;

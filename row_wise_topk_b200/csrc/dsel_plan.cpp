@@ -48,7 +48,10 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
   p.b2 = k <= 1024 ? 1024 : std::min(k, 2048);
   // k + B2 + slack; a round's survivors beyond that wait in registers until a
   // compaction makes room, so the round may be larger than the slack
-  p.capacity = int(round_up(std::max<int64_t>(k + p.b2 + append_slack(k, p.threads), next_pow2(k)), 32));
+  // at least kSeedSlots: the round-0 seed histograms live in the index array
+  p.capacity = int(round_up(
+      std::max<int64_t>({int64_t(k) + p.b2 + append_slack(k, p.threads), int64_t(next_pow2(k)), int64_t(kSeedSlots)}),
+      32));
   p.idx_bits = ceil_log2_u64(uint64_t(row_stride));
 
   // Row split.

@@ -26,6 +26,7 @@ inline int append_slack(int k, int threads) {
   if (threads == kThreadsShort) return 1024;
   return k <= 1024 ? 4096 : 2048;
 }
+constexpr int kSeedSlots = 4096;              // candidate slots that hold the round-0 seed histograms
 constexpr int kStrideReq = 16;                // row_stride multiple (elements)
 constexpr int kMaxStages = 128;               // ring depth cap (one mbarrier per stage)
 constexpr int kMinSliceElems = 8192;          // smallest row share worth its own CTA

@@ -103,6 +103,7 @@ def test_plan_invariants(dtype, rows, stride, k):
     slack = 1024 if p["threads"] == 128 else (4096 if k <= 1024 else 2048)
     assert p["capacity"] >= k + p["b2"] + slack
     assert p["capacity"] >= 1 << (k - 1).bit_length()          # room for the bitonic padding
+    assert p["capacity"] >= 4096                                 # the round-0 seed histograms
     q = p["round"] // p["block"]
     slice_ = -(-(-(-stride // (p["cluster"] * p["groups"]))) // 16) * 16
     nb_max = -(-slice_ // p["block"])
