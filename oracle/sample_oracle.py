@@ -15,8 +15,10 @@ for the draw itself, so this oracle takes the plainest reading:
 
 1. candidates: the row's top-k (``oracle_topk``), in value-descending order with
    ties by ascending index -- the TopK total order;
-2. temperature t > 0: weights e_i = exp((z_i - z_1) / t), z_1 the largest logit
-   (so e_1 = 1); t <= 0 means greedy, the first candidate;
+2. temperature t > 0: weights e_i = exp((z_i - z_1) / t), z_1 the largest logit,
+   and e_i = 1 wherever z_i equals z_1 (the limit; it keeps +-inf logits
+   meaningful: a row whose candidates are all -inf draws uniformly among them);
+   t <= 0 means greedy, the first candidate;
 3. top-p: keep the shortest prefix of c candidates whose weight sum E_c reaches
    top_p * E_m (m = number of candidates); top_p >= 1 keeps all m;
 4. draw: with the caller's uniform u in [0, 1), the token is the first kept
@@ -66,7 +68,8 @@ def sample_row(z: np.ndarray, temperature: float, top_p: float, u: float):
         e = np.zeros(m)
         e[0] = 1.0
     else:
-        e = np.exp((z - z[0]) / temperature)
+        with np.errstate(invalid="ignore", over="ignore"):
+            e = np.where(z == z[0], 1.0, np.exp((z - z[0]) / temperature))
     prefix = np.cumsum(e)
     total = prefix[-1]
     if top_p >= 1.0:

@@ -120,3 +120,13 @@ def test_token_is_always_in_the_top_k():
         top = set(np.argsort(-x[r], kind="stable")[:k].tolist())
         assert int(res.token[r]) in top
         assert 0 < res.prob[r] <= 1
+
+
+def test_infinite_logits():
+    # +inf leaders share all the mass; a row of -inf draws uniformly among them
+    x = np.full((2, 16), -np.inf, dtype=np.float32)
+    x[0, [4, 11]] = np.inf
+    x[0, 2] = 7.0
+    res = S.oracle_sample(f32_bits(x), 3, 1.0, 1.0, np.array([0.75, 0.7]))
+    assert res.token[0] == 11 and res.prob[0] == pytest.approx(0.5)
+    assert res.token[1] == 2 and res.prob[1] == pytest.approx(1 / 3)   # candidates 0, 1, 2
