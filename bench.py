@@ -34,8 +34,10 @@ import workloads as W  # noqa: E402
 METRIC = "effective HBM GB/s and rows/s for TopK (bf16 k=512; fp32 V=129,280) on 1 B200"
 KERNEL_SOURCES = ["row_wise_topk_b200/csrc/dsel_device.cuh", "row_wise_topk_b200/csrc/dsel_kernels.cuh",
                   "row_wise_topk_b200/csrc/dsel_api.cu", "row_wise_topk_b200/csrc/dsel_plan.cpp",
+                  "row_wise_topk_b200/csrc/dsel_shard.cu",
                   "row_wise_topk_b200/csrc/dsel_plan.h"]
 FALLBACK_HBM_GBS = 6650.0
+SAMPLE_T, SAMPLE_P = 1.0, 0.9      # temperature and top-p of the sample_B_k workloads
 
 
 def make_workload(name: str) -> W.Workload:
@@ -46,6 +48,11 @@ def make_workload(name: str) -> W.Workload:
     if name.startswith("sampler"):        # sampler_B_k, e.g. sampler_256_4096
         _, b, k = name.split("_")
         return W.sampler_logits(int(b), int(k))
+    if name.startswith("sample_"):        # sample_B_k: TopK + the sampling draw, tokens only
+        _, b, k = name.split("_")
+        w = W.sampler_logits(int(b), int(k))
+        w.name = "topk_sample_" + w.name + f"_t{SAMPLE_T}_p{SAMPLE_P}"
+        return w
     if name.startswith("long"):           # long_1_1000 (1 x 2^28) or long_16_4096 (16 x 2^24)
         _, r, k = name.split("_")
         r = int(r)
@@ -190,21 +197,28 @@ def whole_job_gbs(bytes_per_step: int, steps: int, elapsed_ms: float, world: int
 def cpu_oracle_throughput(w: W.Workload, budget_s: float):
     """Times the CPU oracle (as it stands) on whole rows of the workload until the
     budget is spent; returns (GB/s effective, rows/s, rows timed)."""
+    import oracle.sample_oracle as S
     import oracle.topk_oracle as O
+    sampling = w.name.startswith("topk_sample_")
+    u = W.uniforms(w.rows)
     lens = w.valid_lengths()
     idx_b = 4 if w.index_dtype == "i32" else 8
     val_b = w.elem_bytes if w.return_value else 0
+    out_b = (4 + 8 + 4) if sampling else w.k * (idx_b + val_b)
     done_rows, done_bytes, t_used = 0, 0, 0.0
     r = 0
     while t_used < budget_s and done_rows < 100000:
         sub = slice(r % w.rows, r % w.rows + 1)
         end = None if w.end is None else w.end[sub]
         t0 = time.perf_counter()
-        O.oracle_topk(w.x[sub], w.dtype, w.k, end=end, sorted_index=w.sorted_index,
-                      return_value=w.return_value, index_dtype=w.index_dtype, nan_mode=w.nan_mode)
+        if sampling:
+            S.oracle_sample(w.x[sub], w.k, SAMPLE_T, SAMPLE_P, u[sub], end=end, nan_mode=w.nan_mode)
+        else:
+            O.oracle_topk(w.x[sub], w.dtype, w.k, end=end, sorted_index=w.sorted_index,
+                          return_value=w.return_value, index_dtype=w.index_dtype, nan_mode=w.nan_mode)
         t_used += time.perf_counter() - t0
         done_rows += 1
-        done_bytes += int(lens[r % w.rows]) * w.elem_bytes + w.k * (idx_b + val_b) + (4 if w.end is not None else 0)
+        done_bytes += int(lens[r % w.rows]) * w.elem_bytes + out_b + (4 if w.end is not None else 0)
         r += 1
     return done_bytes / t_used / 1e9, done_rows / t_used, done_rows, t_used
 
@@ -272,11 +286,22 @@ def run_ours(args, w, world, rank, local, pg):
     nm = T.DSEL_NAN_FLAG if w.nan_mode == "flag" else T.DSEL_NAN_TRAP
     sptr = stream.cuda_stream
 
+    sampling = args.workload.startswith("sample_")
+    u_dev = torch.from_numpy(W.uniforms(w.rows)).to(dev)
+    tok_out = torch.empty(w.rows, dtype=torch.int64, device=dev)
+    prob_out = torch.empty(w.rows, dtype=torch.float32, device=dev)
+
     def step(i):
-        st = T.dsel_topk(copies[i % n_copies].data_ptr(), dt, w.rows, w.row_stride,
-                         None if end_dev is None else end_dev.data_ptr(), w.k, w.sorted_index,
-                         w.return_value, idt, nm, None if val_out is None else val_out.data_ptr(),
-                         idx_out.data_ptr(), sptr)
+        if sampling:
+            st = T.dsel_topk_sample(copies[i % n_copies].data_ptr(), w.rows, w.row_stride,
+                                    None if end_dev is None else end_dev.data_ptr(), w.k, SAMPLE_T, SAMPLE_P,
+                                    u_dev.data_ptr(), nm, None, None, tok_out.data_ptr(), prob_out.data_ptr(),
+                                    sptr)
+        else:
+            st = T.dsel_topk(copies[i % n_copies].data_ptr(), dt, w.rows, w.row_stride,
+                             None if end_dev is None else end_dev.data_ptr(), w.k, w.sorted_index,
+                             w.return_value, idt, nm, None if val_out is None else val_out.data_ptr(),
+                             idx_out.data_ptr(), sptr)
         if st != 0:
             raise T.DselError(st)
 
@@ -346,7 +371,10 @@ def run_ours(args, w, world, rank, local, pg):
 
     elapsed_ms = max_over_ranks(elapsed_ms, pg, dev)
     ms_per_step = elapsed_ms / args.steps
-    eff = w.effective_bytes()
+    if sampling:   # valid logits read once, u read, token + probability written (+ end)
+        eff = int(w.valid_lengths().sum()) * eb + w.rows * (4 + 8 + 4) + (0 if w.end is None else 4 * w.rows)
+    else:
+        eff = w.effective_bytes()
     value = whole_job_gbs(eff, args.steps, elapsed_ms, world)
     rows_per_s = world * w.rows * args.steps / (elapsed_ms / 1e3)
 
@@ -370,17 +398,25 @@ def run_ours(args, w, world, rank, local, pg):
         e0.record()
         for i in range(e2e_steps):
             x_e2e.copy_(host, non_blocking=True)
-            T.topk(xv, w.k, end=end_dev, sorted_index=w.sorted_index,
-                   return_value=bool(w.return_value), index_dtype=itorch, nan_mode=w.nan_mode,
-                   out=(val_out, idx_out), stream=sptr)
-            host_idx.copy_(idx_out, non_blocking=True)
-            if host_val is not None:
-                host_val.copy_(val_out, non_blocking=True)
+            if sampling:
+                tok, _ = T.topk_sample(xv, w.k, u_dev, temperature=SAMPLE_T, top_p=SAMPLE_P, end=end_dev,
+                                       nan_mode=w.nan_mode, stream=sptr)
+                host_idx.view(-1)[: w.rows].copy_(tok, non_blocking=True)
+            else:
+                T.topk(xv, w.k, end=end_dev, sorted_index=w.sorted_index,
+                       return_value=bool(w.return_value), index_dtype=itorch, nan_mode=w.nan_mode,
+                       out=(val_out, idx_out), stream=sptr)
+                host_idx.copy_(idx_out, non_blocking=True)
+                if host_val is not None:
+                    host_val.copy_(val_out, non_blocking=True)
         e1.record()
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg, dev) / e2e_steps
     h2d = in_bytes
-    d2h = idx_out.numel() * idx_out.element_size() + (0 if val_out is None else val_out.numel() * val_out.element_size())
+    if sampling:
+        d2h = w.rows * 8
+    else:
+        d2h = idx_out.numel() * idx_out.element_size() + (0 if val_out is None else val_out.numel() * val_out.element_size())
     e2e_value = world * eff / (e2e_ms / 1e3) / 1e9
 
     if rank != 0:

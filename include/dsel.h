@@ -177,6 +177,96 @@ DSEL_API int dsel_topk_noalloc(const void* x, int dtype, int64_t rows, int64_t r
                                int index_dtype, int nan_mode, void* values_out, void* indices_out,
                                void* stream);
 
+/*
+ * dsel_topk_sample -- TopK of float32 sampler logits followed, in the same
+ * launch, by a sampling draw among each row's k candidates.
+ *
+ * The pages name this use ("DeepSeek releases DeepSelect, a TopK kernel for
+ * sparse attention and sampling", paragraph "Why rewrite TopK at all?": during
+ * sampling TopK picks the candidate tokens out of a large vocabulary) and list
+ * temperature and top-p among the generation settings (deepseek-recipe page,
+ * section "deepseek-recipe: the protocol layer is real engineering"), but print
+ * no formula for the draw.  This library's reading, per row, on the candidates
+ * z_1 >= z_2 >= ... (value order, ties by ascending index):
+ *   - weights e_i = exp((z_i - z_1) / temperature), and e_i = 1 wherever
+ *     z_i == z_1 (so +-inf logits stay meaningful); temperature <= 0 (or NaN)
+ *     draws greedily: the first candidate;
+ *   - top-p: keep the shortest prefix whose weight sum E_c reaches top_p times
+ *     the total; top_p >= 1 (or NaN) keeps every candidate;
+ *   - the token is the first kept candidate whose prefix sum exceeds u[r] * E_c;
+ *     its probability is e / E_c.
+ * Arithmetic is float32 (expf, float32 sums); a different summation order can
+ * change the token only where u[r] * E_c or top_p times the total falls within
+ * rounding distance of a prefix sum.
+ *
+ *   x, rows, row_stride, end, k, nan_mode
+ *                as for dsel_topk, with dtype DSEL_F32 (x holds float32 logits)
+ *   temperature, top_p   as above
+ *   u            device float32 [rows]: the caller's uniform draws in [0, 1), one
+ *                per row (values outside [0, 1) clamp to the first / last kept
+ *                candidate)
+ *   values_out, indices_out
+ *                both NULL (only the draw is wanted) or both set: the TopK result
+ *                as dsel_topk gives it with sorted_index = DSEL_ORDER_VALUE,
+ *                return_value = 1 and int64 indices
+ *   token_out    device int64 [rows]: the drawn index within the row, or a
+ *                negative row code: DSEL_IDX_PAD for an empty row (end = 0),
+ *                DSEL_IDX_NAN for a NaN row in DSEL_NAN_FLAG mode, DSEL_IDX_BAD_END
+ *                for an invalid end in DSEL_NAN_FLAG mode
+ *   prob_out     device float32 [rows] or NULL: the drawn token's probability
+ *                (NaN on rows with a negative code)
+ * NaN policy: as dsel_topk, except that rows of length <= k are checked for NaN
+ * too (TopK skips the check there, but a softmax over a NaN has no meaning).
+ * Returns DSEL_OK or a DSEL_ERR_* code (DSEL_ERR_NULL when x, u or token_out is
+ * NULL, DSEL_ERR_VALUES when exactly one of values_out / indices_out is NULL);
+ * asynchronous on `stream`, allocation behaviour as dsel_topk.
+ */
+DSEL_API int dsel_topk_sample(const void* x, int64_t rows, int64_t row_stride, const int32_t* end, int32_t k,
+                              float temperature, float top_p, const float* u, int nan_mode, void* values_out,
+                              void* indices_out, int64_t* token_out, float* prob_out, void* stream);
+
+/*
+ * Row split over several shards (one per GPU).  A row too long for one GPU is
+ * cut into `shards` contiguous pieces of shard_len elements; each piece's TopK
+ * (dsel_topk with sorted_index = DSEL_ORDER_INDEX, return_value = 1, int64
+ * indices relative to the piece) is exchanged (one all-gather: shard-major
+ * [shards][rows][k]), and the row's TopK is the TopK of the shards' candidates:
+ * none of the row's k largest can be missing from its own shard's k largest.
+ * The pages keep a whole row on one device; this is the library's extension of
+ * their multi-CTA split to several GPUs.  Requires shard_len >= k, so every
+ * shard contributes k real candidates and no padding competes with them.
+ *
+ * dsel_shard_stack lays the gathered candidates out as one row per input row:
+ *   vals_in     device [shards][rows][k] values (dtype), as gathered
+ *   idx_in      device int64 [shards][rows][k] indices relative to each shard
+ *   out_stride  elements per output row: >= shards * k, a multiple of
+ *               dsel_stride_requirement(dtype)
+ *   vals_out    device [rows][out_stride]: candidate j of shard s at column
+ *               s * k + j; columns from shards * k on hold -inf
+ *   idx_out     device int64 [rows][out_stride]: the candidate's index in the
+ *               whole row (idx_in + s * shard_len; negative codes pass through)
+ * Concatenating in shard order keeps the positions in index order, so
+ * dsel_topk on vals_out breaks ties exactly as on the whole row; -inf padding
+ * sits after every real candidate and is never preferred to one.
+ * Returns DSEL_OK, DSEL_ERR_DTYPE / _K / _ROWS / _STRIDE / _NULL, or
+ * DSEL_ERR_CUDA.  Asynchronous on `stream`.
+ */
+DSEL_API int dsel_shard_stack(const void* vals_in, const int64_t* idx_in, int dtype, int64_t rows, int32_t k,
+                              int32_t shards, int64_t shard_len, int64_t out_stride, void* vals_out,
+                              int64_t* idx_out, void* stream);
+
+/*
+ * dsel_take_index -- out[r][j] = table[r][pos[r][j]] for pos >= 0, pos itself
+ * (a sentinel code) otherwise: maps the positions returned by dsel_topk on a
+ * dsel_shard_stack row back to indices in the whole row.
+ *   table        device int64 [rows][table_stride]
+ *   pos          device [rows][k], int32 or int64 (pos_dtype: DSEL_I32 / DSEL_I64)
+ *   indices_out  device [rows][k], int32 or int64 (index_dtype)
+ * Returns DSEL_OK, DSEL_ERR_K / _ROWS / _INDEX_DTYPE / _NULL, or DSEL_ERR_CUDA.
+ */
+DSEL_API int dsel_take_index(const int64_t* table, int64_t table_stride, const void* pos, int pos_dtype, int64_t rows,
+                             int32_t k, int index_dtype, void* indices_out, void* stream);
+
 /* Row-stride requirement in elements for `dtype` (the pages' get_stride_requirement,
  * narracomm paragraph on install and switches): 16 for both dtypes, so every row
  * start is 32-byte (bf16) or 64-byte (f32) aligned.  Returns -1 for a bad dtype. */
@@ -209,7 +299,9 @@ DSEL_API int dsel_device_status(int* status_out, void* stream);
  * With n_ctas == -1, host_out instead receives the per-round timeline of CTA 0:
  * 16 warps x 12 rounds x 10 int64 cycle times from kernel start (round start,
  * screened, counted, append barrier, written, after compaction, prefixed,
- * seeded, blocks arrived, seed returned; 0 = not reached).
+ * seeded, blocks arrived, seed returned; 0 = not reached).  With n_ctas <= -2,
+ * later launches record the timeline of CTA -n_ctas - 2 instead of CTA 0
+ * (host_out is not used).
  * Synchronises `stream`. */
 DSEL_API int dsel_debug_stats(uint64_t* host_out, int64_t n_ctas, void* stream);
 

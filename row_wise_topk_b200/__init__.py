@@ -67,6 +67,13 @@ def _load() -> ctypes.CDLL:
                               vp, vp, vp]
     lib.dsel_topk_noalloc.restype = c_int
     lib.dsel_topk_noalloc.argtypes = list(lib.dsel_topk.argtypes)
+    lib.dsel_topk_sample.restype = c_int
+    lib.dsel_topk_sample.argtypes = [vp, c_i64, c_i64, vp, ctypes.c_int32, ctypes.c_float, ctypes.c_float, vp, c_int,
+                                     vp, vp, vp, vp, vp]
+    lib.dsel_shard_stack.restype = c_int
+    lib.dsel_shard_stack.argtypes = [vp, vp, c_int, c_i64, ctypes.c_int32, ctypes.c_int32, c_i64, c_i64, vp, vp, vp]
+    lib.dsel_take_index.restype = c_int
+    lib.dsel_take_index.argtypes = [vp, c_i64, vp, c_int, c_i64, ctypes.c_int32, c_int, vp, vp]
     lib.dsel_stride_requirement.restype = c_i64
     lib.dsel_stride_requirement.argtypes = [c_int]
     lib.dsel_status_string.restype = ctypes.c_char_p
@@ -106,6 +113,15 @@ def dsel_topk_noalloc(x: int, dtype: int, rows: int, row_stride: int, end: Optio
     call needs more, and calls that overlap on the GPU must be ordered."""
     return lib.dsel_topk_noalloc(x, dtype, rows, row_stride, end, k, sorted_index, return_value,
                                  index_dtype, nan_mode, values_out, indices_out, stream)
+
+
+def dsel_topk_sample(x: int, rows: int, row_stride: int, end: Optional[int], k: int, temperature: float,
+                     top_p: float, u: int, nan_mode: int, values_out: Optional[int], indices_out: Optional[int],
+                     token_out: int, prob_out: Optional[int], stream: Optional[int]) -> int:
+    """Raw entry point of TopK + sampling draw on float32 logits (see include/dsel.h):
+    pointers are integers (device addresses), returns the status."""
+    return lib.dsel_topk_sample(x, rows, row_stride, end, k, temperature, top_p, u, nan_mode, values_out,
+                                indices_out, token_out, prob_out, stream)
 
 
 def dsel_stride_requirement(dtype: int) -> int:
@@ -200,3 +216,48 @@ def topk(x, k: int, *, end=None, sorted_index: int = DSEL_ORDER_INDEX, return_va
     if st != DSEL_OK:
         raise DselError(st)
     return values, indices
+
+
+def topk_sample(logits, k: int, u, *, temperature: float = 1.0, top_p: float = 1.0, end=None,
+                return_topk: bool = False, nan_mode: str = "trap", stream=None):
+    """Sampling draw among the k largest float32 logits of each row.
+
+    ``u`` is a float32 CUDA tensor with one uniform in [0, 1) per row (the caller's
+    random numbers).  Returns ``(token, prob)``, int64 and float32 tensors of one
+    entry per row, plus ``(values, indices)`` of the TopK in value order when
+    ``return_topk`` is set.
+    """
+    import torch
+
+    if logits.dim() != 2 or logits.dtype != torch.float32 or not logits.is_cuda or logits.stride(1) != 1:
+        raise ValueError("logits must be a 2-D float32 CUDA tensor, contiguous in the last dimension")
+    rows = logits.shape[0]
+    row_stride = logits.stride(0) if rows > 1 else logits.shape[1]
+    if end is None and logits.shape[1] != row_stride:
+        raise ValueError("rows narrower than their stride need end= (valid length per row)")
+    if u.dtype != torch.float32 or not u.is_cuda or u.numel() != rows:
+        raise ValueError("u must be a float32 CUDA tensor with one entry per row")
+    u = u.contiguous()
+    token = torch.empty(rows, dtype=torch.int64, device=logits.device)
+    prob = torch.empty(rows, dtype=torch.float32, device=logits.device)
+    values = indices = None
+    if return_topk:
+        values = torch.empty((rows, k), dtype=torch.float32, device=logits.device)
+        indices = torch.empty((rows, k), dtype=torch.int64, device=logits.device)
+    if end is not None:
+        if end.dtype != torch.int32 or not end.is_cuda or end.numel() != rows:
+            raise ValueError("end must be an int32 CUDA tensor with one entry per row")
+        end = end.contiguous()
+    if stream is None:
+        stream = torch.cuda.current_stream(logits.device).cuda_stream
+    st = dsel_topk_sample(logits.data_ptr(), rows, row_stride, None if end is None else end.data_ptr(), k,
+                          float(temperature), float(top_p), u.data_ptr(),
+                          DSEL_NAN_FLAG if nan_mode == "flag" else DSEL_NAN_TRAP,
+                          None if values is None else values.data_ptr(),
+                          None if indices is None else indices.data_ptr(), token.data_ptr(), prob.data_ptr(),
+                          stream)
+    if st != DSEL_OK:
+        raise DselError(st)
+    if return_topk:
+        return token, prob, (values, indices)
+    return token, prob

@@ -11,7 +11,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdsel.so")
 STATS_LIB = os.path.join(HERE, "libdsel_stats.so")   # same library, with per-CTA counters
-SOURCES = ["dsel_api.cu", "dsel_plan.cpp"]
+SOURCES = ["dsel_api.cu", "dsel_plan.cpp", "dsel_shard.cu"]
 HEADERS = ["dsel_device.cuh", "dsel_kernels.cuh", "dsel_plan.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -83,13 +83,18 @@ cudaError_t launch_cluster(Kern kern, unsigned grid, int threads, int cluster, u
   cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the kernels set up shared memory, then wait
+  // for the previous grid (griddepcontrol.wait) before touching global memory,
+  // so their prologue overlaps the tail of the launch before them
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, kp);
 }
 
@@ -179,9 +184,16 @@ DSEL_API const char* dsel_status_string(int status) {
 
 DSEL_API int dsel_debug_stats(uint64_t* host_out, int64_t n_ctas, void* stream) {
 #ifdef DSEL_STATS
-  if (host_out == nullptr || n_ctas < -1) return DSEL_ERR_NULL;
-  const int64_t n = n_ctas < kStatsCtas ? n_ctas : kStatsCtas;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (n_ctas <= -2) {   // select the CTA whose timeline later launches record
+    const int cta = static_cast<int>(-n_ctas - 2);
+    return cudaMemcpyToSymbolAsync(g_trace_cta, &cta, sizeof(int), 0, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+                   cudaStreamSynchronize(cs) == cudaSuccess
+               ? DSEL_OK
+               : DSEL_ERR_CUDA;
+  }
+  if (host_out == nullptr) return DSEL_ERR_NULL;
+  const int64_t n = n_ctas < kStatsCtas ? n_ctas : kStatsCtas;
   if (n_ctas == -1) {   // the per-round timeline instead (4 x 64 x 6 values)
     if (cudaMemcpyFromSymbolAsync(host_out, g_trace, sizeof(long long) * kTraceSize, 0,
                                   cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
@@ -261,6 +273,59 @@ DSEL_API int dsel_topk(const void* x, int dtype, int64_t rows, int64_t row_strid
   }
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   return dtype == DSEL_BF16 ? run<DSEL_BF16>(kp, pl, rows, cs, di) : run<DSEL_F32>(kp, pl, rows, cs, di);
+}
+
+DSEL_API int dsel_topk_sample(const void* x, int64_t rows, int64_t row_stride, const int32_t* end, int32_t k,
+                              float temperature, float top_p, const float* u, int nan_mode, void* values_out,
+                              void* indices_out, int64_t* token_out, float* prob_out, void* stream) {
+  int st = check_shape(DSEL_F32, rows, row_stride, k);
+  if (st != DSEL_OK) return st;
+  if (nan_mode != DSEL_NAN_TRAP && nan_mode != DSEL_NAN_FLAG) return DSEL_ERR_NAN_MODE;
+  if (rows == 0) return DSEL_OK;
+  if (x == nullptr || u == nullptr || token_out == nullptr) return DSEL_ERR_NULL;
+  if ((values_out == nullptr) != (indices_out == nullptr)) return DSEL_ERR_VALUES;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) != 0) return DSEL_ERR_ALIGN;
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSEL_ERR_CUDA;
+  DevInfo* di = nullptr;
+  st = device_info(dev, &di);
+  if (st != DSEL_OK) return st;
+  dsel_plan_t pl;
+  st = make_plan(DSEL_F32, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster, &pl);
+  if (st != DSEL_OK) return st;
+
+  KParams kp = {};
+  kp.x = x;
+  kp.end = end;
+  kp.values_out = values_out;
+  kp.indices_out = indices_out;
+  kp.rows = rows;
+  kp.row_stride = row_stride;
+  kp.k = k;
+  kp.groups = pl.groups;
+  kp.b2 = pl.b2;
+  kp.stages = pl.stages;
+  kp.idx_bits = pl.idx_bits;
+  kp.order = DSEL_ORDER_VALUE;
+  kp.return_value = values_out != nullptr;
+  kp.index_i64 = 1;
+  kp.nan_flag = nan_mode == DSEL_NAN_FLAG;
+  kp.capacity = pl.capacity;
+  kp.u = u;
+  kp.token_out = token_out;
+  kp.prob_out = prob_out;
+  kp.temperature = temperature;
+  kp.top_p = top_p;
+  if (pl.groups > 1) {
+    void* ws = nullptr;
+    st = workspace(dev, stream, size_t(pl.workspace_bytes), &ws);
+    if (st != DSEL_OK) return st;
+    kp.ws_pairs = static_cast<uint2*>(ws);
+    kp.ws_meta = reinterpret_cast<int2*>(static_cast<char*>(ws) + rows * pl.groups * int64_t(k) * 8);
+  }
+  return run<DSEL_F32>(kp, pl, rows, static_cast<cudaStream_t>(stream), di);
 }
 
 // ---------------------------------------------------------------------------

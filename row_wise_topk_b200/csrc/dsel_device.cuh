@@ -238,6 +238,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 
 __device__ __forceinline__ void nan_trap() { asm volatile("trap;"); }
 
+// Programmatic dependent launch.  wait: block until the grids this launch
+// depends on have completed and their writes are visible (a no-op for a launch
+// without the programmatic-serialization attribute); everything before it must
+// not touch global memory.  launch_dependents: let the next launch in the stream
+// start its own prologue (it still waits for this grid before touching memory).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // --------------------------------------------------------------------------- //
 // Shared control block (one per CTA, after the candidate arrays).
 // --------------------------------------------------------------------------- //
@@ -252,12 +260,16 @@ struct __align__(16) Ctl {
   int hb;                       // index of a histogram that is all zero
   int x_cnt, x_nan, x_kept;     // exchanged with peers in the final phase
   int sel_flag;
+  int add[3];                   // survivors appended per round (round r uses add[r % 3])
   int tie_n;                    // radix select: members of a small bucket gathered so far
   unsigned long long tie_v;     // radix select: the selected radix word of that bucket
   int wc[2][kWarpsMax];         // per-warp counts, by round parity
   int wm[kWarpsMax];            // per-warp counts (compaction movers)
   int hist[3][kBins];
   int hsum[kBins];
+  float smp_w[kWarpsMax];       // sampling: per-warp weight sums
+  int smp_c, smp_pos;           // sampling: last kept candidate, drawn candidate
+  float smp_ec;                 // sampling: weight sum of the kept candidates
 #ifdef DSEL_STATS
   unsigned long long st_compact_cycles;
   int st_compactions;

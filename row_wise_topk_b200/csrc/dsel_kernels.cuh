@@ -29,6 +29,12 @@ struct KParams {
   int32_t gather;           // final phase gathers the cluster's partial results on rank 0
   int32_t capacity;         // candidate-buffer slots
   uint32_t off_bars, off_blk, off_cb, off_ci, off_holes, off_ctl;
+  // sampling step after TopK (fp32 only; token_out == nullptr: no draw)
+  const float* u;           // [rows] the caller's uniforms in [0, 1)
+  int64_t* token_out;       // [rows] drawn index, or a negative row code
+  float* prob_out;          // [rows] its probability after the top-p cut (may be nullptr)
+  float temperature;        // <= 0: greedy
+  float top_p;              // >= 1: no cut
 };
 
 #ifdef DSEL_STATS
@@ -41,13 +47,14 @@ constexpr int kTraceRounds = 12;
 constexpr int kTraceEvents = 10;
 constexpr int kTraceSize = kTraceWarps * kTraceRounds * kTraceEvents;
 __device__ long long g_trace[kTraceSize];
+__device__ int g_trace_cta = 0;   // the CTA whose timeline is recorded
 #endif
 
 // Per-warp marks inside a phase (CTA 0, lane 0 of each warp), stats builds
 // only: absolute clocks in trace row kTraceRounds - 2.
 __device__ __forceinline__ void trace_mark(int e) {
 #ifdef DSEL_STATS
-  if (blockIdx.x == 0 && (threadIdx.x & 31) == 0 && (threadIdx.x >> 5) < kTraceWarps)
+  if (blockIdx.x == g_trace_cta && (threadIdx.x & 31) == 0 && (threadIdx.x >> 5) < kTraceWarps)
     g_trace[((threadIdx.x >> 5) * kTraceRounds + kTraceRounds - 2) * kTraceEvents + e] = clock64();
 #else
   (void)e;
@@ -59,7 +66,7 @@ __device__ __forceinline__ void trace_mark(int e) {
 // kernel-start clock.
 __device__ __forceinline__ void trace_final(int e) {
 #ifdef DSEL_STATS
-  if (blockIdx.x == 0 && threadIdx.x == 0) g_trace[(kTraceRounds - 1) * kTraceEvents + e] = clock64();
+  if (blockIdx.x == g_trace_cta && threadIdx.x == 0) g_trace[(kTraceRounds - 1) * kTraceEvents + e] = clock64();
 #else
   (void)e;
 #endif
@@ -75,6 +82,7 @@ template <int DT, int THREADS>
 __device__ void write_rows_out(const KParams& p, int64_t row, int off, int m,
                                const typename Elem<DT>::bits_t* cb, const uint32_t* ci) {
   using bits_t = typename Elem<DT>::bits_t;
+  if (p.indices_out == nullptr) return;   // a sampling call that wants only the token
   const int64_t base = row * p.k + off;
 #pragma unroll 1
   for (int i = threadIdx.x; i < m; i += THREADS) {
@@ -96,6 +104,11 @@ __device__ void write_ws(const KParams& p, int64_t row, int g, int off, int m,
 template <int DT, int THREADS>
 __device__ __noinline__ void write_sentinel_row(const KParams& p, int64_t row, int32_t code) {
   using bits_t = typename Elem<DT>::bits_t;
+  if (p.token_out != nullptr && threadIdx.x == 0) {   // the row's draw carries the same code
+    p.token_out[row] = code;
+    if (p.prob_out != nullptr) p.prob_out[row] = __int_as_float(0x7FC00000);
+  }
+  if (p.indices_out == nullptr) return;
   const int64_t base = row * p.k;
 #pragma unroll 1
   for (int i = threadIdx.x; i < p.k; i += THREADS) {
@@ -109,6 +122,7 @@ __device__ __noinline__ void write_sentinel_row(const KParams& p, int64_t row, i
 template <int DT, int THREADS>
 __device__ __noinline__ void write_short_row(const KParams& p, int64_t row, int64_t n) {
   using bits_t = typename Elem<DT>::bits_t;
+  if (p.indices_out == nullptr) return;
   const bits_t* xr = static_cast<const bits_t*>(p.x) + row * p.row_stride;
   const int64_t base = row * p.k;
 #pragma unroll 1
@@ -120,6 +134,139 @@ __device__ __noinline__ void write_short_row(const KParams& p, int64_t row, int6
     if (p.return_value)
       static_cast<bits_t*>(p.values_out)[base + i] = in ? xr[i] : static_cast<bits_t>(Elem<DT>::kNegInf);
   }
+}
+
+// ---------------------------------------------------------------------------
+// Sampling step on a row's m candidates, fp32 logits zb[0, m) in value order
+// (descending, ties by ascending index) with their indices ci (all threads of
+// one CTA).  Reading of the pages (which name temperature and top-p among the
+// sampler settings but print no formula): weights e_i = exp((z_i - z_1) / t),
+// e_i = 1 where z_i equals the largest logit z_1; the shortest prefix whose
+// weight sum E_c reaches top_p of the total is kept; with the caller's uniform
+// u the token is the first kept candidate whose prefix sum exceeds u * E_c, and
+// its probability is e / E_c.  t <= 0 draws greedily (the first candidate).
+// Float32 throughout; each thread sums a contiguous chunk, so prefix sums are
+// the chunk's running sum on top of a block scan of the chunk sums.
+// ---------------------------------------------------------------------------
+template <int THREADS>
+__device__ __noinline__ void sample_draw(const KParams& p, int64_t row, const uint32_t* zb, const uint32_t* ci,
+                                         int m, Ctl& ctl) {
+  constexpr int NW = THREADS / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (m <= 0) {   // uniform: nothing to draw from
+    if (tid == 0) {
+      p.token_out[row] = DSEL_IDX_PAD;
+      if (p.prob_out != nullptr) p.prob_out[row] = __int_as_float(0x7FC00000);
+    }
+    return;
+  }
+  const float t = p.temperature;
+  if (!(t > 0.0f)) {   // greedy
+    if (tid == 0) {
+      p.token_out[row] = static_cast<int64_t>(ci[0]);
+      if (p.prob_out != nullptr) p.prob_out[row] = 1.0f;
+    }
+    return;
+  }
+  const float z1 = __uint_as_float(zb[0]);
+  auto weight = [&](int i) -> float {
+    const float z = __uint_as_float(zb[i]);
+    return z == z1 ? 1.0f : expf((z - z1) / t);
+  };
+  const int per = (m + THREADS - 1) / THREADS;
+  const int a = min(m, tid * per), b = min(m, a + per);
+  float s = 0.0f;
+#pragma unroll 1
+  for (int i = a; i < b; ++i) s += weight(i);
+  float incl = s;   // warp inclusive scan of the chunk sums
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) ctl.smp_w[warp] = incl;
+  if (tid == 0) {
+    ctl.smp_c = m - 1;        // last kept candidate: all, unless the top-p cut says fewer
+    ctl.smp_pos = m;          // none drawn yet
+  }
+  __syncthreads();
+  float before = 0.0f, total = 0.0f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const float ws = ctl.smp_w[w];
+    before += w < warp ? ws : 0.0f;
+    total += ws;
+  }
+  const float off = before + incl - s;   // weight sum of the candidates before this chunk
+  if (p.top_p < 1.0f) {
+    const float tp = p.top_p * total;
+    float run = off;
+#pragma unroll 1
+    for (int i = a; i < b; ++i) {
+      run += weight(i);
+      if (run >= tp) {   // first prefix sum reaching the cut
+        atomicMin(&ctl.smp_c, i);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+  const int cl = ctl.smp_c;
+  if (a <= cl && cl < b) {   // the chunk holding the last kept candidate: E_c
+    float run = off;
+#pragma unroll 1
+    for (int i = a; i <= cl; ++i) run += weight(i);
+    ctl.smp_ec = run;
+  }
+  __syncthreads();
+  const float ec = ctl.smp_ec;
+  const float target = p.u[row] * ec;
+  {
+    float run = off;
+#pragma unroll 1
+    for (int i = a; i < b && i <= cl; ++i) {
+      run += weight(i);
+      if (run > target) {   // first prefix sum past the target
+        atomicMin(&ctl.smp_pos, i);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const int pos = min(ctl.smp_pos, cl);
+    p.token_out[row] = static_cast<int64_t>(ci[pos]);
+    if (p.prob_out != nullptr) p.prob_out[row] = weight(pos) / ec;
+  }
+}
+
+// Rows no longer than k: the TopK output (every entry in index order, then
+// padding) and, for a sampling call, the draw among the n entries, which are
+// checked for NaN first (the softmax has no meaning with one).
+template <int DT, int THREADS>
+__device__ __noinline__ void finish_short_row(const KParams& p, int64_t row, int64_t n,
+                                              typename Elem<DT>::bits_t* cb, uint32_t* ci, Ctl& ctl) {
+  write_short_row<DT, THREADS>(p, row, n);
+  if (DT != DSEL_F32 || p.token_out == nullptr) return;
+  const uint32_t* xr = static_cast<const uint32_t*>(p.x) + row * p.row_stride;
+  bool nan = false;
+#pragma unroll 1
+  for (int i = threadIdx.x; i < n; i += THREADS) {
+    const uint32_t bits = xr[i];
+    cb[i] = static_cast<typename Elem<DT>::bits_t>(bits);
+    ci[i] = static_cast<uint32_t>(i);
+    nan |= Elem<DT>::is_nan(bits);
+  }
+  if (__syncthreads_or(nan)) {   // uniform
+    if (!p.nan_flag) nan_trap();   // the pages' default NaN policy
+    if (threadIdx.x == 0) {
+      p.token_out[row] = DSEL_IDX_NAN;
+      if (p.prob_out != nullptr) p.prob_out[row] = __int_as_float(0x7FC00000);
+    }
+    return;
+  }
+  bitonic_sort<DT, THREADS, true>(cb, ci, static_cast<int>(n));
+  sample_draw<THREADS>(p, row, reinterpret_cast<const uint32_t*>(cb), ci, static_cast<int>(n), ctl);
 }
 
 // Valid length of a row, with the end[] rules; *bad is set for an invalid end in
@@ -217,6 +364,7 @@ __device__ __noinline__ void finish_sorted(const KParams& p, int64_t row, int g,
   const int64_t obase = row * p.k + off;
   uint2* wsd = to_workspace ? p.ws_pairs + (row * p.groups + g) * static_cast<int64_t>(p.k) + off : nullptr;
   auto put = [&](int slot, int i) {
+    if (!to_workspace && p.indices_out == nullptr) return;
     if (to_workspace) {
       wsd[slot] = make_uint2(ci[i], static_cast<uint32_t>(cb[i]));
     } else {
@@ -292,6 +440,8 @@ __device__ __noinline__ void finish_sorted(const KParams& p, int64_t row, int g,
   }
   const int m = sel.depth == 0 ? n : holes_compact<DT, THREADS>(cb, ci, n, sel.kept, sel, p.idx_bits, ctl, holes);
   sort_kept<DT, THREADS>(cb, ci, m, sort_mode);
+  if (DT == DSEL_F32 && p.token_out != nullptr && !to_workspace && sort_mode == 2)   // the row's final candidates
+    sample_draw<THREADS>(p, row, reinterpret_cast<const uint32_t*>(cb), ci, m, ctl);
   emit<DT, THREADS>(p, row, g, to_workspace, off, m, total, write_meta, cb, ci);
 }
 
@@ -843,13 +993,13 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
   const int D = p.stages;
 #ifdef DSEL_STATS
   const long long st_t0 = clock64();
-  if (blockIdx.x == 0 && threadIdx.x == 0) g_trace[(kTraceRounds - 1) * kTraceEvents + kTraceEvents - 1] = st_t0;
+  if (blockIdx.x == g_trace_cta && threadIdx.x == 0) g_trace[(kTraceRounds - 1) * kTraceEvents + kTraceEvents - 1] = st_t0;
   long long st_t1 = st_t0;
   int st_rounds = 0;
   long long st_ev[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   long long st_wait = 0;
 #define DSEL_EV(i) do { if (tid == 0) st_ev[i] = clock64() - st_t0; } while (0)
-  const int tr_w = (blockIdx.x == 0 && lane == 0 && warp < kTraceWarps) ? warp : -1;
+  const int tr_w = (blockIdx.x == g_trace_cta && lane == 0 && warp < kTraceWarps) ? warp : -1;
 #define DSEL_TR(r, e) do { if (tr_w >= 0 && (r) < kTraceRounds - 2) \
     g_trace[(tr_w * kTraceRounds + (r)) * kTraceEvents + (e)] = clock64() - st_t0; } while (0)
 #else
@@ -857,19 +1007,17 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
 #define DSEL_TR(r, e) do { } while (0)
 #endif
 
-  bool bad_end;
-  const int64_t n = row_length(p, row, &bad_end);
-
 #pragma unroll 1
   for (int i = tid; i < 3 * kBins; i += THREADS) (&ctl.hist[0][0])[i] = 0;
-#pragma unroll 1
   {   // round-0 seed histograms: two levels of kSeedBins for large k, else 1024 bins
     static_assert(2 * kSeedBins <= kSeedSlots, "seed histograms fit the index array");
     const int nz = 2 * p.k > SG * THREADS ? 2 * kSeedBins : 1024;
+#pragma unroll 1
     for (int i = tid; i < nz; i += THREADS) seed_hist[i] = 0;
   }
   if (tid == 0) {
     ctl.t_w = 0ull;
+    ctl.add[0] = ctl.add[1] = ctl.add[2] = 0;
     ctl.nan_found = 0;
     ctl.abort = 0;
     ctl.hb = 0;
@@ -888,12 +1036,16 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
   if (C > 1) cluster.sync();   // peers' control blocks are ready before anyone touches them remotely
   else __syncthreads();
   DSEL_EV(0);
+  // the set-up above touched shared memory only: it may overlap the previous launch
+  grid_dependency_wait();
+  bool bad_end;
+  const int64_t n = row_length(p, row, &bad_end);
 
   const bool leader = (g == 0 && crank == 0);
   if (bad_end || n <= p.k) {
     if (p.groups == 1 && leader) {
       if (bad_end) write_sentinel_row<DT, THREADS>(p, row, DSEL_IDX_BAD_END);
-      else write_short_row<DT, THREADS>(p, row, n);
+      else finish_short_row<DT, THREADS>(p, row, n, cb, ci, ctl);
     }
   } else {
     // ---- this CTA's slice: [lo, hi), a multiple of 16 elements wide ----
@@ -953,7 +1105,8 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
       // any CTA's threshold is a valid bound for the whole row: push it to the peers
       if (C > 1 && warp == 0 && lane < C && lane != crank) atomicMax(cluster.map_shared_rank(&ctl.t_w, lane), co.tw);
     };
-    const int rounds = (nb + Q - 1) / Q;
+    // every CTA runs round 0, even on an empty slice: the cluster meets there
+    const int rounds = max(1, (nb + Q - 1) / Q);
 #pragma unroll 1
     for (int r = 0; r < rounds; ++r) {
       DSEL_TR(r, 0);
@@ -1027,6 +1180,15 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
           vlo = so.vlo;
           w = so.t > w ? so.t : w;
         }
+        if (C > 1) {
+          // every CTA's seed bounds the whole row: share them, so that a slice of
+          // low values screens against its neighbours' higher threshold
+          if (so.ok && warp == 0 && lane < C && lane != crank)
+            atomicMax(cluster.map_shared_rank(&ctl.t_w, lane), so.t);
+          cluster.sync();
+          const unsigned long long wp = *reinterpret_cast<volatile unsigned long long*>(&ctl.t_w);
+          w = wp > w ? wp : w;
+        }
         tk = static_cast<uint32_t>(w >> 32);
         ti = ~static_cast<uint32_t>(w);
         // a vector whose largest key is below T's key holds no survivor
@@ -1056,10 +1218,14 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
 
       DSEL_TR(r, 7);
 
-      // ---- 3. exact test of the flagged vectors (rare once T has settled) ----
-      Keep128 keep;            // bit v*PV + e: element e of vector v survives
-      keep.w[0] = keep.w[1] = 0ull;
-      if (__any_sync(0xffffffffu, maybe_mask != 0u)) {
+      // ---- 3. exact test of the flagged vectors, appended at once: per batch of
+      //      one vector per lane, the warp reserves slots with one shared atomic
+      //      on this round's counter; survivors past the buffer's end wait ----
+      const int radd = r % 3;
+      if (tid == 0) ctl.add[(r + 1) % 3] = 0;   // last read before the previous round's barrier
+      Keep128 pend;            // survivors of this thread: bit v*PV + e
+      pend.w[0] = pend.w[1] = 0ull;
+      {
 #ifdef DSEL_STATS
         if (lane == 0) atomicAdd(&ctl.st_slow_vectors, __popc(maybe_mask));
 #endif
@@ -1088,91 +1254,128 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
             nan_thread = true;
           }
           const int bit = v * PV;          // a vector's bits never straddle the two words
-          if (bit < 64) keep.w[0] |= static_cast<uint64_t>(kb) << bit;
-          else keep.w[1] |= static_cast<uint64_t>(kb) << (bit - 64);
+          if (bit < 64) pend.w[0] |= static_cast<uint64_t>(kb) << bit;
+          else pend.w[1] |= static_cast<uint64_t>(kb) << (bit - 64);
         }
-      }
-      int mine = keep.count();   // survivors of this thread not yet in the buffer
-      if (r == 0) DSEL_EV(2);
-      DSEL_TR(r, 2);
-
-      // ---- 4. append at offsets from per-warp counts; what does not fit waits ----
-      bool first = true;
-      while (true) {   // uniform: every thread takes the same path
-        const int wcount = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(mine)));
-        if (lane == 0) ctl.wc[par][warp] = wcount;
-        __syncthreads();
-        if (first) {
-          DSEL_TR(r, 3);
-          if (r == 0) DSEL_EV(3);
-          first = false;
-        }
-        int total;
-        const int woff = warp_prefix_of<NW>(ctl.wc[par], warp, lane, total);
-        par ^= 1;
-        const int space = cap - cnt;
-        DSEL_TR(r, 6);
-        if (wcount != 0) {   // warp-uniform
-          int rank = woff + warp_incl_scan(mine, lane) - mine;
+        // one reservation per warp for the round: a scan and one shared atomic
+        const int mine = pend.count();
+        const int incl = warp_incl_scan(mine, lane);
+        const int wtot = __shfl_sync(0xffffffffu, incl, 31);
+        if (wtot != 0) {   // warp-uniform
+          int base = 0;
+          if (lane == 0) base = atomicAdd(&ctl.add[radd], wtot);
+          int pos = cnt + __shfl_sync(0xffffffffu, base, 0) + incl - mine;
 #pragma unroll
           for (int wi = 0; wi < 2; ++wi) {
-            uint64_t kb = keep.w[wi];
-            while (kb) {
+            uint64_t kb = pend.w[wi];
+            while (kb && pos < cap) {   // slots past the buffer's end: the survivor waits
               const int bit = wi * 64 + __ffsll(static_cast<long long>(kb)) - 1;
               kb &= kb - 1ull;
-              if (rank < space) {
-                const int v = bit / PV, e = bit % PV;
-                uint32_t voff, eidx;
-                wr.locate(v, voff, eidx);
-                const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
-                const uint32_t bv = vec_elem_dyn<DT>(val, e);
-                cb[cnt + rank] = static_cast<bits_t>(bv);
-                ci[cnt + rank] = eidx + e;
-                const uint64_t vv = (static_cast<uint64_t>(E::key(bv)) << p.idx_bits) | (idx_mask - (eidx + e));
-                vmax = vv > vmax ? vv : vmax;   // largest radix word this thread wrote
-                keep.clr(bit);
-              }
-              ++rank;
+              const int v = bit / PV, e = bit % PV;
+              const uint32_t eidx = wr.eb + static_cast<uint32_t>(v * 32 * PV);
+              const uint4 val = *reinterpret_cast<const uint4*>(ring + wr.sb + v * 512);
+              const uint32_t bv = vec_elem_dyn<DT>(val, e);
+              cb[pos] = static_cast<bits_t>(bv);
+              ci[pos] = eidx + e;
+              const uint64_t vv = (static_cast<uint64_t>(E::key(bv)) << p.idx_bits) | (idx_mask - (eidx + e));
+              vmax = vv > vmax ? vv : vmax;   // largest radix word this thread wrote
+              pend.clr(bit);
+              ++pos;
             }
           }
         }
+      }
+      if (r == 0) DSEL_EV(2);
+      DSEL_TR(r, 2);
+
+      // ---- 4. the round's count (uniform after the barrier) ----
+      const bool my_pend = (pend.w[0] | pend.w[1]) != 0ull;
+      const bool warp_pend = __any_sync(0xffffffffu, my_pend);
+      // ---- 5. refill this warp's stage (no other warp reads it), unless waiting
+      //      survivors of the warp still have to be read from it ----
+      auto refill = [&]() {
+        __syncwarp();
+        if (lane == 0) {
+          fence_proxy_async();   // our reads of the stage come before the copy that overwrites it
+          if (j0 + D < nb) issue(j0 + D);
+        }
+      };
+      if (!warp_pend) refill();
+      const bool any_pend = __syncthreads_or(my_pend) != 0;
+      const int added = ctl.add[radd];
+      if (r == 0) DSEL_EV(3);
+      DSEL_TR(r, 3);
 #ifdef DSEL_STATS
-        if (tid == 0) ctl.st_appended += min(total, space);
+      if (tid == 0) ctl.st_appended += min(added, cap - cnt);
 #endif
-        if (total <= space) {
-          cnt += total;
-          break;
-        }
-        // buffer full: compact it, raise T, and re-test the survivors still waiting
+      if (!any_pend) {   // uniform
+        cnt += added;
+      } else {
+        // rare: the buffer filled up; compact it, raise T, re-test the waiting
+        // survivors and append them at offsets from per-warp counts
         cnt = cap;
-        compact(p.b2 / 2);
-        w = *reinterpret_cast<volatile unsigned long long*>(&ctl.t_w);
-        w = w > t_own ? w : t_own;
-        tk = static_cast<uint32_t>(w >> 32);
-        ti = ~static_cast<uint32_t>(w);
+        while (true) {   // uniform
+          compact(p.b2 / 2);
+          unsigned long long w2 = *reinterpret_cast<volatile unsigned long long*>(&ctl.t_w);
+          w2 = w2 > t_own ? w2 : t_own;
+          tk = static_cast<uint32_t>(w2 >> 32);
+          ti = ~static_cast<uint32_t>(w2);
+          int mine = 0;
 #pragma unroll
-        for (int wi = 0; wi < 2; ++wi) {
-          uint64_t kb = keep.w[wi];
-          while (kb) {
-            const int bit = wi * 64 + __ffsll(static_cast<long long>(kb)) - 1;
-            kb &= kb - 1ull;
-            const int v = bit / PV, e = bit % PV;
-            uint32_t voff, eidx;
-            wr.locate(v, voff, eidx);
-            const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
-            const uint32_t kk = E::key(vec_elem_dyn<DT>(val, e));
-            if (!(kk > tk || (kk == tk && eidx + e < ti))) keep.clr(bit);
+          for (int wi = 0; wi < 2; ++wi) {
+            uint64_t kb = pend.w[wi];
+            while (kb) {
+              const int bit = wi * 64 + __ffsll(static_cast<long long>(kb)) - 1;
+              kb &= kb - 1ull;
+              const int v = bit / PV, e = bit % PV;
+              uint32_t voff, eidx;
+              wr.locate(v, voff, eidx);
+              const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
+              const uint32_t kk = E::key(vec_elem_dyn<DT>(val, e));
+              if (!(kk > tk || (kk == tk && eidx + e < ti))) pend.clr(bit);
+              else ++mine;
+            }
           }
+          const int wcount = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(mine)));
+          if (lane == 0) ctl.wc[par][warp] = wcount;
+          __syncthreads();
+          int total;
+          const int woff = warp_prefix_of<NW>(ctl.wc[par], warp, lane, total);
+          par ^= 1;
+          const int space = cap - cnt;
+          if (wcount != 0) {   // warp-uniform
+            int rank = woff + warp_incl_scan(mine, lane) - mine;
+#pragma unroll
+            for (int wi = 0; wi < 2; ++wi) {
+              uint64_t kb = pend.w[wi];
+              while (kb) {
+                const int bit = wi * 64 + __ffsll(static_cast<long long>(kb)) - 1;
+                kb &= kb - 1ull;
+                if (rank < space) {
+                  const int v = bit / PV, e = bit % PV;
+                  uint32_t voff, eidx;
+                  wr.locate(v, voff, eidx);
+                  const uint4 val = *reinterpret_cast<const uint4*>(ring + voff);
+                  const uint32_t bv = vec_elem_dyn<DT>(val, e);
+                  cb[cnt + rank] = static_cast<bits_t>(bv);
+                  ci[cnt + rank] = eidx + e;
+                  const uint64_t vv = (static_cast<uint64_t>(E::key(bv)) << p.idx_bits) | (idx_mask - (eidx + e));
+                  vmax = vv > vmax ? vv : vmax;
+                  pend.clr(bit);
+                }
+                ++rank;
+              }
+            }
+          }
+          if (total <= space) {
+            cnt += total;
+            break;
+          }
+          cnt = cap;
         }
-        mine = keep.count();
+        if (warp_pend) refill();
       }
       DSEL_TR(r, 4);
-      // ---- 5. refill this warp's stage: no other warp reads it ----
-      __syncwarp();
-      if (lane == 0) {
-        fence_proxy_async();   // our reads of the stages come before the copies that overwrite them
-        if (j0 + D < nb) issue(j0 + D);
-      }
 #ifdef DSEL_STATS
       ++st_rounds;
 #endif
@@ -1203,6 +1406,7 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
     st_t1 = clock64();
 #endif
     DSEL_EV(5);
+    grid_launch_dependents();   // the next launch may start its prologue during the final phase
 
     const bool to_ws = p.groups > 1;
     const int sort_mode = to_ws ? (p.order == DSEL_ORDER_INDEX ? 1 : 0) : p.order;
@@ -1260,8 +1464,6 @@ __global__ void __launch_bounds__(THREADS, 1) topk_merge_kernel(const __grid_con
   const int tid = threadIdx.x;
   const int64_t row = static_cast<int64_t>(blockIdx.x) / C;
 
-  bool bad_end;
-  const int64_t n = row_length(p, row, &bad_end);
 #pragma unroll 1
   for (int i = tid; i < 3 * kBins; i += THREADS) (&ctl.hist[0][0])[i] = 0;
   if (tid == 0) {
@@ -1272,10 +1474,13 @@ __global__ void __launch_bounds__(THREADS, 1) topk_merge_kernel(const __grid_con
   }
   if (C > 1) cluster.sync();
   else __syncthreads();
+  grid_dependency_wait();   // the streaming launch's workspace is complete and visible
+  bool bad_end;
+  const int64_t n = row_length(p, row, &bad_end);
   if (bad_end || n <= p.k) {
     if (crank == 0) {
       if (bad_end) write_sentinel_row<DT, THREADS>(p, row, DSEL_IDX_BAD_END);
-      else write_short_row<DT, THREADS>(p, row, n);
+      else finish_short_row<DT, THREADS>(p, row, n, cb, ci, ctl);
     }
   } else {
     // group prefix sums (groups <= kBins) in the histogram scratch

@@ -79,6 +79,35 @@ def test_host_argument_checks(kw, err):
     assert call(**kw) == header_define(err)
 
 
+def call_sample(**kw):
+    a = dict(x=0x1000, rows=4, row_stride=8192, end=None, k=64, temperature=1.0, top_p=0.9, u=0x4000,
+             nan_mode=T.DSEL_NAN_FLAG, values_out=0x2000, indices_out=0x3000, token_out=0x5000, prob_out=None,
+             stream=None)
+    a.update(kw)
+    return T.dsel_topk_sample(**a)
+
+
+@pytest.mark.parametrize("kw,err", [
+    (dict(k=0), "DSEL_ERR_K"),
+    (dict(k=4097), "DSEL_ERR_K"),
+    (dict(rows=-1), "DSEL_ERR_ROWS"),
+    (dict(row_stride=8190), "DSEL_ERR_STRIDE"),
+    (dict(nan_mode=5), "DSEL_ERR_NAN_MODE"),
+    (dict(x=None), "DSEL_ERR_NULL"),
+    (dict(u=None), "DSEL_ERR_NULL"),
+    (dict(token_out=None), "DSEL_ERR_NULL"),
+    (dict(values_out=None), "DSEL_ERR_VALUES"),
+    (dict(indices_out=None), "DSEL_ERR_VALUES"),
+    (dict(x=0x1008), "DSEL_ERR_ALIGN"),
+])
+def test_sample_host_argument_checks(kw, err):
+    assert call_sample(**kw) == header_define(err)
+
+
+def test_sample_zero_rows_is_a_noop():
+    assert call_sample(rows=0, x=None, u=None, token_out=None) == 0
+
+
 def test_zero_rows_is_a_noop():
     assert call(rows=0, x=None, indices_out=None, values_out=None, return_value=0) == 0
 

@@ -159,6 +159,13 @@ def sampler_logits(batch: int, k: int, seed: int = 3, vocab: int = SAMPLER_VOCAB
                     sorted_index=1, return_value=1, index_dtype="i64")
 
 
+def uniforms(rows: int, seed: int = 5) -> np.ndarray:
+    """One float32 uniform in [0, 1) per row: the random numbers of a sampling draw,
+    passed to the draw as an input."""
+    rng = np.random.default_rng(seed)
+    return rng.random(rows, dtype=np.float32)
+
+
 def long_rows(rows: int, n: int, k: int, variant: str = "uniform", seed: int = 4,
               inject_nan: bool = False) -> Workload:
     """float32 long rows, U[-1, 1] (``uniform``), sorted descending (``desc``) or all
