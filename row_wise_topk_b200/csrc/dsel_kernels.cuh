@@ -527,10 +527,22 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
       cluster.sync();
       lo = 0ull;
     }
-    if (crank != 0) return;
+    // the CTA holding the most candidates gathers the others' (ties: the lower
+    // rank), so that the fewest cross the cluster: under a drift across the row
+    // one slice holds nearly all of them
+    int held = 0;
+    if (lane < C) {
+      Ctl* pc = cluster.map_shared_rank(&ctl, lane);
+      held = direct ? pc->x_cnt : pc->x_kept;
+    }
+    const unsigned lkey = __reduce_max_sync(
+        0xffffffffu, lane < C ? (static_cast<unsigned>(held) << 8) | static_cast<unsigned>(255 - lane) : 0u);
+    const int leader = 255 - static_cast<int>(lkey & 255u);
+    if (crank != leader) return;
     int off = m;
 #pragma unroll 1
-    for (int r = 1; r < C; ++r) {
+    for (int r = 0; r < C; ++r) {
+      if (r == leader) continue;
       Ctl* pr = cluster.map_shared_rank(&ctl, r);
       const int mr = direct ? pr->x_cnt : pr->x_kept;
       const bits_t* rcb = cluster.map_shared_rank(cb, r);
@@ -1170,6 +1182,13 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
             so.t = make_w(tkey, 0xFFFFFFFFu);     // passes every key >= tkey
             so.vlo = static_cast<uint64_t>(tkey) << p.idx_bits;
             so.ok = true;
+          } else {
+            // fewer than k group maxima (a short slice): seed from the elements
+            // themselves rather than start at -inf and take the whole slice in
+#pragma unroll 1
+            for (int i = tid; i < 2 * kSeedBins; i += THREADS) seed_hist[i] = 0;
+            __syncthreads();
+            so = seed_threshold<DT, THREADS, VPT>(ring, wr, p.k, p.idx_bits, ctl, seed_hist);
           }
         } else {
           so = seed_threshold<DT, THREADS, VPT>(ring, wr, p.k, p.idx_bits, ctl, seed_hist);
