@@ -275,6 +275,7 @@ struct __align__(16) Ctl {
   int st_compactions;
   int st_appended;
   int st_slow_vectors;
+  int st_refetch;                 // passes restarted because a sampled seed was not certified
 #endif
 };
 

@@ -916,12 +916,13 @@ __device__ __noinline__ SeedOut seed_threshold(const unsigned char* ring, WarpRo
 
 // ---------------------------------------------------------------------------
 // Bulk copy of the j-th block in visiting order, (pa * j + pc) mod nb, of the
-// slice [lo, hi) into ring stage j mod D.  Out of line: it is called from the
+// slice [lo, hi) into ring stage jg mod D (jg: the CTA's running block count).  Out of line: it is called from the
 // prologue and from every refill, and inlining would repeat its 64-bit modulo.
 // ---------------------------------------------------------------------------
 template <int DT>
-__device__ __noinline__ void issue_block(int j, uint32_t pa, uint32_t pc, int nb, int64_t lo, int64_t hi, int D,
-                                         const char* rowp, unsigned char* ring, uint64_t* bars, uint32_t* blk_off) {
+__device__ __noinline__ void issue_block(int j, int jg, uint32_t pa, uint32_t pc, int nb, int64_t lo, int64_t hi,
+                                         int D, const char* rowp, unsigned char* ring, uint64_t* bars,
+                                         uint32_t* blk_off) {
   using E = Elem<DT>;
   constexpr int B = block_elems_for(E::kBytes);
   const uint32_t m = static_cast<uint32_t>((static_cast<uint64_t>(pa) * static_cast<uint32_t>(j) + pc) %
@@ -929,7 +930,7 @@ __device__ __noinline__ void issue_block(int j, uint32_t pa, uint32_t pc, int nb
   const int64_t e0 = lo + static_cast<int64_t>(m) * B;
   const int64_t ce = min(static_cast<int64_t>(B), hi - e0);
   const uint32_t bytes = static_cast<uint32_t>((ce * E::kBytes + 15) & ~static_cast<int64_t>(15));
-  const int s = j % D;
+  const int s = jg % D;   // jg counts every block this CTA has issued: stages and phases run on
   blk_off[s] = static_cast<uint32_t>(e0);
   const uint32_t bar = smem_u32(&bars[s]);
   mbar_expect_tx(bar, bytes);
@@ -1038,6 +1039,7 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
     ctl.st_compactions = 0;
     ctl.st_appended = 0;
     ctl.st_slow_vectors = 0;
+    ctl.st_refetch = 0;
 #endif
   }
 #pragma unroll 1
@@ -1086,17 +1088,10 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
                          (static_cast<uint64_t>(sid) + 1) * 0xBF58476D1CE4E5B9ull;
       pc = static_cast<uint32_t>((h >> 29) % unb);
     }
+    int jb = 0;   // blocks issued in earlier passes over the slice
     auto issue = [&](int j) {
-      issue_block<DT>(j, pa, pc, nb, lo, hi, D, rowp, ring, bars, blk_off);
+      issue_block<DT>(j, jb + j, pa, pc, nb, lo, hi, D, rowp, ring, bars, blk_off);
     };
-    {   // prologue: the first D blocks, each issued by lane 0 of the warp that owns its stage
-      const int first = min(D, nb);
-#pragma unroll 1
-      for (int j = warp; j < first; j += Q) {
-        if (lane == 0) issue(j);
-      }
-    }
-    DSEL_EV(1);
 
     const uint32_t uhi = static_cast<uint32_t>(hi);
     const uint32_t idx_mask = mask_bits(p.idx_bits);
@@ -1119,8 +1114,27 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
     };
     // every CTA runs round 0, even on an empty slice: the cluster meets there
     const int rounds = max(1, (nb + Q - 1) / Q);
+    int rg = 0;              // rounds run so far over all passes (per-round counters rotate on it)
+    bool spec = false;       // round 0 seeded T from a sample: certified at the end of the pass
+    bool compacted = false;  // a compaction ran in this pass
 #pragma unroll 1
-    for (int r = 0; r < rounds; ++r) {
+    for (int pass = 0;; ++pass) {
+    {   // prologue: the pass's first D blocks, each issued by lane 0 of the warp that owns its stage
+      if (pass > 0) {   // the previous pass's reads of the ring come before these copies
+        __syncthreads();
+      }
+      const int first = min(D, nb);
+#pragma unroll 1
+      for (int j = warp; j < first; j += Q) {
+        if (lane == 0) {
+          if (pass > 0) fence_proxy_async();
+          issue(j);
+        }
+      }
+    }
+    DSEL_EV(1);
+#pragma unroll 1
+    for (int r = 0; r < rounds; ++r, ++rg) {
       DSEL_TR(r, 0);
       WarpRound<DT> wr;
       wr.j0 = r * Q + warp;                            // the block this warp owns in the round
@@ -1131,11 +1145,12 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
       const int j0 = wr.j0;
       // ---- 1. wait for the owned block ----
       if (wr.owns) {   // warp-uniform
-        const int st = j0 % D;
+        const int jg = jb + j0;
+        const int st = jg % D;
 #ifdef DSEL_STATS
         const long long w0 = clock64();
 #endif
-        if (!mbar_wait(smem_u32(&bars[st]), static_cast<uint32_t>((j0 / D) & 1))) ctl.abort = 1;
+        if (!mbar_wait(smem_u32(&bars[st]), static_cast<uint32_t>((jg / D) & 1))) ctl.abort = 1;
 #ifdef DSEL_STATS
         st_wait += clock64() - w0;
 #endif
@@ -1175,9 +1190,29 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
         }
         DSEL_TR(r, 1);
         SeedOut so{0ull, 0ull, false};
-        if (2 * p.k <= SG * THREADS) {
-          // the k-th largest group maximum: k distinct elements are at or above it
-          const uint32_t tkey = cta_kth_largest<THREADS, SG>(gm, p.k, ctl, seed_hist);
+        // Sampled seed: when this CTA streams a whole row in several rounds, the
+        // round's blocks (visited in random order) are a random sample of the row;
+        // T goes near the expected number of the row's top k in it, plus a wide
+        // margin (6 standard deviations).  It is certified after the pass.
+        int kseed = p.k;
+        if (pass == 0 && C == 1 && p.groups == 1 && rounds > 1) {
+          const float n_sl = static_cast<float>(hi - lo);
+          const float m0 = fminf(n_sl, static_cast<float>(R));
+          const float e = static_cast<float>(p.k) * m0 / n_sl;
+          const int j = static_cast<int>(ceilf(e + 6.0f * sqrtf(e) + 16.0f));
+          if (j < p.k) {
+            kseed = j;
+            spec = true;
+          }
+        }
+        if (pass > 0) {   // the histograms still hold the previous pass's seed
+#pragma unroll 1
+          for (int i = tid; i < 2 * kSeedBins; i += THREADS) seed_hist[i] = 0;
+          __syncthreads();
+        }
+        if (2 * kseed <= SG * THREADS) {
+          // the kseed-th largest group maximum: kseed distinct elements are at or above it
+          const uint32_t tkey = cta_kth_largest<THREADS, SG>(gm, kseed, ctl, seed_hist);
           if (tkey != 0u) {   // uniform
             so.t = make_w(tkey, 0xFFFFFFFFu);     // passes every key >= tkey
             so.vlo = static_cast<uint64_t>(tkey) << p.idx_bits;
@@ -1188,11 +1223,12 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
 #pragma unroll 1
             for (int i = tid; i < 2 * kSeedBins; i += THREADS) seed_hist[i] = 0;
             __syncthreads();
-            so = seed_threshold<DT, THREADS, VPT>(ring, wr, p.k, p.idx_bits, ctl, seed_hist);
+            so = seed_threshold<DT, THREADS, VPT>(ring, wr, kseed, p.idx_bits, ctl, seed_hist);
           }
         } else {
-          so = seed_threshold<DT, THREADS, VPT>(ring, wr, p.k, p.idx_bits, ctl, seed_hist);
+          so = seed_threshold<DT, THREADS, VPT>(ring, wr, kseed, p.idx_bits, ctl, seed_hist);
         }
+        spec = spec && so.ok;
         DSEL_TR(r, 9);
         if (so.ok) {
           t_own = so.t;
@@ -1240,8 +1276,8 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
       // ---- 3. exact test of the flagged vectors, appended at once: per batch of
       //      one vector per lane, the warp reserves slots with one shared atomic
       //      on this round's counter; survivors past the buffer's end wait ----
-      const int radd = r % 3;
-      if (tid == 0) ctl.add[(r + 1) % 3] = 0;   // last read before the previous round's barrier
+      const int radd = rg % 3;
+      if (tid == 0) ctl.add[(rg + 1) % 3] = 0;   // last read before the previous round's barrier
       Keep128 pend;            // survivors of this thread: bit v*PV + e
       pend.w[0] = pend.w[1] = 0ull;
       {
@@ -1335,6 +1371,7 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
         cnt = cap;
         while (true) {   // uniform
           compact(p.b2 / 2);
+          compacted = true;
           unsigned long long w2 = *reinterpret_cast<volatile unsigned long long*>(&ctl.t_w);
           w2 = w2 > t_own ? w2 : t_own;
           tk = static_cast<uint32_t>(w2 >> 32);
@@ -1404,6 +1441,7 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
         const long long sc0 = clock64();
 #endif
         compact(p.b2 / 2);
+        compacted = true;
 #ifdef DSEL_STATS
         if (tid == 0) {
           ctl.st_compactions += 1;
@@ -1414,12 +1452,27 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
       }
       DSEL_TR(r, 5);
     }
+    // A sampled threshold holds only if at least k elements reached it; a
+    // compaction proves that (it runs at k + B2 candidates).  Otherwise stream
+    // the slice again with a proven seed (all values uniform in the CTA).
+    if (!(spec && !compacted && cnt < p.k) || ctl.abort) break;
+#ifdef DSEL_STATS
+    if (tid == 0) ctl.st_refetch += 1;
+#endif
+    jb += nb;
+    spec = false;
+    compacted = false;
+    cnt = 0;
+    t_own = 0ull;
+    vlo = 0ull;
+    vmax = 0ull;
+    }
     // A wait that gave up may leave a copy in flight: wait for it (bounded) before
     // this CTA's shared memory can go away.
     __syncthreads();
     if (ctl.abort && tid == 0) {
 #pragma unroll 1
-      for (int j = max(0, nb - D); j < nb; ++j) mbar_wait(smem_u32(&bars[j % D]), (j / D) & 1);
+      for (int j = max(0, nb - D); j < nb; ++j) mbar_wait(smem_u32(&bars[(jb + j) % D]), ((jb + j) / D) & 1);
     }
 #ifdef DSEL_STATS
     st_t1 = clock64();
@@ -1448,7 +1501,7 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
     st[4] = static_cast<unsigned long long>(ctl.st_appended);
     st[5] = static_cast<unsigned long long>(ctl.st_slow_vectors);
     st[6] = static_cast<unsigned long long>(st_rounds);
-    st[7] = 0;
+    st[7] = static_cast<unsigned long long>(ctl.st_refetch);
 #pragma unroll 1
     for (int i = 0; i < 6; ++i) st[8 + i] = static_cast<unsigned long long>(st_ev[i]);
     st[14] = static_cast<unsigned long long>(st_wait);
