@@ -18,7 +18,7 @@ struct DevInfo {
   int sms = 0;
   int smem_optin = 0;
   int major = 0;
-  bool attrs_set[2][2] = {{false, false}, {false, false}};   // [dtype][short shape]
+  bool attrs_set[2][3] = {{false, false, false}, {false, false, false}};   // [dtype][shape]
 };
 
 std::mutex g_mu;
@@ -102,7 +102,7 @@ template <int DT, int THREADS>
 int run_shape(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
   auto sk = topk_stream_kernel<DT, THREADS>;
   auto mk = topk_merge_kernel<DT, kThreads>;
-  constexpr int shp = THREADS == kThreads ? 0 : 1;
+  constexpr int shp = THREADS == kThreads ? 0 : (THREADS == kThreadsMid ? 1 : 2);
   if (!di->attrs_set[DT][shp]) {
     if (cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) != cudaSuccess ||
         cudaFuncSetAttribute(sk, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
@@ -142,6 +142,7 @@ int run_shape(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStre
 template <int DT>
 int run(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
   if (pl.threads == kThreadsShort) return run_shape<DT, kThreadsShort>(base, pl, rows, st, di);
+  if (pl.threads == kThreadsMid) return run_shape<DT, kThreadsMid>(base, pl, rows, st, di);
   if (pl.threads == kThreads) return run_shape<DT, kThreads>(base, pl, rows, st, di);
   return DSEL_ERR_DEVICE;
 }

@@ -5,9 +5,13 @@
 // should sit "on the order of k"; B2 follows them, B is one warp's share of a
 // round (4096 bf16 / 1024 f32 elements, see block_elems_for), and everything
 // else here is this library's choice for a 148-SM B200:
-//   * one CTA per row while there are at least as many rows as SMs; when rows
-//     are also short (at most two 128-thread rounds), a 128-thread CTA, several
-//     per SM, each with at most one round of blocks in flight;
+//   * one CTA per row while there are at least as many rows as SMs:
+//       - rows of at most two 128-thread rounds: a 128-thread CTA, several per
+//         SM, each with at most one round of blocks in flight;
+//       - longer rows with k <= 1024: a 256-thread CTA when two fit an SM (two
+//         rows per SM: one wave for up to 2 x SMs rows, and one CTA's barrier
+//         waits overlap the other's work);
+//       - otherwise a 512-thread CTA, one per SM;
 //   * otherwise each row is cut into S contiguous slices, one CTA each, grouped in
 //     thread-block clusters of C CTAs that share the threshold and merge through
 //     distributed shared memory; rows too long for one cluster (S > max_cluster)
@@ -32,6 +36,28 @@ int check_shape(int dtype, int64_t rows, int64_t row_stride, int32_t k) {
 static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 static int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 
+namespace {
+
+// Buffer sizes and block geometry for one CTA shape (ring depth still open).
+void shape_plan(int dtype, int32_t k, int threads, dsel_plan_t* p) {
+  p->threads = threads;
+  p->block = block_elems(dtype);
+  p->round = round_elems(dtype, threads);
+  p->b2 = k <= 1024 ? 1024 : std::min(k, 2048);
+  // k + B2 + slack; a round's survivors beyond that wait in registers until a
+  // compaction makes room, so the round may be larger than the slack;
+  // at least kSeedSlots: the round-0 seed histograms live in the index array
+  p->capacity = int(round_up(
+      std::max<int64_t>({int64_t(k) + p->b2 + append_slack(k, threads), int64_t(next_pow2(k)), int64_t(kSeedSlots)}),
+      32));
+}
+
+int64_t shape_smem(const dsel_plan_t& p, int64_t stages, int32_t k, int eb) {
+  return stream_layout(stages, p.block, p.capacity, int64_t(k) + p.b2, eb).total;
+}
+
+}  // namespace
+
 int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t num_sms,
               int32_t smem_optin, int32_t max_cluster, dsel_plan_t* out) {
   int st = check_shape(dtype, rows, row_stride, k);
@@ -41,22 +67,31 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
 
   const int eb = elem_bytes(dtype);
   dsel_plan_t p{};
-  const bool short_rows = rows >= num_sms && row_stride <= 2 * int64_t(round_elems(dtype, kThreadsShort));
-  p.threads = short_rows ? kThreadsShort : kThreads;
-  p.block = block_elems(dtype);
-  p.round = round_elems(dtype, p.threads);
-  p.b2 = k <= 1024 ? 1024 : std::min(k, 2048);
-  // k + B2 + slack; a round's survivors beyond that wait in registers until a
-  // compaction makes room, so the round may be larger than the slack
-  // at least kSeedSlots: the round-0 seed histograms live in the index array
-  p.capacity = int(round_up(
-      std::max<int64_t>({int64_t(k) + p.b2 + append_slack(k, p.threads), int64_t(next_pow2(k)), int64_t(kSeedSlots)}),
-      32));
+  const bool one_per_row = rows >= num_sms;
+  const bool short_rows = one_per_row && row_stride <= 2 * int64_t(round_elems(dtype, kThreadsShort));
+
+  // 256-thread shape: two CTAs per SM (half of the SM's shared memory each, less
+  // the 1 KB the hardware reserves per CTA) with at least one round in flight
+  int64_t mid_stages = 0;
+  if (one_per_row && !short_rows && k <= 1024) {
+    dsel_plan_t m{};
+    shape_plan(dtype, k, kThreadsMid, &m);
+    const int64_t budget = (int64_t(smem_optin) + 1024) / 2 - 1024;
+    const int64_t nb = ceil_div(row_stride, m.block);
+    const int64_t q = m.round / m.block;
+    for (int64_t s = std::min<int64_t>(nb, 2 * q); s >= std::min<int64_t>(nb, q); --s) {
+      if ((s == nb || s % q == 0) && shape_smem(m, s, k, eb) <= budget) {
+        mid_stages = s;
+        break;
+      }
+    }
+  }
+  shape_plan(dtype, k, short_rows ? kThreadsShort : (mid_stages > 0 ? kThreadsMid : kThreads), &p);
   p.idx_bits = ceil_log2_u64(uint64_t(row_stride));
 
   // Row split.
   int64_t splits = 1;
-  if (rows < num_sms) {
+  if (!one_per_row) {
     splits = num_sms / std::max<int64_t>(rows, 1);
     splits = std::min<int64_t>(splits, std::max<int64_t>(1, row_stride / kMinSliceElems));
     splits = std::max<int64_t>(splits, 1);
@@ -74,12 +109,14 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
   const int64_t slice = round_up(ceil_div(row_stride, groups * cluster), kStrideReq);
   const int64_t nb_max = ceil_div(slice, p.block);
   const int64_t per_round = p.round / p.block;
-  const int64_t base = stream_layout(0, p.block, p.capacity, int64_t(k) + p.b2, eb).total + 256;
+  const int64_t base = shape_smem(p, 0, k, eb) + 256;
   const int64_t per_stage = int64_t(p.block) * eb + 8 + 4;
   int64_t stages = (int64_t(smem_optin) - base) / per_stage;
   stages = std::min<int64_t>(stages, kMaxStages);
   if (short_rows) {
     stages = std::min(nb_max, per_round);    // one round in flight: keeps several CTAs per SM
+  } else if (mid_stages > 0) {
+    stages = mid_stages;                     // two CTAs per SM
   } else if (nb_max <= stages) {
     stages = nb_max;                         // the whole slice in flight at once, no refills
   } else {
@@ -87,7 +124,7 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
   }
   stages = std::max<int64_t>(stages, std::min<int64_t>(per_round, nb_max));
   p.stages = int(stages);
-  const int64_t smem = stream_layout(stages, p.block, p.capacity, int64_t(k) + p.b2, eb).total;
+  const int64_t smem = shape_smem(p, stages, k, eb);
   if (smem > smem_optin) return DSEL_ERR_K;
   p.smem_bytes = int(smem);
 

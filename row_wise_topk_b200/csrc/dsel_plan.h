@@ -9,10 +9,11 @@ namespace dsel {
 
 // Compile-time CTA shapes.  The streaming kernel is instantiated for exactly
 // these (dtype, threads) pairs; the planner only ever returns one of them:
-// 512 threads, one CTA per SM, for long rows and split rows; 128 threads for
-// many short rows, so that several rows share an SM and one CTA's loads overlap
-// another's selection.
+// 512 threads, one CTA per SM, for long rows and split rows; 256 threads, two per
+// SM, for batches of long rows with k <= 1024; 128 threads for many short rows,
+// so that several rows share an SM and one CTA's loads overlap another's work.
 constexpr int kThreads = 512;
+constexpr int kThreadsMid = 256;
 constexpr int kThreadsShort = 128;
 constexpr int kVecBytes = 16;                 // one 128-bit shared-memory load per vector
 // Vectors each thread screens per round (a warp owns whole blocks): 16 for bf16
@@ -23,7 +24,7 @@ constexpr int vecs_per_thread_for(int eb) { return eb == 2 ? 16 : 8; }
 // Candidate-buffer slots beyond k + B2.  A round's survivors that do not fit
 // wait until a compaction makes room, so this need not cover a whole round.
 inline int append_slack(int k, int threads) {
-  if (threads == kThreadsShort) return 1024;
+  if (threads != kThreads) return 1024;
   return k <= 1024 ? 4096 : 2048;
 }
 constexpr int kSeedSlots = 4096;              // candidate slots that hold the round-0 seed histograms

@@ -120,7 +120,7 @@ PEAK = dict(num_sms=148, smem_optin=232448, max_cluster=8)
     (T.DSEL_BF16, 64, 131072, 512),
     (T.DSEL_BF16, 4096, 16384, 512),
     (T.DSEL_F32, 1, 129280, 50), (T.DSEL_F32, 8, 129280, 1024), (T.DSEL_F32, 64, 129280, 4096),
-    (T.DSEL_F32, 256, 129280, 4096),
+    (T.DSEL_F32, 256, 129280, 4096), (T.DSEL_F32, 256, 129280, 1024), (T.DSEL_BF16, 300, 131072, 512),
     (T.DSEL_F32, 1, 1 << 28, 1000), (T.DSEL_F32, 16, 1 << 24, 4096),
     (T.DSEL_BF16, 3, 16, 4096), (T.DSEL_F32, 1, 16, 1),
 ])
@@ -129,7 +129,7 @@ def test_plan_invariants(dtype, rows, stride, k):
     assert st == 0
     eb = 2 if dtype == T.DSEL_BF16 else 4
     assert p["smem_bytes"] <= PEAK["smem_optin"]
-    slack = 1024 if p["threads"] == 128 else (4096 if k <= 1024 else 2048)
+    slack = 1024 if p["threads"] != 512 else (4096 if k <= 1024 else 2048)
     assert p["capacity"] >= k + p["b2"] + slack
     assert p["capacity"] >= 1 << (k - 1).bit_length()          # room for the bitonic padding
     assert p["capacity"] >= 4096                                 # the round-0 seed histograms
@@ -137,12 +137,16 @@ def test_plan_invariants(dtype, rows, stride, k):
     slice_ = -(-(-(-stride // (p["cluster"] * p["groups"]))) // 16) * 16
     nb_max = -(-slice_ // p["block"])
     assert p["stages"] == nb_max or (p["stages"] % q == 0 and p["stages"] < nb_max)
-    assert p["threads"] in (128, 512)
+    assert p["threads"] in (128, 256, 512)
     assert p["round"] == p["threads"] * (16 if dtype == T.DSEL_BF16 else 8) * (16 // eb)
     if p["threads"] == 128:   # short rows: one CTA per row, one round in flight, several CTAs per SM
         assert rows >= PEAK["num_sms"] and stride <= 2 * p["round"]
         assert (p["cluster"], p["groups"]) == (1, 1) and p["stages"] <= q
         assert p["smem_bytes"] <= 232448 // 2
+    if p["threads"] == 256:   # long rows, k <= 1024: one CTA per row, two CTAs per SM
+        assert rows >= PEAK["num_sms"] and k <= 1024
+        assert (p["cluster"], p["groups"]) == (1, 1)
+        assert 2 * (p["smem_bytes"] + 1024) <= PEAK["smem_optin"] + 1024
     assert p["round"] % p["block"] == 0 and (p["block"] * eb) % 16 == 0
     assert 1 <= p["cluster"] <= PEAK["max_cluster"]
     assert p["groups"] >= 1 and p["groups"] * k <= 8 * p["capacity"]
@@ -161,6 +165,8 @@ def test_plan_splits():
     p = T.dsel_plan(T.DSEL_BF16, 4096, 16384, 512, **PEAK)[1]
     assert p["cluster"] == 1 and p["threads"] == 128
     assert T.dsel_plan(T.DSEL_F32, 256, 129280, 4096, **PEAK)[1]["threads"] == 512
+    # long rows, k <= 1024, at least as many rows as SMs: 256 threads, two CTAs per SM
+    assert T.dsel_plan(T.DSEL_F32, 256, 129280, 1024, **PEAK)[1]["threads"] == 256
     # 64 indexer rows: two CTAs per row
     p = T.dsel_plan(T.DSEL_BF16, 64, 131072, 512, **PEAK)[1]
     assert (p["cluster"], p["groups"]) == (2, 1)

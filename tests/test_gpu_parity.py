@@ -173,6 +173,25 @@ def test_short_row_shape(seed, dtype, rows, stride, k, dist, order):
     check(w, order=order)
 
 
+MID = [
+    # (seed, dtype, rows, stride, k, dist, order): the 256-thread shape, two CTAs per SM
+    (401, "f32", 150, 65536, 1024, "normal", 1),
+    (402, "f32", 160, 40960, 50, "ties", 0),
+    (403, "bf16", 152, 131072, 512, "ascending", 1),
+    (404, "f32", 149, 16400, 700, "equal", 2),
+]
+
+
+@pytest.mark.parametrize("seed,dtype,rows,stride,k,dist,order", MID)
+def test_mid_row_shape(seed, dtype, rows, stride, k, dist, order):
+    st, plan = T.dsel_plan(T.DSEL_BF16 if dtype == "bf16" else T.DSEL_F32, rows, stride, k,
+                           num_sms=torch.cuda.get_device_properties(0).multi_processor_count)
+    assert st == 0 and plan["threads"] == 256, "the case must use the 256-thread shape"
+    w = W.random_small(seed, dtype, rows, stride, k, dist=dist, with_end=(seed % 2 == 0),
+                       end_lo=0, sorted_index=1, return_value=1, index_dtype="i64")
+    check(w, order=order)
+
+
 def test_pr1_duplicates_full():
     check(W.pr1_duplicates())
 
