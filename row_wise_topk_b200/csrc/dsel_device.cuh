@@ -505,6 +505,117 @@ __device__ __noinline__ SelResult radix_select(const typename Elem<DT>::bits_t* 
   return {prefix, depth, kept};
 }
 
+// The need-th largest radix word among the n candidates whose key lies in
+// [klo, khi] (at most kTieMax of them, `members`): gathered into a short list,
+// each ranked by its whole word, which is unique.  ctl.tie_n must be zero on
+// entry and ordered by an earlier barrier.  Two barriers.
+template <int DT, int THREADS>
+__device__ __noinline__ uint64_t rank_members(const typename Elem<DT>::bits_t* cb, const uint32_t* ci, int n,
+                                              uint32_t klo, uint32_t khi, int members, int need, int idx_bits,
+                                              Ctl& ctl) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t idx_mask = mask_bits(idx_bits);
+  unsigned long long* lst = reinterpret_cast<unsigned long long*>(ctl.hsum);
+#pragma unroll 1
+  for (int i0 = 0; i0 < n; i0 += THREADS) {   // same trip count in every thread
+    const int i = i0 + tid;
+    uint64_t v = 0;
+    bool in = false;
+    if (i < n) {
+      const uint32_t key = Elem<DT>::key(cb[i]);
+      in = key >= klo && key <= khi;
+      v = make_v<DT>(cb[i], ci[i], idx_bits, idx_mask);
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, in);
+    int base = 0;
+    if (lane == 0 && bal != 0u) base = atomicAdd(&ctl.tie_n, __popc(bal));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (in) lst[base + __popc(bal & ((1u << lane) - 1u))] = v;
+  }
+  __syncthreads();
+  if (tid < members) {   // the member with need - 1 larger words is the need-th
+    const unsigned long long vj = lst[tid];
+    int r = 0;
+#pragma unroll 4
+    for (int i = 0; i < members; ++i) r += lst[i] > vj ? 1 : 0;
+    if (r == need - 1) ctl.tie_v = vj;
+  }
+  __syncthreads();
+  return ctl.tie_v;
+}
+
+// Exact selection of the k best of n candidates (all radix words in [vlo, vhi]),
+// as a SelResult, starting with one pass of a histogram of 1024 bins spread
+// evenly over the candidates' key range (bins of 2^sh keys; one key per bin when
+// the range is under 1024 keys, as bf16 candidates usually are).  Radix digits
+// aligned to key bits put the first digit on the exponent, so on data with few
+// distinct values nearly all candidates fall into one or two bins and their
+// atomics serialise; the range-adaptive bins do not.  The boundary bin is then
+// finished by ranking its members (at most kTieMax) or, failing that, by the
+// radix select (restricted to the boundary key when bins are single keys).
+// `hist` is 1024 ints of scratch, 16-byte aligned.
+template <int DT, int THREADS>
+__device__ __noinline__ SelResult select_by_key_hist(const typename Elem<DT>::bits_t* cb, const uint32_t* ci, int n,
+                                                     int k, int idx_bits, uint64_t vlo, uint64_t vhi, Ctl& ctl,
+                                                     int* hist, cg::cluster_group& cluster) {
+  using E = Elem<DT>;
+  constexpr int NB = 1024;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int total_bits = E::kKeyBits + idx_bits;
+  const uint32_t kmin = static_cast<uint32_t>(vlo >> idx_bits), kmax = static_cast<uint32_t>(vhi >> idx_bits);
+  const int sh = max(0, (32 - __clz(kmax - kmin)) - 10);   // ((kmax - kmin) >> sh) < NB
+#pragma unroll 1
+  for (int i = tid; i < NB; i += THREADS) hist[i] = 0;
+  if (tid == 0) ctl.tie_n = 0;
+  __syncthreads();
+#pragma unroll 1
+  for (int i = tid; i < n; i += THREADS)   // the clamp only guards the array: keys lie in [kmin, kmax]
+    atomicAdd(&hist[min((E::key(cb[i]) - kmin) >> sh, static_cast<uint32_t>(NB - 1))], 1);
+  __syncthreads();
+  // every warp: lane l sums bins NB-32-32l .. NB-1-32l (int4s 8(31-l) ..), scans,
+  // and the lane holding the k-th largest walks its bins from the top
+  const int top = NB - 1 - lane * 32;
+  const int sum = chunk_sum4<8>(reinterpret_cast<const int4*>(hist), 0, 31 - lane);
+  const int incl = warp_incl_scan(sum, lane);
+  const bool mine = incl - sum < k && k <= incl;
+  int bin = 0, above = 0;
+  if (mine) {
+    int acc = incl - sum;
+#pragma unroll 1
+    for (int j = 0; j < 32; ++j) {
+      const int c = hist[top - j];
+      if (acc + c >= k) {
+        bin = top - j;
+        above = acc;
+        break;
+      }
+      acc += c;
+    }
+  }
+  const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+  bin = __shfl_sync(0xffffffffu, bin, src);
+  above = __shfl_sync(0xffffffffu, above, src);
+  const int bucket = hist[bin];
+  const int need = k - above;
+  const uint32_t klo = kmin + (static_cast<uint32_t>(bin) << sh);
+  if (sh == 0) {   // the boundary bin is one key
+    if (bucket == need) return SelResult{klo, E::kKeyBits, k};   // every candidate of that key is kept
+    if (bucket <= kTieMax)
+      return SelResult{rank_members<DT, THREADS>(cb, ci, n, klo, klo, bucket, need, idx_bits, ctl), total_bits, k};
+    // many candidates of that key: their index digits
+    const uint32_t idx_mask = mask_bits(idx_bits);
+    const uint64_t base = static_cast<uint64_t>(klo) << idx_bits;
+    const SelResult r =
+        radix_select<DT, THREADS, false>(cb, ci, n, need, 0, idx_bits, base, base | idx_mask, ctl, cluster);
+    return SelResult{r.prefix, r.depth, k};
+  }
+  if (bucket <= kTieMax) {
+    const uint32_t khi = klo + ((1u << sh) - 1u);
+    return SelResult{rank_members<DT, THREADS>(cb, ci, n, klo, khi, bucket, need, idx_bits, ctl), total_bits, k};
+  }
+  return radix_select<DT, THREADS, false>(cb, ci, n, k, 0, idx_bits, vlo, vhi, ctl, cluster);
+}
+
 // Keep the candidates whose top `depth` bits are >= prefix (`kept` of them, or
 // counted here when kept < 0), moving those found past position kept into the
 // holes below it.  Order is not preserved; positions come from per-warp counts

@@ -449,9 +449,19 @@ __device__ __noinline__ void finish_sorted(const KParams& p, int64_t row, int g,
 // selection result for finish_sorted (depth 0: all of them).
 template <int DT, int THREADS>
 __device__ __forceinline__ SelResult select_best(const KParams& p, typename Elem<DT>::bits_t* cb, uint32_t* ci, int n,
-                                                 uint64_t vlo, uint64_t vhi, Ctl& ctl, cg::cluster_group& cluster) {
+                                                 uint64_t vlo, uint64_t vhi, Ctl& ctl, uint32_t* holes,
+                                                 cg::cluster_group& cluster) {
   if (n <= p.k) return SelResult{0ull, 0, n};
-  return radix_select<DT, THREADS, false>(cb, ci, n, p.k, 0, p.idx_bits, vlo, vhi, ctl, cluster);
+  // When the candidates' keys differ only in their low 8 bits, the radix
+  // select's first 256-bin pass already resolves the key; otherwise its first
+  // digit would be cut at key bits (for floats: the exponent) and one pass of
+  // range-adaptive bins does better.  The hole list (k + B2 >= 1025 slots) is
+  // idle here and holds those bins.
+  const uint32_t kx = static_cast<uint32_t>(vlo >> p.idx_bits) ^ static_cast<uint32_t>(vhi >> p.idx_bits);
+  if (32 - __clz(kx) <= kDigitBits)
+    return radix_select<DT, THREADS, false>(cb, ci, n, p.k, 0, p.idx_bits, vlo, vhi, ctl, cluster);
+  return select_by_key_hist<DT, THREADS>(cb, ci, n, p.k, p.idx_bits, vlo, vhi, ctl, reinterpret_cast<int*>(holes),
+                                         cluster);
 }
 
 template <int DT, int THREADS>
@@ -477,7 +487,7 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
       emit_nan<DT, THREADS>(p, row, g, to_workspace);
       return;
     }
-    const SelResult sel = select_best<DT, THREADS>(p, cb, ci, cnt, vlo, vhi, ctl, cluster);
+    const SelResult sel = select_best<DT, THREADS>(p, cb, ci, cnt, vlo, vhi, ctl, holes, cluster);
     trace_final(5);
     finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, cnt, sel, sort_mode, ctl, holes, ring, ring_bytes,
                                span_lo, span_len, 0, sel.kept, true);
@@ -556,7 +566,7 @@ __device__ __noinline__ void finalize(const KParams& p, int64_t row, int g, type
     }
     __syncthreads();   // the gathered list is complete
     trace_final(3);
-    const SelResult sel = select_best<DT, THREADS>(p, cb, ci, off, lo, hi, ctl, cluster);
+    const SelResult sel = select_best<DT, THREADS>(p, cb, ci, off, lo, hi, ctl, holes, cluster);
     trace_final(5);
     finish_sorted<DT, THREADS>(p, row, g, to_workspace, cb, ci, off, sel, sort_mode, ctl, holes, ring, ring_bytes,
                                span_lo, span_len, 0, sel.kept, true);
@@ -925,8 +935,11 @@ __device__ __noinline__ void issue_block(int j, int jg, uint32_t pa, uint32_t pc
                                          uint32_t* blk_off) {
   using E = Elem<DT>;
   constexpr int B = block_elems_for(E::kBytes);
-  const uint32_t m = static_cast<uint32_t>((static_cast<uint64_t>(pa) * static_cast<uint32_t>(j) + pc) %
-                                           static_cast<uint32_t>(nb));
+  // pa, j mod nb and pc are below nb: 32-bit products while nb < 2^16
+  const uint32_t jj = static_cast<uint32_t>(j) % static_cast<uint32_t>(nb);
+  const uint32_t m = nb < 65536 ? (pa * jj + pc) % static_cast<uint32_t>(nb)
+                                : static_cast<uint32_t>((static_cast<uint64_t>(pa) * jj + pc) %
+                                                        static_cast<uint32_t>(nb));
   const int64_t e0 = lo + static_cast<int64_t>(m) * B;
   const int64_t ce = min(static_cast<int64_t>(B), hi - e0);
   const uint32_t bytes = static_cast<uint32_t>((ce * E::kBytes + 15) & ~static_cast<int64_t>(15));
@@ -1065,7 +1078,9 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
     // ---- this CTA's slice: [lo, hi), a multiple of 16 elements wide ----
     const int S = p.groups * C;
     const int sid = g * C + crank;
-    const int64_t slice = ((n + S - 1) / S + 15) / 16 * 16;
+    // 32-bit arithmetic: n <= row_stride <= INT32_MAX (64-bit division is a software routine)
+    const int64_t slice = static_cast<int64_t>(((static_cast<uint32_t>(n) + static_cast<uint32_t>(S) - 1u) /
+                                                    static_cast<uint32_t>(S) + 15u) / 16u * 16u);
     const int64_t lo = min(n, static_cast<int64_t>(sid) * slice);
     const int64_t hi = min(n, lo + slice);
     const int nb = static_cast<int>((hi - lo + B - 1) / B);
@@ -1075,7 +1090,8 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
     uint32_t pa = 1, pc = 0;
     if (nb > 1) {
       const uint32_t unb = static_cast<uint32_t>(nb);
-      pa = static_cast<uint32_t>((static_cast<uint64_t>(unb) * 618u + 500u) / 1000u) | 1u;
+      pa = (unb < 6000000u ? (unb * 618u + 500u) / 1000u
+                           : static_cast<uint32_t>((static_cast<uint64_t>(unb) * 618u + 500u) / 1000u)) | 1u;
 #pragma unroll 1
       for (;;) {
         uint32_t a = pa, b = unb;
@@ -1086,7 +1102,7 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
       pa %= unb;
       const uint64_t h = (static_cast<uint64_t>(row) + 1) * 0x9E3779B97F4A7C15ull ^
                          (static_cast<uint64_t>(sid) + 1) * 0xBF58476D1CE4E5B9ull;
-      pc = static_cast<uint32_t>((h >> 29) % unb);
+      pc = static_cast<uint32_t>(h >> 29) % unb;   // the low 32 bits of h >> 29
     }
     int jb = 0;   // blocks issued in earlier passes over the slice
     auto issue = [&](int j) {

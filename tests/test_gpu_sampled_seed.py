@@ -45,7 +45,7 @@ def round0_blocks(row: int, nb: int, q: int) -> list:
         pa += 2
     pa %= nb
     h = (((row + 1) * 0x9E3779B97F4A7C15) & M64) ^ ((1 * 0xBF58476D1CE4E5B9) & M64)
-    pc = (h >> 29) % nb
+    pc = ((h >> 29) & 0xFFFFFFFF) % nb
     return [(pa * j + pc) % nb for j in range(min(q, nb))]
 
 
