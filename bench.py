@@ -35,7 +35,7 @@ METRIC = "effective HBM GB/s and rows/s for TopK (bf16 k=512; fp32 V=129,280) on
 KERNEL_SOURCES = ["row_wise_topk_b200/csrc/dsel_device.cuh", "row_wise_topk_b200/csrc/dsel_kernels.cuh",
                   "row_wise_topk_b200/csrc/dsel_api.cu", "row_wise_topk_b200/csrc/dsel_plan.cpp",
                   "row_wise_topk_b200/csrc/dsel_shard.cu",
-                  "row_wise_topk_b200/csrc/dsel_plan.h"]
+                  "row_wise_topk_b200/csrc/dsel_plan.h", "row_wise_topk_b200/csrc/dsel_resident.cuh"]
 FALLBACK_HBM_GBS = 6650.0
 SAMPLE_T, SAMPLE_P = 1.0, 0.9      # temperature and top-p of the sample_B_k workloads
 
@@ -449,14 +449,15 @@ def run_ours(args, w, world, rank, local, pg):
         "data": "synthetic", "config": workload_config(args, w, world),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
-                     "kernel": "topk_stream_kernel" + ("+topk_merge_kernel" if launches_per_step > 1 else ""),
+                     "kernel": ("topk_resident_kernel" if plan.get("kernel") == T.DSEL_KERNEL_RESIDENT
+                                else "topk_stream_kernel" + ("+topk_merge_kernel" if launches_per_step > 1 else "")),
                      "launch_ms": round(kern_ms, 5)},
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
-        "plan": {k_: plan[k_] for k_ in ("cluster", "groups", "stages", "smem_bytes")},
+        "plan": {k_: plan[k_] for k_ in ("kernel", "threads", "cluster", "groups", "stages", "smem_bytes")},
         "input_copies": n_copies,
     }
     print(json.dumps(line), flush=True)

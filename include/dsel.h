@@ -130,7 +130,14 @@ typedef struct {
   int32_t idx_bits;      /* bits of the in-row index used to break ties */
   int32_t smem_bytes;    /* dynamic shared memory per CTA */
   int64_t workspace_bytes; /* split-row workspace (0 unless groups > 1) */
+  int32_t kernel;        /* DSEL_KERNEL_STREAM, or DSEL_KERNEL_RESIDENT: at least as many rows as
+                            SMs and rows of at most 32 KB, one 256-thread CTA per row holding the
+                            whole row in shared memory (block = the 4 KB bulk-copy chunk,
+                            round = row_stride, stages = chunks per row, b2 = 0) */
 } dsel_plan_t;
+
+#define DSEL_KERNEL_STREAM 0
+#define DSEL_KERNEL_RESIDENT 1
 
 /*
  * dsel_topk -- batched row-wise TopK (the operation described at the top).

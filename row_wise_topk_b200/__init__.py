@@ -25,6 +25,7 @@ DSEL_I32, DSEL_I64 = 0, 1
 DSEL_NAN_TRAP, DSEL_NAN_FLAG = 0, 1
 DSEL_ORDER_NONE, DSEL_ORDER_INDEX, DSEL_ORDER_VALUE = 0, 1, 2
 DSEL_IDX_PAD, DSEL_IDX_NAN, DSEL_IDX_BAD_END = -1, -2, -3
+DSEL_KERNEL_STREAM, DSEL_KERNEL_RESIDENT = 0, 1
 DSEL_OK = 0
 DSEL_ERR_SCRATCH_LIMIT = -16
 DSEL_NOALLOC_SCRATCH_BYTES = 512 * 1024
@@ -43,6 +44,7 @@ class DselPlan(ctypes.Structure):
         ("idx_bits", ctypes.c_int32),
         ("smem_bytes", ctypes.c_int32),
         ("workspace_bytes", ctypes.c_int64),
+        ("kernel", ctypes.c_int32),
     ]
 
     def as_dict(self):

@@ -7,6 +7,7 @@
 #include "../../include/dsel.h"
 #include "dsel_kernels.cuh"
 #include "dsel_plan.h"
+#include "dsel_resident.cuh"
 
 namespace dsel {
 namespace {
@@ -19,6 +20,7 @@ struct DevInfo {
   int smem_optin = 0;
   int major = 0;
   bool attrs_set[2][3] = {{false, false, false}, {false, false, false}};   // [dtype][shape]
+  bool res_attrs_set[2] = {false, false};                                  // [dtype], resident kernel
 };
 
 std::mutex g_mu;
@@ -138,9 +140,32 @@ int run_shape(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStre
   return DSEL_OK;
 }
 
+template <int DT>
+int run_resident(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
+  auto rk = topk_resident_kernel<DT>;
+  if (!di->res_attrs_set[DT]) {
+    if (cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) != cudaSuccess)
+      return DSEL_ERR_CUDA;
+    di->res_attrs_set[DT] = true;
+  }
+  const ResLayout rl = resident_layout(base.row_stride, base.k, elem_bytes(DT));
+  KParams kp = base;
+  kp.off_bars = rl.bars;
+  kp.off_hist = rl.hist;
+  kp.off_tab = rl.tab;
+  kp.off_cb = rl.cb;
+  kp.off_ci = rl.ci;
+  kp.off_ctl = rl.ctl;
+  if (rows > 0x7FFFFFFF) return DSEL_ERR_ROWS;
+  if (launch_cluster(rk, unsigned(rows), kResThreads, 1, rl.total, st, kp) != cudaSuccess) return DSEL_ERR_CUDA;
+  (void)pl;
+  return DSEL_OK;
+}
+
 // The planner returns split-row plans (groups > 1) only with the 512-thread shape.
 template <int DT>
 int run(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
+  if (pl.kernel == DSEL_KERNEL_RESIDENT) return run_resident<DT>(base, pl, rows, st, di);
   if (pl.threads == kThreadsShort) return run_shape<DT, kThreadsShort>(base, pl, rows, st, di);
   if (pl.threads == kThreadsMid) return run_shape<DT, kThreadsMid>(base, pl, rows, st, di);
   if (pl.threads == kThreads) return run_shape<DT, kThreads>(base, pl, rows, st, di);

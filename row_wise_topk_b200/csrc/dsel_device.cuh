@@ -125,6 +125,19 @@ __device__ __forceinline__ float f32_max_nan(float a, float b) {
   return d;
 }
 
+// NaN-propagating minima.
+__device__ __forceinline__ uint32_t bf16x2_min_nan(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ float f32_min_nan(float a, float b) {
+  float d;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
 // Candidate mask of a vector: bit e set when element e is >= T as a float, or NaN
 // (unordered compare).  A superset of the elements that can rank above T.
 __device__ __forceinline__ uint32_t bf16x2_geu_mask(uint32_t a, uint32_t t) {
@@ -270,6 +283,10 @@ struct __align__(16) Ctl {
   float smp_w[kWarpsMax];       // sampling: per-warp weight sums
   int smp_c, smp_pos;           // sampling: last kept candidate, drawn candidate
   float smp_ec;                 // sampling: weight sum of the kept candidates
+  unsigned r_kmax, r_kmin;      // row-resident kernel: the row's largest and smallest keys,
+  unsigned r_gmin;              //   the smallest vector maximum,
+  unsigned r_tkey;              //   the k-th largest key and
+  int r_ngt;                    //   how many keys exceed it
 #ifdef DSEL_STATS
   unsigned long long st_compact_cycles;
   int st_compactions;

@@ -29,6 +29,7 @@ struct KParams {
   int32_t gather;           // final phase gathers the cluster's partial results on rank 0
   int32_t capacity;         // candidate-buffer slots
   uint32_t off_bars, off_blk, off_cb, off_ci, off_holes, off_ctl;
+  uint32_t off_hist, off_tab;   // row-resident kernel: histograms, scan table
   // sampling step after TopK (fp32 only; token_out == nullptr: no draw)
   const float* u;           // [rows] the caller's uniforms in [0, 1)
   int64_t* token_out;       // [rows] drawn index, or a negative row code

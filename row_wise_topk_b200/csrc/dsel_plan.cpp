@@ -6,6 +6,8 @@
 // round (4096 bf16 / 1024 f32 elements, see block_elems_for), and everything
 // else here is this library's choice for a 148-SM B200:
 //   * one CTA per row while there are at least as many rows as SMs:
+//       - rows of at most 32 KB: the row-resident kernel (dsel_resident.cuh),
+//         which holds the whole row in shared memory;
 //       - rows of at most two 128-thread rounds: a 128-thread CTA, several per
 //         SM, each with at most one round of blocks in flight;
 //       - longer rows with k <= 1024: a 256-thread CTA when two fit an SM (two
@@ -68,6 +70,27 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
   const int eb = elem_bytes(dtype);
   dsel_plan_t p{};
   const bool one_per_row = rows >= num_sms;
+
+  // Rows that fit in shared memory: the row-resident kernel.
+  if (one_per_row && row_stride * eb <= kResRowBytes) {
+    const ResLayout rl = resident_layout(row_stride, k, eb);
+    if (int64_t(rl.total) <= smem_optin) {
+      p.kernel = DSEL_KERNEL_RESIDENT;
+      p.threads = kResThreads;
+      p.cluster = 1;
+      p.groups = 1;
+      p.block = kResThreads * kVecBytes / eb;
+      p.b2 = 0;
+      p.round = int(row_stride);
+      p.capacity = next_pow2(k);
+      p.stages = int(ceil_div(row_stride * eb, int64_t(kResThreads) * kVecBytes));
+      p.idx_bits = ceil_log2_u64(uint64_t(row_stride));
+      p.smem_bytes = int(rl.total);
+      p.workspace_bytes = 0;
+      *out = p;
+      return DSEL_OK;
+    }
+  }
   const bool short_rows = one_per_row && row_stride <= 2 * int64_t(round_elems(dtype, kThreadsShort));
 
   // 256-thread shape: two CTAs per SM (half of the SM's shared memory each, less
@@ -86,6 +109,7 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
       }
     }
   }
+  p.kernel = DSEL_KERNEL_STREAM;
   shape_plan(dtype, k, short_rows ? kThreadsShort : (mid_stages > 0 ? kThreadsMid : kThreads), &p);
   p.idx_bits = ceil_log2_u64(uint64_t(row_stride));
 

@@ -16,6 +16,10 @@ constexpr int kThreads = 512;
 constexpr int kThreadsMid = 256;
 constexpr int kThreadsShort = 128;
 constexpr int kVecBytes = 16;                 // one 128-bit shared-memory load per vector
+// Row-resident kernel: one 256-thread CTA per row holds the whole row (at most
+// 32 KB: 16,384 bf16 or 8,192 f32 elements) in shared memory.
+constexpr int kResThreads = 256;
+constexpr int kResRowBytes = 32 * 1024;
 // Vectors each thread screens per round (a warp owns whole blocks): 16 for bf16
 // (a 64K-element round, the whole slice of a 131,072-position row split in two),
 // 8 for f32 (16K elements, so that two rounds fit the ring for double buffering).
@@ -94,6 +98,35 @@ inline SmemLayout stream_layout(int64_t stages, int64_t block, int64_t capacity,
   off += up(capacity * 4, 16);
   l.holes = uint32_t(off);
   off += up(holes * 4, 16);
+  l.ctl = uint32_t(off);
+  off += kSharedFixedBytes;
+  l.total = uint32_t(off);
+  return l;
+}
+
+// Row-resident kernel: the row, one mbarrier per 4 KB chunk, three 1024-bin
+// histograms, the scan table ([8 rounds][8 warps] totals, then [8 warps][8
+// rounds] offsets), candidate arrays of next_pow2(k) entries (value order and the
+// sampling step sort there) and the control block.
+struct ResLayout {
+  uint32_t bars, hist, tab, cb, ci, ctl, total;
+};
+
+inline ResLayout resident_layout(int64_t row_stride, int32_t k, int eb) {
+  auto up = [](int64_t v, int64_t a) { return (v + a - 1) / a * a; };
+  ResLayout l{};
+  int64_t off = up(row_stride * eb, 128);
+  l.bars = uint32_t(off);
+  off += 8 * 8;
+  l.hist = uint32_t(off);
+  off += 3 * 1024 * 4;
+  l.tab = uint32_t(off);
+  off += 2 * 8 * 8 * 4;
+  const int64_t kp2 = next_pow2(k);
+  l.cb = uint32_t(off);
+  off += up(kp2 * eb, 16);
+  l.ci = uint32_t(off);
+  off += up(kp2 * 4, 16);
   l.ctl = uint32_t(off);
   off += kSharedFixedBytes;
   l.total = uint32_t(off);

@@ -1,0 +1,419 @@
+// Row-resident TopK: rows that fit in shared memory, one CTA of 256 threads per row.
+//
+// The streaming kernel (topk_stream_kernel) follows the method of "DeepSeek
+// releases DeepSelect, a TopK kernel for sparse attention and sampling" (method
+// paragraph): a threshold filter over blocks read once, a candidate buffer, and
+// radix-select compactions.  Its fixed cost per row (seed histogram, exact test,
+// final select, index ranking, each behind several barriers) dominates when a
+// row is only a few thousand elements, as in a batch of variable-length indexer
+// rows.  A row of at most 32 KB fits in shared memory next to everything else,
+// so this kernel reads it once into shared memory and selects there, exactly:
+//
+//   1. bulk copies of the row, one 4 KB chunk (one 16-byte vector per thread)
+//      per mbarrier, so that step 2 starts on the first chunk;
+//   2. each thread keeps the largest key of each of its vectors in a register,
+//      and the CTA finds the row's largest and smallest keys and any NaN;
+//   3. seed: when the row has at least k vectors, the k-th largest vector
+//      maximum T0 is a lower bound of the k-th largest element (k vectors each
+//      hold an element >= T0); a histogram of the vector maxima gives it;
+//   4. the exact k-th largest key: histograms of the keys >= T0 in 1024 bins
+//      spread over the remaining key range, one level per pass, until the
+//      boundary bin is a single key or holds at most 128 elements, which are
+//      then ranked directly;
+//   5. output in index order without sorting: each vector's counts of keys
+//      above the k-th key and equal to it, scanned over the row in index order,
+//      give every selected element its output slot (equal keys are taken in
+//      index order, the tie rule value-descending then index-ascending).
+//
+// Value order and the sampling step put the k selected entries in shared memory
+// instead and finish as the streaming kernel does (bitonic sort, draw).
+// Histogram levels rotate over three buffers; the buffer of level L + 2 is
+// cleared after the barrier of level L, when its last readers are done.
+#pragma once
+
+#include "dsel_kernels.cuh"
+
+namespace dsel {
+
+constexpr int kResVpt = 8;                    // vectors per thread: rows up to 256 x 8 x 16 B = 32 KB
+constexpr int kResBins = 1024;
+static_assert(kResThreads * kResVpt * kVecBytes == kResRowBytes, "resident row capacity");
+
+// Largest and smallest key of a 16-byte vector; true when it holds a NaN.
+template <int DT>
+__device__ __forceinline__ bool vec_minmax_key(const uint4 x, uint32_t& kmx, uint32_t& kmn) {
+  using E = Elem<DT>;
+  if (DT == DSEL_BF16) {
+    const uint32_t hi = bf16x2_max_nan(bf16x2_max_nan(x.x, x.y), bf16x2_max_nan(x.z, x.w));
+    const uint32_t lo = bf16x2_min_nan(bf16x2_min_nan(x.x, x.y), bf16x2_min_nan(x.z, x.w));
+    if (E::is_nan(hi & 0xFFFFu) || E::is_nan(hi >> 16)) return true;
+    kmx = max(E::key(hi & 0xFFFFu), E::key(hi >> 16));
+    kmn = min(E::key(lo & 0xFFFFu), E::key(lo >> 16));
+    return false;
+  } else {
+    const float a = __uint_as_float(x.x), b = __uint_as_float(x.y), c = __uint_as_float(x.z),
+                d = __uint_as_float(x.w);
+    const float hi = f32_max_nan(f32_max_nan(a, b), f32_max_nan(c, d));
+    const float lo = f32_min_nan(f32_min_nan(a, b), f32_min_nan(c, d));
+    if (hi != hi) return true;
+    kmx = E::key(__float_as_uint(hi));
+    kmn = E::key(__float_as_uint(lo));
+    return false;
+  }
+}
+
+// Shift that spreads the key range [lo, lo + range] over at most 1024 bins.
+__device__ __forceinline__ int res_shift(uint32_t range) { return max(0, (32 - __clz(range)) - 10); }
+
+// Lowest key of bin b (bins of 2^s keys counted down from hi), not below lo.
+__device__ __forceinline__ uint32_t res_bin_lo(uint32_t hi, uint32_t lo, int b, int s) {
+  const uint64_t span = (static_cast<uint64_t>(b) + 1u) << s;   // keys from hi down to the bin's end
+  return span > static_cast<uint64_t>(hi - lo) ? lo : hi - static_cast<uint32_t>(span) + 1u;
+}
+
+struct BinHit {
+  int bin;      // the bin holding the t-th largest entry (bin 0 = the top)
+  int before;   // entries in the bins above it
+  int cnt;      // entries in it
+};
+
+// Bin of the t-th largest entry in a 1024-bin histogram (bin 0 = largest keys),
+// found by one warp with no barrier; every warp may run it on the same
+// histogram.  The histogram must hold at least t entries.
+__device__ __forceinline__ BinHit res_find_bin(const int* h, int t, int lane) {
+  const int sum = chunk_sum4<8>(reinterpret_cast<const int4*>(h), 0, lane);   // bins 32*lane .. +31
+  const int incl = warp_incl_scan(sum, lane);
+  const int L = max(0, __ffs(__ballot_sync(0xffffffffu, incl >= t)) - 1);
+  const int base = __shfl_sync(0xffffffffu, incl - sum, L);
+  const int c = h[32 * L + lane];
+  const int incl2 = warp_incl_scan(c, lane) + base;
+  const int j = max(0, __ffs(__ballot_sync(0xffffffffu, incl2 >= t)) - 1);
+  BinHit r;
+  r.bin = 32 * L + j;
+  r.cnt = __shfl_sync(0xffffffffu, c, j);
+  r.before = __shfl_sync(0xffffffffu, incl2, j) - r.cnt;
+  return r;
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __grid_constant__ KParams p) {
+  using E = Elem<DT>;
+  using bits_t = typename E::bits_t;
+  constexpr int T = kResThreads;
+  constexpr int NW = T / 32;
+  constexpr int PV = E::kPerVec;
+  constexpr int VPT = kResVpt;
+  constexpr int CH = T * kVecBytes;   // bytes per chunk: one vector per thread
+
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const unsigned char* rowb = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bars);
+  int* hist = reinterpret_cast<int*>(smem + p.off_hist);            // 3 x kResBins
+  uint32_t* tab = reinterpret_cast<uint32_t*>(smem + p.off_tab);    // [VPT][NW] packed warp totals
+  uint32_t* offw = tab + VPT * NW;                                   // [NW][VPT] packed offsets
+  bits_t* cb = reinterpret_cast<bits_t*>(smem + p.off_cb);
+  uint32_t* ci = reinterpret_cast<uint32_t*>(smem + p.off_ci);
+  Ctl& ctl = *reinterpret_cast<Ctl*>(smem + p.off_ctl);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t row = blockIdx.x;
+  const int k = p.k;
+
+#pragma unroll 1
+  for (int i = tid; i < 3 * kResBins / 4; i += T) reinterpret_cast<int4*>(hist)[i] = make_int4(0, 0, 0, 0);
+  if (tid == 0) {
+    ctl.nan_found = 0;
+    ctl.abort = 0;
+    ctl.tie_n = 0;
+    ctl.r_kmax = 0u;
+    ctl.r_kmin = 0xFFFFFFFFu;
+    ctl.r_gmin = 0xFFFFFFFFu;
+  }
+  if (tid < VPT) {
+    mbar_init(smem_u32(&bars[tid]), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // the set-up above touched shared memory only: it may overlap the previous launch
+  grid_dependency_wait();
+  bool bad_end;
+  const int64_t n64 = row_length(p, row, &bad_end);
+  if (bad_end || n64 <= k) {
+    if (bad_end) write_sentinel_row<DT, T>(p, row, DSEL_IDX_BAD_END);
+    else finish_short_row<DT, T>(p, row, n64, cb, ci, ctl);
+    return;
+  }
+  const int n = static_cast<int>(n64);   // <= kResRowBytes / 2
+  const int nvec = (n + PV - 1) / PV;
+  const uint32_t row_bytes = static_cast<uint32_t>((n + 15) / 16 * 16) * E::kBytes;   // multiple of 16 B
+  const int nch = static_cast<int>((row_bytes + CH - 1) / CH);                        // <= VPT
+
+  // ---- 1. bulk copies: chunk c (vectors c*T .. c*T + T - 1) by lane c of warp 0 ----
+  if (warp == 0 && lane < nch) {
+    const uint32_t b = min(static_cast<uint32_t>(CH), row_bytes - static_cast<uint32_t>(lane) * CH);
+    const uint32_t bar = smem_u32(&bars[lane]);
+    mbar_expect_tx(bar, b);
+    bulk_g2s(smem_u32(smem + lane * CH),
+             static_cast<const char*>(p.x) + (row * p.row_stride) * E::kBytes + static_cast<int64_t>(lane) * CH, b,
+             bar);
+  }
+
+  // ---- 2. vector maxima, row extremes, NaN ----
+  uint32_t gk[VPT];   // largest key of vector i * T + tid; 0 = no vector (keys of numbers are >= 1)
+  uint32_t kmax = 0u, kmin = 0xFFFFFFFFu, gmin = 0xFFFFFFFFu;
+  bool nan = false, late = false;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    gk[i] = 0u;
+    if (i < nch) {
+      if (!mbar_wait(smem_u32(&bars[i]), 0u)) late = true;
+      const int v = i * T + tid;
+      if (v < nvec) {
+        const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
+        const int valid = min(PV, n - v * PV);
+        uint32_t mx = 0u, mn = 0xFFFFFFFFu;
+        bool vn = false;
+        if (valid == PV) {
+          vn = vec_minmax_key<DT>(x, mx, mn);
+        } else {
+#pragma unroll 1
+          for (int e = 0; e < valid; ++e) {
+            const uint32_t b = vec_elem_dyn<DT>(x, e);
+            if (E::is_nan(b)) vn = true;
+            const uint32_t kk = E::key(b);
+            mx = max(mx, kk);
+            mn = min(mn, kk);
+          }
+        }
+        if (vn) {
+          nan = true;
+        } else {
+          gk[i] = mx;
+          kmax = max(kmax, mx);
+          kmin = min(kmin, mn);
+          gmin = min(gmin, mx);
+        }
+      }
+    }
+  }
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  gmin = __reduce_min_sync(0xffffffffu, gmin);
+  const bool wnan = __any_sync(0xffffffffu, nan), wlate = __any_sync(0xffffffffu, late);
+  if (lane == 0) {
+    atomicMax(&ctl.r_kmax, kmax);
+    atomicMin(&ctl.r_kmin, kmin);
+    atomicMin(&ctl.r_gmin, gmin);
+    if (wnan) ctl.nan_found = 1;
+    if (wlate) ctl.abort = 1;
+  }
+  __syncthreads();
+  if (ctl.abort) {   // a copy may still be in flight: wait for it (bounded) before the CTA exits
+    if (tid < nch) mbar_wait(smem_u32(&bars[tid]), 0u);
+    return;
+  }
+  grid_launch_dependents();   // the row is in shared memory: the next launch may start its prologue
+  if (ctl.nan_found) {
+    if (!p.nan_flag) nan_trap();   // the pages' default NaN policy
+    write_sentinel_row<DT, T>(p, row, DSEL_IDX_NAN);
+    return;
+  }
+  kmax = ctl.r_kmax;
+  kmin = ctl.r_kmin;
+  gmin = ctl.r_gmin;
+
+  // ---- 3. seed: the k-th largest vector maximum (or a bin edge below it) ----
+  uint32_t lo = kmin, hi = kmax;   // the k-th largest key lies in [lo, hi]
+  int above = 0;                   // elements with key > hi
+  if (nvec >= k) {
+    const int s = res_shift(kmax - gmin);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i)
+      if (gk[i] != 0u) atomicAdd(&hist[(kmax - gk[i]) >> s], 1);
+    __syncthreads();
+    const BinHit bh = res_find_bin(hist, k, lane);
+    lo = max(lo, res_bin_lo(kmax, gmin, bh.bin, s));
+  }
+
+  // ---- 4. the exact k-th largest key: histogram levels over [lo, hi] ----
+  uint32_t tkey;   // the k-th largest key
+  int n_gt;        // elements with key > tkey (< k)
+#pragma unroll 1
+  for (int level = 1;; ++level) {
+    int* h = hist + (level % 3) * kResBins;
+    const int s = res_shift(hi - lo);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      if (gk[i] >= lo) {   // only vectors whose maximum reaches lo hold such keys
+        const int v = i * T + tid;
+        const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
+        const int valid = min(PV, n - v * PV);
+#pragma unroll
+        for (int e = 0; e < PV; ++e) {
+          const uint32_t kk = E::key(vec_elem<DT>(x, e));
+          if (e < valid && kk >= lo && kk <= hi) atomicAdd(&h[(hi - kk) >> s], 1);
+        }
+      }
+    }
+    __syncthreads();
+    const BinHit bh = res_find_bin(h, k - above, lane);
+    const uint32_t bhi = hi - (static_cast<uint32_t>(bh.bin) << s);
+    const uint32_t blo = res_bin_lo(hi, lo, bh.bin, s);
+    above += bh.before;
+    if (s == 0) {   // the boundary bin is one key
+      tkey = bhi;
+      n_gt = above;
+      break;
+    }
+    if (bh.cnt <= kTieMax) {
+      // rank the boundary bin's members by key; the free buffer of level + 1 holds them
+      uint32_t* lst = reinterpret_cast<uint32_t*>(hist + ((level + 1) % 3) * kResBins);
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        if (gk[i] >= blo) {
+          const int v = i * T + tid;
+          const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
+          const int valid = min(PV, n - v * PV);
+#pragma unroll
+          for (int e = 0; e < PV; ++e) {
+            const uint32_t kk = E::key(vec_elem<DT>(x, e));
+            if (e < valid && kk >= blo && kk <= bhi) {
+              const int pos = atomicAdd(&ctl.tie_n, 1);
+              if (pos < kResBins) lst[pos] = kk;
+            }
+          }
+        }
+      }
+      __syncthreads();
+      const int need = k - above;
+      if (tid < bh.cnt) {
+        const uint32_t kj = lst[tid];
+        int gt = 0, eq = 0;
+#pragma unroll 4
+        for (int i = 0; i < bh.cnt; ++i) {
+          const uint32_t ki = lst[i];
+          gt += ki > kj ? 1 : 0;
+          eq += ki == kj ? 1 : 0;
+        }
+        if (gt < need && need <= gt + eq) {   // the need-th largest member
+          ctl.r_tkey = kj;
+          ctl.r_ngt = above + gt;
+        }
+      }
+      __syncthreads();
+      tkey = ctl.r_tkey;
+      n_gt = ctl.r_ngt;
+      break;
+    }
+    // another level over the boundary bin; clear the buffer of level + 2
+    int4* z = reinterpret_cast<int4*>(hist + ((level + 2) % 3) * kResBins);
+#pragma unroll 1
+    for (int i = tid; i < kResBins / 4; i += T) z[i] = make_int4(0, 0, 0, 0);
+    lo = blo;
+    hi = bhi;
+  }
+
+  // ---- 5. output slots in index order ----
+  // per vector: (keys > tkey) | (keys == tkey) << 16, scanned over the row in
+  // vector order (round i, then thread); both fields stay below 2^16
+  const int need_eq = k - n_gt;
+  uint32_t excl[VPT];
+  uint32_t has = 0u;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    uint32_t c = 0u;
+    if (gk[i] >= tkey) {
+      const int v = i * T + tid;
+      const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
+      const int valid = min(PV, n - v * PV);
+#pragma unroll
+      for (int e = 0; e < PV; ++e) {
+        const uint32_t kk = E::key(vec_elem<DT>(x, e));
+        if (e < valid) c += kk > tkey ? 1u : (kk == tkey ? 0x10000u : 0u);
+      }
+    }
+    has |= c != 0u ? 1u << i : 0u;
+    excl[i] = 0u;
+    if (i < nch && __any_sync(0xffffffffu, c != 0u)) {
+      uint32_t incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      excl[i] = incl - c;
+      if (lane == 31) tab[i * NW + warp] = incl;
+    } else if (i < nch && lane == 0) {
+      tab[i * NW + warp] = 0u;
+    }
+  }
+  __syncthreads();
+  {   // every warp: exclusive prefix of the [round][warp] totals; keep this warp's column
+    static_assert(VPT * NW <= 128, "four table entries per lane");
+    const int ne = nch * NW;
+    uint32_t t4[4], run = 0u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = 4 * lane + j;
+      t4[j] = run;
+      run += e < ne ? tab[e] : 0u;
+    }
+    uint32_t incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t base = incl - run;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = 4 * lane + j;
+      if (e < ne && e % NW == warp) offw[warp * VPT + e / NW] = base + t4[j];
+    }
+    __syncwarp();
+  }
+  const bool to_smem = p.order == DSEL_ORDER_VALUE || p.token_out != nullptr;
+  const int64_t obase = row * static_cast<int64_t>(k);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    if (has & (1u << i)) {
+      const uint32_t pre = offw[warp * VPT + i] + excl[i];
+      int gtb = static_cast<int>(pre & 0xFFFFu), eqb = static_cast<int>(pre >> 16);
+      const int v = i * T + tid;
+      const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
+      const int valid = min(PV, n - v * PV);
+#pragma unroll
+      for (int e = 0; e < PV; ++e) {
+        const uint32_t b = vec_elem<DT>(x, e);
+        const uint32_t kk = E::key(b);
+        if (e < valid && kk >= tkey) {
+          const bool gt = kk > tkey;
+          if (gt || eqb < need_eq) {
+            const int pos = gtb + min(eqb, need_eq);
+            const uint32_t idx = static_cast<uint32_t>(v * PV + e);
+            if (pos < k) {
+              if (to_smem) {
+                cb[pos] = static_cast<bits_t>(b);
+                ci[pos] = idx;
+              } else {
+                if (p.index_i64) static_cast<int64_t*>(p.indices_out)[obase + pos] = static_cast<int64_t>(idx);
+                else static_cast<int32_t*>(p.indices_out)[obase + pos] = static_cast<int32_t>(idx);
+                if (p.return_value) static_cast<bits_t*>(p.values_out)[obase + pos] = static_cast<bits_t>(b);
+              }
+            }
+          }
+          if (gt) ++gtb;
+          else ++eqb;
+        }
+      }
+    }
+  }
+  if (!to_smem) return;
+  __syncthreads();
+  bitonic_sort<DT, T, true>(cb, ci, k);
+  write_rows_out<DT, T>(p, row, 0, k, cb, ci);
+  if (DT == DSEL_F32 && p.token_out != nullptr)
+    sample_draw<T>(p, row, reinterpret_cast<const uint32_t*>(cb), ci, k, ctl);
+}
+
+}  // namespace dsel

@@ -123,12 +123,26 @@ PEAK = dict(num_sms=148, smem_optin=232448, max_cluster=8)
     (T.DSEL_F32, 256, 129280, 4096), (T.DSEL_F32, 256, 129280, 1024), (T.DSEL_BF16, 300, 131072, 512),
     (T.DSEL_F32, 1, 1 << 28, 1000), (T.DSEL_F32, 16, 1 << 24, 4096),
     (T.DSEL_BF16, 3, 16, 4096), (T.DSEL_F32, 1, 16, 1),
+    (T.DSEL_BF16, 4096, 16400, 512), (T.DSEL_F32, 300, 8192, 4096), (T.DSEL_F32, 300, 8208, 64),
+    (T.DSEL_BF16, 148, 16, 4096), (T.DSEL_F32, 200, 4096, 1),
 ])
 def test_plan_invariants(dtype, rows, stride, k):
     st, p = T.dsel_plan(dtype, rows, stride, k, **PEAK)
     assert st == 0
     eb = 2 if dtype == T.DSEL_BF16 else 4
     assert p["smem_bytes"] <= PEAK["smem_optin"]
+    assert p["kernel"] in (T.DSEL_KERNEL_STREAM, T.DSEL_KERNEL_RESIDENT)
+    if rows >= PEAK["num_sms"] and stride * eb <= 32 * 1024:
+        # rows that fit in shared memory: one 256-thread CTA per row holds the whole row
+        assert p["kernel"] == T.DSEL_KERNEL_RESIDENT
+        assert (p["threads"], p["cluster"], p["groups"], p["b2"]) == (256, 1, 1, 0)
+        assert p["block"] * eb == 4096 and p["round"] == stride
+        assert p["stages"] == -(-(stride * eb) // 4096) <= 8
+        assert p["capacity"] == 1 << (k - 1).bit_length()          # value order sorts k entries in place
+        assert p["smem_bytes"] >= stride * eb + 3 * 4096 + p["capacity"] * (eb + 4)
+        assert (1 << p["idx_bits"]) >= stride and p["workspace_bytes"] == 0
+        return
+    assert p["kernel"] == T.DSEL_KERNEL_STREAM
     slack = 1024 if p["threads"] != 512 else (4096 if k <= 1024 else 2048)
     assert p["capacity"] >= k + p["b2"] + slack
     assert p["capacity"] >= 1 << (k - 1).bit_length()          # room for the bitonic padding
@@ -161,9 +175,14 @@ def test_plan_invariants(dtype, rows, stride, k):
 
 
 def test_plan_splits():
-    # many rows: one CTA per row; short ones get the 128-thread shape
+    # many rows of at most 32 KB: the row-resident kernel; a little longer: the
+    # streaming kernel's 128-thread shape
     p = T.dsel_plan(T.DSEL_BF16, 4096, 16384, 512, **PEAK)[1]
-    assert p["cluster"] == 1 and p["threads"] == 128
+    assert p["kernel"] == T.DSEL_KERNEL_RESIDENT and p["threads"] == 256
+    p = T.dsel_plan(T.DSEL_BF16, 4096, 16400, 512, **PEAK)[1]
+    assert p["kernel"] == T.DSEL_KERNEL_STREAM and p["cluster"] == 1 and p["threads"] == 128
+    # fewer rows than SMs: never resident
+    assert T.dsel_plan(T.DSEL_BF16, 147, 16384, 512, **PEAK)[1]["kernel"] == T.DSEL_KERNEL_STREAM
     assert T.dsel_plan(T.DSEL_F32, 256, 129280, 4096, **PEAK)[1]["threads"] == 512
     # long rows, k <= 1024, at least as many rows as SMs: 256 threads, two CTAs per SM
     assert T.dsel_plan(T.DSEL_F32, 256, 129280, 1024, **PEAK)[1]["threads"] == 256

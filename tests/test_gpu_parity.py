@@ -148,18 +148,17 @@ def test_torch_wrapper_bf16():
 # the workload families at full size (the bench's launch configuration)
 # --------------------------------------------------------------------------- #
 # --------------------------------------------------------------------------- #
-# the 128-thread shape: at least as many rows as SMs, rows of one or two rounds
+# the 128-thread shape: at least as many rows as SMs, bf16 rows of one or two rounds
 # --------------------------------------------------------------------------- #
 SHORT = [
-    # (seed, dtype, rows, stride, k, dist, order)
+    # (seed, dtype, rows, stride, k, dist, order): bf16 rows above 32 KB (longer ones
+    # are resident in shared memory), at most two 128-thread rounds
     (301, "bf16", 160, 32768, 1, "normal", 1),
     (302, "bf16", 160, 32768, 512, "ties", 0),
-    (303, "bf16", 150, 16384, 4096, "normal", 1),
-    (304, "bf16", 300, 2048, 512, "ties", 1),
-    (305, "f32", 150, 8192, 64, "normal", 2),
-    (306, "f32", 160, 8192, 2000, "ties", 1),
-    (307, "f32", 200, 4096, 4096, "normal", 0),
-    (308, "f32", 149, 6144, 700, "ascending", 1),
+    (303, "bf16", 150, 16400, 4096, "normal", 1),
+    (304, "bf16", 300, 20480, 512, "ties", 1),
+    (305, "bf16", 150, 24576, 64, "ascending", 0),
+    (306, "bf16", 160, 30000 // 16 * 16, 2000, "equal", 1),
 ]
 
 
