@@ -95,6 +95,17 @@ __device__ __forceinline__ BinHit res_find_bin(const int* h, int t, int lane) {
   return r;
 }
 
+// Bit e set when element e of the vector is valid (e < valid) and its key is
+// >= t: one packed float compare against t's value per element pair (no NaN is
+// left when this runs, and -0 and +0 compare equal as floats and as keys).
+template <int DT>
+__device__ __forceinline__ uint32_t res_mask_ge(const uint4& x, uint32_t t, int valid) {
+  using E = Elem<DT>;
+  const uint32_t b = E::bits_of_key(t);
+  const uint32_t m = candidate_mask<DT>(x, DT == DSEL_BF16 ? (b | (b << 16)) : b);
+  return valid >= E::kPerVec ? m : (m & ((1u << valid) - 1u));
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __grid_constant__ KParams p) {
   using E = Elem<DT>;
@@ -226,13 +237,16 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
   uint32_t lo = kmin, hi = kmax;   // the k-th largest key lies in [lo, hi]
   int above = 0;                   // elements with key > hi
   if (nvec >= k) {
-    const int s = res_shift(kmax - gmin);
+    // bins 16 times narrower than [gmin, kmax] needs, the last one open below: the
+    // top sixteenth of the range, where the k-th largest maximum usually lies, at
+    // fine resolution
+    const int s = max(0, res_shift(kmax - gmin) - 4);
 #pragma unroll
     for (int i = 0; i < VPT; ++i)
-      if (gk[i] != 0u) atomicAdd(&hist[(kmax - gk[i]) >> s], 1);
+      if (gk[i] != 0u) atomicAdd(&hist[min((kmax - gk[i]) >> s, static_cast<uint32_t>(kResBins - 1))], 1);
     __syncthreads();
     const BinHit bh = res_find_bin(hist, k, lane);
-    lo = max(lo, res_bin_lo(kmax, gmin, bh.bin, s));
+    lo = max(lo, bh.bin == kResBins - 1 ? gmin : res_bin_lo(kmax, gmin, bh.bin, s));
   }
 
   // ---- 4. the exact k-th largest key: histogram levels over [lo, hi] ----
@@ -247,11 +261,13 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
       if (gk[i] >= lo) {   // only vectors whose maximum reaches lo hold such keys
         const int v = i * T + tid;
         const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
-        const int valid = min(PV, n - v * PV);
-#pragma unroll
-        for (int e = 0; e < PV; ++e) {
-          const uint32_t kk = E::key(vec_elem<DT>(x, e));
-          if (e < valid && kk >= lo && kk <= hi) atomicAdd(&h[(hi - kk) >> s], 1);
+        uint32_t m = res_mask_ge<DT>(x, lo, n - v * PV);
+#pragma unroll 1
+        while (m != 0u) {
+          const int e = __ffs(m) - 1;
+          m &= m - 1u;
+          const uint32_t kk = E::key(vec_elem_dyn<DT>(x, e));
+          if (kk <= hi) atomicAdd(&h[(hi - kk) >> s], 1);
         }
       }
     }
@@ -273,11 +289,13 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
         if (gk[i] >= blo) {
           const int v = i * T + tid;
           const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
-          const int valid = min(PV, n - v * PV);
-#pragma unroll
-          for (int e = 0; e < PV; ++e) {
-            const uint32_t kk = E::key(vec_elem<DT>(x, e));
-            if (e < valid && kk >= blo && kk <= bhi) {
+          uint32_t m = res_mask_ge<DT>(x, blo, n - v * PV);
+#pragma unroll 1
+          while (m != 0u) {
+            const int e = __ffs(m) - 1;
+            m &= m - 1u;
+            const uint32_t kk = E::key(vec_elem_dyn<DT>(x, e));
+            if (kk <= bhi) {
               const int pos = atomicAdd(&ctl.tie_n, 1);
               if (pos < kResBins) lst[pos] = kk;
             }
@@ -325,11 +343,12 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
     if (gk[i] >= tkey) {
       const int v = i * T + tid;
       const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
-      const int valid = min(PV, n - v * PV);
-#pragma unroll
-      for (int e = 0; e < PV; ++e) {
-        const uint32_t kk = E::key(vec_elem<DT>(x, e));
-        if (e < valid) c += kk > tkey ? 1u : (kk == tkey ? 0x10000u : 0u);
+      uint32_t m = res_mask_ge<DT>(x, tkey, n - v * PV);
+#pragma unroll 1
+      while (m != 0u) {
+        const int e = __ffs(m) - 1;
+        m &= m - 1u;
+        c += E::key(vec_elem_dyn<DT>(x, e)) > tkey ? 1u : 0x10000u;
       }
     }
     has |= c != 0u ? 1u << i : 0u;
@@ -381,13 +400,14 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
       int gtb = static_cast<int>(pre & 0xFFFFu), eqb = static_cast<int>(pre >> 16);
       const int v = i * T + tid;
       const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
-      const int valid = min(PV, n - v * PV);
-#pragma unroll
-      for (int e = 0; e < PV; ++e) {
-        const uint32_t b = vec_elem<DT>(x, e);
-        const uint32_t kk = E::key(b);
-        if (e < valid && kk >= tkey) {
-          const bool gt = kk > tkey;
+      uint32_t m = res_mask_ge<DT>(x, tkey, n - v * PV);
+#pragma unroll 1
+      while (m != 0u) {   // ascending element order: index order
+        const int e = __ffs(m) - 1;
+        m &= m - 1u;
+        const uint32_t b = vec_elem_dyn<DT>(x, e);
+        {
+          const bool gt = E::key(b) > tkey;
           if (gt || eqb < need_eq) {
             const int pos = gtb + min(eqb, need_eq);
             const uint32_t idx = static_cast<uint32_t>(v * PV + e);
