@@ -116,8 +116,9 @@ extern "C" {
 /* Launch plan chosen for a call (see dsel_plan). */
 typedef struct {
   int32_t threads;       /* threads per CTA: 512 (one CTA per SM); with at least as many rows as
-                            SMs, 128 for short rows (several CTAs per SM) or 256 for long rows
-                            with k <= 1024 (two CTAs per SM) */
+                            SMs, 256 for the row-resident kernel (rows of at most 32 KB, four
+                            CTAs per SM), 128 for other short rows (several CTAs per SM) or 256
+                            for long rows with k <= 1024 (two CTAs per SM) */
   int32_t cluster;       /* CTAs per thread-block cluster working on one row */
   int32_t groups;        /* clusters per row (> 1: split-row plan with a merge launch) */
   int32_t block;         /* B: elements per contiguous block visited in random order */
@@ -125,7 +126,7 @@ typedef struct {
   int32_t round;         /* elements the CTA filters between two buffer checks */
   int32_t capacity;      /* candidate-buffer slots per CTA: k + B2 + slack (512 threads: 4096, or
                             2048 for k > 1024; 128 or 256 threads: 1024), at least next_pow2(k)
-                            and 4096 */
+                            and 4096; the row-resident kernel: next_pow2(k) */
   int32_t stages;        /* blocks kept in flight per CTA (shared-memory ring) */
   int32_t idx_bits;      /* bits of the in-row index used to break ties */
   int32_t smem_bytes;    /* dynamic shared memory per CTA */

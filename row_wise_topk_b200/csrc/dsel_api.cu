@@ -141,7 +141,7 @@ int run_shape(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStre
 }
 
 template <int DT>
-int run_resident(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
+int run_resident(const KParams& base, int64_t rows, cudaStream_t st, DevInfo* di) {
   auto rk = topk_resident_kernel<DT>;
   if (!di->res_attrs_set[DT]) {
     if (cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) != cudaSuccess)
@@ -158,14 +158,13 @@ int run_resident(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaS
   kp.off_ctl = rl.ctl;
   if (rows > 0x7FFFFFFF) return DSEL_ERR_ROWS;
   if (launch_cluster(rk, unsigned(rows), kResThreads, 1, rl.total, st, kp) != cudaSuccess) return DSEL_ERR_CUDA;
-  (void)pl;
   return DSEL_OK;
 }
 
 // The planner returns split-row plans (groups > 1) only with the 512-thread shape.
 template <int DT>
 int run(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
-  if (pl.kernel == DSEL_KERNEL_RESIDENT) return run_resident<DT>(base, pl, rows, st, di);
+  if (pl.kernel == DSEL_KERNEL_RESIDENT) return run_resident<DT>(base, rows, st, di);
   if (pl.threads == kThreadsShort) return run_shape<DT, kThreadsShort>(base, pl, rows, st, di);
   if (pl.threads == kThreadsMid) return run_shape<DT, kThreadsMid>(base, pl, rows, st, di);
   if (pl.threads == kThreads) return run_shape<DT, kThreads>(base, pl, rows, st, di);

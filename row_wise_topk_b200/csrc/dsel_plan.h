@@ -104,24 +104,26 @@ inline SmemLayout stream_layout(int64_t stages, int64_t block, int64_t capacity,
   return l;
 }
 
-// Row-resident kernel: the row, one mbarrier per 4 KB chunk, three 1024-bin
-// histograms, the scan table ([8 rounds][8 warps] totals, then [8 warps][8
-// rounds] offsets), candidate arrays of next_pow2(k) entries (value order and the
-// sampling step sort there) and the control block.
+// Row-resident kernel: the row, one mbarrier per 4 KB chunk (256 threads x 16
+// bytes), three 1024-bin histograms, the scan table ([8 rounds][8 warps] totals,
+// then [8 warps][8 rounds] offsets), candidate arrays of next_pow2(k) entries
+// (value order and the sampling step sort there) and the control block.
 struct ResLayout {
   uint32_t bars, hist, tab, cb, ci, ctl, total;
 };
 
 inline ResLayout resident_layout(int64_t row_stride, int32_t k, int eb) {
   auto up = [](int64_t v, int64_t a) { return (v + a - 1) / a * a; };
+  const int vpt = kResRowBytes / (kResThreads * kVecBytes);
+  const int threads = kResThreads;
   ResLayout l{};
   int64_t off = up(row_stride * eb, 128);
   l.bars = uint32_t(off);
-  off += 8 * 8;
+  off += up(int64_t(vpt) * 8, 16);
   l.hist = uint32_t(off);
   off += 3 * 1024 * 4;
   l.tab = uint32_t(off);
-  off += 2 * 8 * 8 * 4;
+  off += 2 * int64_t(vpt) * (threads / 32) * 4;
   const int64_t kp2 = next_pow2(k);
   l.cb = uint32_t(off);
   off += up(kp2 * eb, 16);

@@ -1,4 +1,5 @@
-// Row-resident TopK: rows that fit in shared memory, one CTA of 256 threads per row.
+// Row-resident TopK: one CTA of 256 threads per row holds the whole row (at most
+// 32 KB: 16,384 bf16 or 8,192 f32 elements) in shared memory.
 //
 // The streaming kernel (topk_stream_kernel) follows the method of "DeepSeek
 // releases DeepSelect, a TopK kernel for sparse attention and sampling" (method
@@ -6,8 +7,8 @@
 // radix-select compactions.  Its fixed cost per row (seed histogram, exact test,
 // final select, index ranking, each behind several barriers) dominates when a
 // row is only a few thousand elements, as in a batch of variable-length indexer
-// rows.  A row of at most 32 KB fits in shared memory next to everything else,
-// so this kernel reads it once into shared memory and selects there, exactly:
+// rows.  Such a row fits in shared memory next to everything else, so this
+// kernel reads it once into shared memory and selects there, exactly:
 //
 //   1. bulk copies of the row, one 4 KB chunk (one 16-byte vector per thread)
 //      per mbarrier, so that step 2 starts on the first chunk;
@@ -25,19 +26,22 @@
 //      give every selected element its output slot (equal keys are taken in
 //      index order, the tie rule value-descending then index-ascending).
 //
-// Value order and the sampling step put the k selected entries in shared memory
-// instead and finish as the streaming kernel does (bitonic sort, draw).
-// Histogram levels rotate over three buffers; the buffer of level L + 2 is
-// cleared after the barrier of level L, when its last readers are done.
+// Every pass tests a whole vector against its bound with packed compares and
+// visits only the elements that pass, in rolled loops.  Histogram levels rotate
+// over three buffers; the buffer of level L + 2 is cleared after the barrier of
+// level L, when its last readers are done.  Value order and the sampling step
+// put the k selected entries in shared memory instead and finish as the
+// streaming kernel does (bitonic sort, draw).
 #pragma once
 
 #include "dsel_kernels.cuh"
 
 namespace dsel {
 
-constexpr int kResVpt = 8;                    // vectors per thread: rows up to 256 x 8 x 16 B = 32 KB
 constexpr int kResBins = 1024;
-static_assert(kResThreads * kResVpt * kVecBytes == kResRowBytes, "resident row capacity");
+constexpr int kResVpt = kResRowBytes / (kResThreads * kVecBytes);   // vectors per thread: 8
+static_assert(kResVpt == 8, "rows of up to 32 KB: 8 vectors per thread");
+static_assert(kMaxK <= 4096 && kResRowBytes / 2 < (1 << 20), "output counts pack as 12 + 20 bits");
 
 // Largest and smallest key of a 16-byte vector; true when it holds a NaN.
 template <int DT>
@@ -88,11 +92,11 @@ __device__ __forceinline__ BinHit res_find_bin(const int* h, int t, int lane) {
   const int c = h[32 * L + lane];
   const int incl2 = warp_incl_scan(c, lane) + base;
   const int j = max(0, __ffs(__ballot_sync(0xffffffffu, incl2 >= t)) - 1);
-  BinHit r;
-  r.bin = 32 * L + j;
-  r.cnt = __shfl_sync(0xffffffffu, c, j);
-  r.before = __shfl_sync(0xffffffffu, incl2, j) - r.cnt;
-  return r;
+  BinHit res;
+  res.bin = 32 * L + j;
+  res.cnt = __shfl_sync(0xffffffffu, c, j);
+  res.before = __shfl_sync(0xffffffffu, incl2, j) - res.cnt;
+  return res;
 }
 
 // Bit e set when element e of the vector is valid (e < valid) and its key is
@@ -106,22 +110,26 @@ __device__ __forceinline__ uint32_t res_mask_ge(const uint4& x, uint32_t t, int 
   return valid >= E::kPerVec ? m : (m & ((1u << valid) - 1u));
 }
 
+// One CTA per row (blockIdx.x).
 template <int DT>
 __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __grid_constant__ KParams p) {
   using E = Elem<DT>;
   using bits_t = typename E::bits_t;
   constexpr int T = kResThreads;
+  constexpr int VPT = kResVpt;
   constexpr int NW = T / 32;
   constexpr int PV = E::kPerVec;
-  constexpr int VPT = kResVpt;
-  constexpr int CH = T * kVecBytes;   // bytes per chunk: one vector per thread
+  constexpr int CH = T * kVecBytes;    // bytes per chunk: one vector per thread
+  constexpr int NE = VPT * NW;         // scan-table entries
+  constexpr int EPL = (NE + 31) / 32;  // of them per lane
+  static_assert(VPT <= 32, "one bit per round");
 
   extern __shared__ __align__(1024) unsigned char smem[];
   const unsigned char* rowb = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bars);
   int* hist = reinterpret_cast<int*>(smem + p.off_hist);            // 3 x kResBins
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem + p.off_tab);    // [VPT][NW] packed warp totals
-  uint32_t* offw = tab + VPT * NW;                                   // [NW][VPT] packed offsets
+  uint32_t* offw = tab + NE;                                         // [NW][VPT] packed offsets
   bits_t* cb = reinterpret_cast<bits_t*>(smem + p.off_cb);
   uint32_t* ci = reinterpret_cast<uint32_t*>(smem + p.off_ci);
   Ctl& ctl = *reinterpret_cast<Ctl*>(smem + p.off_ctl);
@@ -156,12 +164,12 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
   }
   const int n = static_cast<int>(n64);   // <= kResRowBytes / 2
   const int nvec = (n + PV - 1) / PV;
-  const uint32_t row_bytes = static_cast<uint32_t>((n + 15) / 16 * 16) * E::kBytes;   // multiple of 16 B
-  const int nch = static_cast<int>((row_bytes + CH - 1) / CH);                        // <= VPT
+  const uint32_t bytes = static_cast<uint32_t>((n + 15) / 16 * 16) * E::kBytes;   // multiple of 16 B
+  const int nch = static_cast<int>((bytes + CH - 1) / CH);                       // <= VPT
 
   // ---- 1. bulk copies: chunk c (vectors c*T .. c*T + T - 1) by lane c of warp 0 ----
   if (warp == 0 && lane < nch) {
-    const uint32_t b = min(static_cast<uint32_t>(CH), row_bytes - static_cast<uint32_t>(lane) * CH);
+    const uint32_t b = min(static_cast<uint32_t>(CH), bytes - static_cast<uint32_t>(lane) * CH);
     const uint32_t bar = smem_u32(&bars[lane]);
     mbar_expect_tx(bar, b);
     bulk_g2s(smem_u32(smem + lane * CH),
@@ -249,6 +257,16 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
     lo = max(lo, bh.bin == kResBins - 1 ? gmin : res_bin_lo(kmax, gmin, bh.bin, s));
   }
 
+  // Rounds whose vector (this thread's) has a key >= t: one bit per round.  The
+  // passes below loop over these bits, and over the passing elements of each
+  // vector, in rolled loops (small code: the instruction cache holds it).
+  auto rounds_ge = [&](uint32_t t) -> uint32_t {
+    uint32_t r = 0u;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) r |= gk[i] >= t ? (1u << i) : 0u;
+    return r;
+  };
+
   // ---- 4. the exact k-th largest key: histogram levels over [lo, hi] ----
   uint32_t tkey;   // the k-th largest key
   int n_gt;        // elements with key > tkey (< k)
@@ -256,19 +274,20 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
   for (int level = 1;; ++level) {
     int* h = hist + (level % 3) * kResBins;
     const int s = res_shift(hi - lo);
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-      if (gk[i] >= lo) {   // only vectors whose maximum reaches lo hold such keys
-        const int v = i * T + tid;
-        const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
-        uint32_t m = res_mask_ge<DT>(x, lo, n - v * PV);
+    uint32_t rm = rounds_ge(lo);   // only vectors whose maximum reaches lo hold such keys
 #pragma unroll 1
-        while (m != 0u) {
-          const int e = __ffs(m) - 1;
-          m &= m - 1u;
-          const uint32_t kk = E::key(vec_elem_dyn<DT>(x, e));
-          if (kk <= hi) atomicAdd(&h[(hi - kk) >> s], 1);
-        }
+    while (rm != 0u) {
+      const int i = __ffs(rm) - 1;
+      rm &= rm - 1u;
+      const int v = i * T + tid;
+      const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
+      uint32_t m = res_mask_ge<DT>(x, lo, n - v * PV);
+#pragma unroll 1
+      while (m != 0u) {
+        const int e = __ffs(m) - 1;
+        m &= m - 1u;
+        const uint32_t kk = E::key(vec_elem_dyn<DT>(x, e));
+        if (kk <= hi) atomicAdd(&h[(hi - kk) >> s], 1);
       }
     }
     __syncthreads();
@@ -284,21 +303,22 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
     if (bh.cnt <= kTieMax) {
       // rank the boundary bin's members by key; the free buffer of level + 1 holds them
       uint32_t* lst = reinterpret_cast<uint32_t*>(hist + ((level + 1) % 3) * kResBins);
-#pragma unroll
-      for (int i = 0; i < VPT; ++i) {
-        if (gk[i] >= blo) {
-          const int v = i * T + tid;
-          const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
-          uint32_t m = res_mask_ge<DT>(x, blo, n - v * PV);
+      uint32_t rb = rounds_ge(blo);
 #pragma unroll 1
-          while (m != 0u) {
-            const int e = __ffs(m) - 1;
-            m &= m - 1u;
-            const uint32_t kk = E::key(vec_elem_dyn<DT>(x, e));
-            if (kk <= bhi) {
-              const int pos = atomicAdd(&ctl.tie_n, 1);
-              if (pos < kResBins) lst[pos] = kk;
-            }
+      while (rb != 0u) {
+        const int i = __ffs(rb) - 1;
+        rb &= rb - 1u;
+        const int v = i * T + tid;
+        const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
+        uint32_t m = res_mask_ge<DT>(x, blo, n - v * PV);
+#pragma unroll 1
+        while (m != 0u) {
+          const int e = __ffs(m) - 1;
+          m &= m - 1u;
+          const uint32_t kk = E::key(vec_elem_dyn<DT>(x, e));
+          if (kk <= bhi) {
+            const int pos = atomicAdd(&ctl.tie_n, 1);
+            if (pos < kResBins) lst[pos] = kk;
           }
         }
       }
@@ -332,48 +352,35 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
   }
 
   // ---- 5. output slots in index order ----
-  // per vector: (keys > tkey) | (keys == tkey) << 16, scanned over the row in
-  // vector order (round i, then thread); both fields stay below 2^16
+  // per vector: (keys > tkey) | (keys == tkey) << 12, scanned over the row in
+  // vector order (round, thread).  Fewer than k <= 4096 keys exceed tkey, so
+  // every prefix of the first field fits its 12 bits; the second counts at most
+  // the row's 16,384 elements.  Both come from two packed compares (keys >= tkey,
+  // keys >= tkey + 1; no key exceeds kmax).
   const int need_eq = k - n_gt;
-  uint32_t excl[VPT];
-  uint32_t has = 0u;
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    uint32_t c = 0u;
-    if (gk[i] >= tkey) {
-      const int v = i * T + tid;
-      const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
-      uint32_t m = res_mask_ge<DT>(x, tkey, n - v * PV);
+  const uint32_t rt = rounds_ge(tkey);
+  auto vec_count = [&](int i) -> uint32_t {
+    const int v = i * T + tid;
+    const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
+    const uint32_t ge = __popc(res_mask_ge<DT>(x, tkey, n - v * PV));
+    const uint32_t gt = tkey < kmax ? __popc(res_mask_ge<DT>(x, tkey + 1u, n - v * PV)) : 0u;
+    return gt | ((ge - gt) << 12);
+  };
 #pragma unroll 1
-      while (m != 0u) {
-        const int e = __ffs(m) - 1;
-        m &= m - 1u;
-        c += E::key(vec_elem_dyn<DT>(x, e)) > tkey ? 1u : 0x10000u;
-      }
-    }
-    has |= c != 0u ? 1u << i : 0u;
-    excl[i] = 0u;
-    if (i < nch && __any_sync(0xffffffffu, c != 0u)) {
-      uint32_t incl = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      excl[i] = incl - c;
-      if (lane == 31) tab[i * NW + warp] = incl;
-    } else if (i < nch && lane == 0) {
-      tab[i * NW + warp] = 0u;
-    }
+  for (int i = 0; i < nch; ++i) {   // warp totals per round
+    const bool mine = (rt >> i) & 1u;
+    uint32_t w = 0u;
+    if (__any_sync(0xffffffffu, mine)) w = __reduce_add_sync(0xffffffffu, mine ? vec_count(i) : 0u);
+    if (lane == 0) tab[i * NW + warp] = w;
   }
   __syncthreads();
+  const bool to_smem = p.order == DSEL_ORDER_VALUE || p.token_out != nullptr;
   {   // every warp: exclusive prefix of the [round][warp] totals; keep this warp's column
-    static_assert(VPT * NW <= 128, "four table entries per lane");
     const int ne = nch * NW;
-    uint32_t t4[4], run = 0u;
+    uint32_t t4[EPL], run = 0u;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = 4 * lane + j;
+    for (int j = 0; j < EPL; ++j) {
+      const int e = EPL * lane + j;
       t4[j] = run;
       run += e < ne ? tab[e] : 0u;
     }
@@ -383,49 +390,54 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
       const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += y;
     }
-    const uint32_t base = incl - run;
+    const uint32_t b0 = incl - run;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = 4 * lane + j;
-      if (e < ne && e % NW == warp) offw[warp * VPT + e / NW] = base + t4[j];
+    for (int j = 0; j < EPL; ++j) {
+      const int e = EPL * lane + j;
+      if (e < ne && e % NW == warp) offw[warp * VPT + e / NW] = b0 + t4[j];
     }
     __syncwarp();
   }
-  const bool to_smem = p.order == DSEL_ORDER_VALUE || p.token_out != nullptr;
   const int64_t obase = row * static_cast<int64_t>(k);
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    if (has & (1u << i)) {
-      const uint32_t pre = offw[warp * VPT + i] + excl[i];
-      int gtb = static_cast<int>(pre & 0xFFFFu), eqb = static_cast<int>(pre >> 16);
-      const int v = i * T + tid;
-      const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
-      uint32_t m = res_mask_ge<DT>(x, tkey, n - v * PV);
 #pragma unroll 1
-      while (m != 0u) {   // ascending element order: index order
-        const int e = __ffs(m) - 1;
-        m &= m - 1u;
-        const uint32_t b = vec_elem_dyn<DT>(x, e);
-        {
-          const bool gt = E::key(b) > tkey;
-          if (gt || eqb < need_eq) {
-            const int pos = gtb + min(eqb, need_eq);
-            const uint32_t idx = static_cast<uint32_t>(v * PV + e);
-            if (pos < k) {
-              if (to_smem) {
-                cb[pos] = static_cast<bits_t>(b);
-                ci[pos] = idx;
-              } else {
-                if (p.index_i64) static_cast<int64_t*>(p.indices_out)[obase + pos] = static_cast<int64_t>(idx);
-                else static_cast<int32_t*>(p.indices_out)[obase + pos] = static_cast<int32_t>(idx);
-                if (p.return_value) static_cast<bits_t*>(p.values_out)[obase + pos] = static_cast<bits_t>(b);
-              }
-            }
+  for (int i = 0; i < nch; ++i) {
+    const bool mine = (rt >> i) & 1u;
+    if (!__any_sync(0xffffffffu, mine)) continue;   // warp-uniform
+    const uint32_t c = mine ? vec_count(i) : 0u;
+    uint32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (c == 0u) continue;
+    const uint32_t pre = offw[warp * VPT + i] + incl - c;
+    int gtb = static_cast<int>(pre & 0xFFFu), eqb = static_cast<int>(pre >> 12);
+    const int v = i * T + tid;
+    const uint4 x = *reinterpret_cast<const uint4*>(rowb + v * kVecBytes);
+    uint32_t m = res_mask_ge<DT>(x, tkey, n - v * PV);
+#pragma unroll 1
+    while (m != 0u) {   // ascending element order: index order
+      const int e = __ffs(m) - 1;
+      m &= m - 1u;
+      const uint32_t b = vec_elem_dyn<DT>(x, e);
+      const bool gt = E::key(b) > tkey;
+      if (gt || eqb < need_eq) {
+        const int pos = gtb + min(eqb, need_eq);
+        const uint32_t idx = static_cast<uint32_t>(v * PV + e);
+        if (pos < k) {
+          if (to_smem) {
+            cb[pos] = static_cast<bits_t>(b);
+            ci[pos] = idx;
+          } else {
+            if (p.index_i64) static_cast<int64_t*>(p.indices_out)[obase + pos] = static_cast<int64_t>(idx);
+            else static_cast<int32_t*>(p.indices_out)[obase + pos] = static_cast<int32_t>(idx);
+            if (p.return_value) static_cast<bits_t*>(p.values_out)[obase + pos] = static_cast<bits_t>(b);
           }
-          if (gt) ++gtb;
-          else ++eqb;
         }
       }
+      if (gt) ++gtb;
+      else ++eqb;
     }
   }
   if (!to_smem) return;

@@ -125,6 +125,8 @@ PEAK = dict(num_sms=148, smem_optin=232448, max_cluster=8)
     (T.DSEL_BF16, 3, 16, 4096), (T.DSEL_F32, 1, 16, 1),
     (T.DSEL_BF16, 4096, 16400, 512), (T.DSEL_F32, 300, 8192, 4096), (T.DSEL_F32, 300, 8208, 64),
     (T.DSEL_BF16, 148, 16, 4096), (T.DSEL_F32, 200, 4096, 1),
+    (T.DSEL_BF16, 100, 65536, 512), (T.DSEL_F32, 37, 131072, 1000), (T.DSEL_BF16, 20, 1 << 19, 64),
+    (T.DSEL_F32, 73, 32768, 64), (T.DSEL_BF16, 147, 16400, 4096),
 ])
 def test_plan_invariants(dtype, rows, stride, k):
     st, p = T.dsel_plan(dtype, rows, stride, k, **PEAK)
@@ -188,7 +190,7 @@ def test_plan_splits():
     assert T.dsel_plan(T.DSEL_F32, 256, 129280, 1024, **PEAK)[1]["threads"] == 256
     # 64 indexer rows: two CTAs per row
     p = T.dsel_plan(T.DSEL_BF16, 64, 131072, 512, **PEAK)[1]
-    assert (p["cluster"], p["groups"]) == (2, 1)
+    assert (p["kernel"], p["cluster"], p["groups"]) == (T.DSEL_KERNEL_STREAM, 2, 1)
     # a single 2^28 row uses several clusters
     p = T.dsel_plan(T.DSEL_F32, 1, 1 << 28, 1000, **PEAK)[1]
     assert p["groups"] > 1 and p["cluster"] == 8

@@ -133,3 +133,4 @@ def test_resident_sampling_step():
     u = W.uniforms(rows, seed=11)
     check_sample(w, 0.8, 0.9, u)
     check_sample(w, 0.0, 1.0, u, return_topk=False)
+
