@@ -366,11 +366,21 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
     const uint32_t gt = tkey < kmax ? __popc(res_mask_ge<DT>(x, tkey + 1u, n - v * PV)) : 0u;
     return gt | ((ge - gt) << 12);
   };
+  // this thread's counts per round, one byte each (greater | equal << 4, both <= 8):
+  // rounds 0-3 in cnt_lo, 4-7 in cnt_hi, for the write pass
+  static_assert(VPT <= 8 && PV <= 8, "a round's counts fit one byte");
+  uint32_t cnt_lo = 0u, cnt_hi = 0u;
 #pragma unroll 1
   for (int i = 0; i < nch; ++i) {   // warp totals per round
     const bool mine = (rt >> i) & 1u;
     uint32_t w = 0u;
-    if (__any_sync(0xffffffffu, mine)) w = __reduce_add_sync(0xffffffffu, mine ? vec_count(i) : 0u);
+    if (__any_sync(0xffffffffu, mine)) {
+      const uint32_t c = mine ? vec_count(i) : 0u;
+      w = __reduce_add_sync(0xffffffffu, c);
+      const uint32_t byte = (c & 0xFu) | ((c >> 12) << 4);
+      if (i < 4) cnt_lo |= byte << (8 * i);
+      else cnt_hi |= byte << (8 * (i - 4));
+    }
     if (lane == 0) tab[i * NW + warp] = w;
   }
   __syncthreads();
@@ -403,7 +413,8 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
   for (int i = 0; i < nch; ++i) {
     const bool mine = (rt >> i) & 1u;
     if (!__any_sync(0xffffffffu, mine)) continue;   // warp-uniform
-    const uint32_t c = mine ? vec_count(i) : 0u;
+    const uint32_t byte = ((i < 4 ? cnt_lo : cnt_hi) >> (8 * (i & 3))) & 0xFFu;
+    const uint32_t c = (byte & 0xFu) | ((byte >> 4) << 12);
     uint32_t incl = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
