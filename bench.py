@@ -451,7 +451,9 @@ def run_ours(args, w, world, rank, local, pg):
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
                      "kernel": ("topk_resident_kernel" if plan.get("kernel") == T.DSEL_KERNEL_RESIDENT
                                 else "topk_stream_kernel" + ("+topk_merge_kernel" if launches_per_step > 1 else "")),
-                     "launch_ms": round(kern_ms, 5)},
+                     "launch_ms": round(kern_ms, 5),
+                     "launch_ms_median": round(statistics.median(per_step_ms), 5),
+                     "launch_ms_min": round(min(per_step_ms), 5)},
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},

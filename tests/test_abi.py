@@ -199,3 +199,14 @@ def test_plan_splits():
 def test_plan_rejects_bad_args():
     assert T.dsel_plan(T.DSEL_F32, 4, 8191, 64, **PEAK)[0] == header_define("DSEL_ERR_STRIDE")
     assert T.dsel_plan(T.DSEL_F32, 4, 8192, 5000, **PEAK)[0] == header_define("DSEL_ERR_K")
+
+
+def test_resident_plan_fits_four_ctas_per_sm():
+    # the varlen indexer batch: 16,384-element bf16 rows, k = 512; a B200 SM has 228 KB of
+    # shared memory and reserves 1 KB per CTA
+    p = T.dsel_plan(T.DSEL_BF16, 4096, 16384, 512, **PEAK)[1]
+    assert p["kernel"] == T.DSEL_KERNEL_RESIDENT
+    assert 4 * (p["smem_bytes"] + 1024) <= 228 * 1024
+    # value order with the largest k on f32 rows still fits one CTA's opt-in limit
+    p = T.dsel_plan(T.DSEL_F32, 4096, 8192, 4096, **PEAK)[1]
+    assert p["kernel"] == T.DSEL_KERNEL_RESIDENT and p["smem_bytes"] <= PEAK["smem_optin"]
