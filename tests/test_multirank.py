@@ -172,3 +172,9 @@ def test_row_split_over_two_ranks_gloo(dtype, rows, n, k):
     vals = np.frombuffer(got[0][0], dtype=np.uint16 if dtype == "bf16" else np.uint32).reshape(rows, k)
     assert np.array_equal(idx, exp.indices)
     assert np.array_equal(vals, exp.values)
+
+
+def test_roofline_launch_time():
+    # one launch per step: the timed region's average; two (stream + merge): the isolated mean
+    assert bench.roofline_launch_ms(0.0225, 1, [0.0286, 0.0290]) == 0.0225
+    assert abs(bench.roofline_launch_ms(0.5, 2, [0.2, 0.4]) - 0.3) < 1e-12
