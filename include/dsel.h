@@ -41,9 +41,14 @@
  *   stream       a cudaStream_t passed as void* (NULL = legacy default stream).
  * The caller owns all memory.  Calls are asynchronous on `stream` and never
  * synchronise the host.  Plans that split one row over several thread-block
- * clusters use a per-(device, stream) workspace that the library allocates once
- * (cudaMalloc, outside any stream capture) and reuses; all other plans allocate
- * nothing.
+ * clusters (rows longer than sixteen 128 KB slices) use a per-(device, stream)
+ * workspace that the library allocates on first use and grows in stream order
+ * (cudaMallocAsync / cudaFreeAsync on `stream`); it never allocates inside a stream
+ * capture (such a call returns DSEL_ERR_WORKSPACE: make the first call of a
+ * split-row shape on a stream before capturing).  At most 16 streams per device
+ * keep a workspace; a further stream evicts the least recently used one with
+ * cudaFree, which waits for the device.  All other plans allocate nothing;
+ * dsel_topk_noalloc never allocates.
  *
  * Special rows and sentinel values
  *   - end[r] <= k ("short row"): all end[r] entries are returned in index order
@@ -104,7 +109,7 @@ extern "C" {
 #define DSEL_ERR_NAN_MODE (-9)     /* nan_mode not DSEL_NAN_TRAP / DSEL_NAN_FLAG */
 #define DSEL_ERR_ORDER (-10)       /* sorted_index out of range, or value order on bf16 */
 #define DSEL_ERR_DEVICE (-11)      /* current device is not sm_100 */
-#define DSEL_ERR_WORKSPACE (-12)   /* the split-row workspace could not be allocated */
+#define DSEL_ERR_WORKSPACE (-12)   /* the split-row workspace could not be allocated (or the stream is capturing) */
 #define DSEL_ERR_CUDA (-13)        /* a CUDA runtime call failed (launch error forwarded) */
 #define DSEL_ERR_DEVICE_TIMEOUT (-14) /* a kernel gave up a bounded wait (see dsel_device_status) */
 #define DSEL_ERR_UNAVAILABLE (-15) /* the entry point is not part of this build */
@@ -134,11 +139,17 @@ typedef struct {
   int32_t kernel;        /* DSEL_KERNEL_STREAM, or DSEL_KERNEL_RESIDENT: at least as many rows as
                             SMs and rows of at most 32 KB, one 256-thread CTA per row holding the
                             whole row in shared memory (block = the 4 KB bulk-copy chunk,
-                            round = row_stride, stages = chunks per row, b2 = 0) */
+                            round = row_stride, stages = chunks per row, b2 = 0), or
+                            DSEL_KERNEL_SLICE: rows cut into `cluster` slices of at most 160 KB,
+                            one 512-thread CTA per slice holding it whole in shared memory, the
+                            slices of a row in one cluster (round = slice elements, block =
+                            elements per warp block, stages = 16-byte vectors per thread,
+                            b2 = capacity = 0); index order and unspecified order only */
 } dsel_plan_t;
 
 #define DSEL_KERNEL_STREAM 0
 #define DSEL_KERNEL_RESIDENT 1
+#define DSEL_KERNEL_SLICE 2
 
 /*
  * dsel_topk -- batched row-wise TopK (the operation described at the top).
@@ -174,9 +185,10 @@ DSEL_API int dsel_topk(const void* x, int dtype, int64_t rows, int64_t row_strid
  *   - A call whose plan needs more scratch than that returns DSEL_ERR_SCRATCH_LIMIT
  *     and launches nothing (on a 148-SM B200 this happens only for k >= 3640, on
  *     at most nine long rows split over several clusters).
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) and sets kernel attributes; make that first call
- *     before any stream capture.
+ *   - The first call on a device, whatever its shape, looks up the array's
+ *     device address (cudaGetSymbolAddress); the first call of each kernel shape
+ *     also sets that kernel's attributes.  Make those first calls before any
+ *     stream capture.
  *   - All calls on a device share the one array, which keeps the last call's
  *     contents (no slot has to start at zero: each call writes every slot it
  *     reads).  Calls whose work overlaps on the GPU (different streams, not
@@ -292,6 +304,14 @@ DSEL_API const char* dsel_status_string(int status);
 DSEL_API int dsel_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k,
                        int32_t num_sms, int32_t smem_optin, int32_t max_cluster,
                        dsel_plan_t* out);
+
+/* dsel_plan for a given output order: the plan dsel_topk would use with this
+ * sorted_index (value order, DSEL_ORDER_VALUE, and the sampling call never use the
+ * slice kernel; pass DSEL_ORDER_VALUE for the plan of dsel_topk_sample).  Makes no
+ * CUDA call.  Returns DSEL_OK or a DSEL_ERR_* code (DSEL_ERR_ORDER for a bad
+ * order). */
+DSEL_API int dsel_plan_for(int dtype, int64_t rows, int64_t row_stride, int32_t k, int sorted_index,
+                           int32_t num_sms, int32_t smem_optin, int32_t max_cluster, dsel_plan_t* out);
 
 /* Reads and clears the device-side status word that kernels set when a bounded
  * wait runs out (it should never happen).  Synchronises `stream`.  *status_out

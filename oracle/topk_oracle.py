@@ -116,6 +116,27 @@ def brute_force_row(v, k: int) -> list:
     return sorted(order[:k])
 
 
+def value_order(bits: np.ndarray, idx: np.ndarray, dtype: str) -> np.ndarray:
+    """Permutation that lists the entries (bits[i], idx[i]) in value order.
+
+    Value order (``sorted_index=2``, float32 only: narracomm, paragraph on install
+    and switches) is value descending, ties by ascending index, -0.0 equal to +0.0.
+    Reading for the rows no longer than k, which skip the NaN check and so may hold
+    a NaN: such a row is put in value order too (as torch.topk would order it), a
+    NaN taking its IEEE 754 totalOrder place -- sign bit clear: above +inf, a larger
+    payload higher; sign bit set: below -inf, a larger payload lower.
+    """
+    bits = np.asarray(bits)
+    v = decode(bits, dtype)
+    nan = np.isnan(v)
+    neg = np.signbit(v)
+    payload = bits.astype(np.int64) & (0x7F if dtype == "bf16" else 0x7FFFFF)
+    cls = np.where(nan, np.where(neg, 0, 2), 1)                  # -NaN < numbers < +NaN
+    within = np.where(nan, np.where(neg, payload, -payload), 0)  # rank inside a NaN class
+    num = np.where(nan, 0.0, -v) + 0.0                           # value descending, -0.0 == +0.0
+    return np.lexsort((np.asarray(idx), num, within, -cls))
+
+
 @dataclasses.dataclass
 class OracleResult:
     indices: np.ndarray                 # [rows, k] int32 | int64

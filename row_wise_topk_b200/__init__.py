@@ -25,7 +25,7 @@ DSEL_I32, DSEL_I64 = 0, 1
 DSEL_NAN_TRAP, DSEL_NAN_FLAG = 0, 1
 DSEL_ORDER_NONE, DSEL_ORDER_INDEX, DSEL_ORDER_VALUE = 0, 1, 2
 DSEL_IDX_PAD, DSEL_IDX_NAN, DSEL_IDX_BAD_END = -1, -2, -3
-DSEL_KERNEL_STREAM, DSEL_KERNEL_RESIDENT = 0, 1
+DSEL_KERNEL_STREAM, DSEL_KERNEL_RESIDENT, DSEL_KERNEL_SLICE = 0, 1, 2
 DSEL_OK = 0
 DSEL_ERR_SCRATCH_LIMIT = -16
 DSEL_NOALLOC_SCRATCH_BYTES = 512 * 1024
@@ -80,6 +80,9 @@ def _load() -> ctypes.CDLL:
     lib.dsel_stride_requirement.argtypes = [c_int]
     lib.dsel_status_string.restype = ctypes.c_char_p
     lib.dsel_status_string.argtypes = [c_int]
+    lib.dsel_plan_for.restype = c_int
+    lib.dsel_plan_for.argtypes = [c_int, c_i64, c_i64, ctypes.c_int32, c_int, ctypes.c_int32, ctypes.c_int32,
+                                  ctypes.c_int32, ctypes.POINTER(DselPlan)]
     lib.dsel_plan.restype = c_int
     lib.dsel_plan.argtypes = [c_int, c_i64, c_i64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                               ctypes.c_int32, ctypes.POINTER(DselPlan)]
@@ -141,6 +144,14 @@ def dsel_plan(dtype: int, rows: int, row_stride: int, k: int, num_sms: int = 148
               smem_optin: int = 232448, max_cluster: int = 8) -> Tuple[int, dict]:
     p = DselPlan()
     st = lib.dsel_plan(dtype, rows, row_stride, k, num_sms, smem_optin, max_cluster, ctypes.byref(p))
+    return st, p.as_dict()
+
+
+def dsel_plan_for(dtype: int, rows: int, row_stride: int, k: int, sorted_index: int, num_sms: int = 148,
+                  smem_optin: int = 232448, max_cluster: int = 8) -> Tuple[int, dict]:
+    p = DselPlan()
+    st = lib.dsel_plan_for(dtype, rows, row_stride, k, sorted_index, num_sms, smem_optin, max_cluster,
+                           ctypes.byref(p))
     return st, p.as_dict()
 
 

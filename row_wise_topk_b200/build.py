@@ -12,7 +12,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdsel.so")
 STATS_LIB = os.path.join(HERE, "libdsel_stats.so")   # same library, with per-CTA counters
 SOURCES = ["dsel_api.cu", "dsel_plan.cpp", "dsel_shard.cu"]
-HEADERS = ["dsel_device.cuh", "dsel_kernels.cuh", "dsel_plan.h", "dsel_resident.cuh"]
+HEADERS = ["dsel_device.cuh", "dsel_kernels.cuh", "dsel_plan.h", "dsel_resident.cuh", "dsel_slice.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

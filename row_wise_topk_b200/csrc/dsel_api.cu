@@ -8,11 +8,13 @@
 #include "dsel_kernels.cuh"
 #include "dsel_plan.h"
 #include "dsel_resident.cuh"
+#include "dsel_slice.cuh"
 
 namespace dsel {
 namespace {
 
 static_assert(sizeof(Ctl) <= kSharedFixedBytes, "control block outgrew its reservation");
+static_assert(sizeof(SliceCtl) <= kSliceCtlBytes, "slice control block outgrew its reservation");
 
 struct DevInfo {
   bool ready = false;
@@ -21,6 +23,8 @@ struct DevInfo {
   int major = 0;
   bool attrs_set[2][3] = {{false, false, false}, {false, false, false}};   // [dtype][shape]
   bool res_attrs_set[2] = {false, false};                                  // [dtype], resident kernel
+  bool slice_attrs_set[2] = {false, false};                                // [dtype], slice kernel
+  int slice_cluster = 0;   // largest cluster the slice kernel launches with (16 when schedulable, else 8)
 };
 
 std::mutex g_mu;
@@ -31,8 +35,11 @@ struct Workspace {
   void* stream;
   void* ptr;
   size_t bytes;
+  uint64_t used;   // last use (a counter), for eviction
 };
 std::vector<Workspace> g_ws;
+uint64_t g_ws_clock = 0;
+constexpr int kMaxWorkspaces = 16;   // per device
 
 int device_info(int dev, DevInfo** out) {
   if (dev < 0 || dev >= 64) return DSEL_ERR_DEVICE;
@@ -51,28 +58,53 @@ int device_info(int dev, DevInfo** out) {
   return DSEL_OK;
 }
 
-// One workspace per (device, stream), grown on demand.  Growing frees the old
-// buffer after synchronising the stream that used it.
+// The split-row workspace of (device, stream), grown stream-ordered on that stream
+// (cudaFreeAsync of the old buffer, cudaMallocAsync of the new one: the kernels
+// that used the old buffer were launched on the same stream, so nothing waits on
+// the host).  Never allocates inside a stream capture: the caller's first call of a
+// split-row shape on a stream comes before capturing.  At most kMaxWorkspaces
+// streams per device keep one; a further stream evicts the least recently used
+// entry with cudaFree, which waits for the device.
 int workspace(int dev, void* stream, size_t bytes, void** out) {
-  for (auto& w : g_ws) {
-    if (w.dev == dev && w.stream == stream) {
-      if (w.bytes >= bytes) {
-        *out = w.ptr;
-        return DSEL_OK;
-      }
-      if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSEL_ERR_CUDA;
-      cudaFree(w.ptr);
-      w.ptr = nullptr;
-      w.bytes = 0;
-      if (cudaMalloc(&w.ptr, bytes) != cudaSuccess) return DSEL_ERR_WORKSPACE;
-      w.bytes = bytes;
-      *out = w.ptr;
-      return DSEL_OK;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  Workspace* w = nullptr;
+  int on_dev = 0;
+  Workspace* lru = nullptr;
+  for (auto& e : g_ws) {
+    if (e.dev != dev) continue;
+    ++on_dev;
+    if (e.stream == stream) w = &e;
+    if (lru == nullptr || e.used < lru->used) lru = &e;
+  }
+  if (w != nullptr && w->bytes >= bytes) {
+    w->used = ++g_ws_clock;
+    *out = w->ptr;
+    return DSEL_OK;
+  }
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(cs, &cap) != cudaSuccess) return DSEL_ERR_CUDA;
+  if (cap != cudaStreamCaptureStatusNone) return DSEL_ERR_WORKSPACE;
+  if (w != nullptr) {   // grow in stream order
+    if (cudaFreeAsync(w->ptr, cs) != cudaSuccess) return DSEL_ERR_CUDA;
+    w->ptr = nullptr;
+    w->bytes = 0;
+    if (cudaMallocAsync(&w->ptr, bytes, cs) != cudaSuccess) {
+      w->ptr = nullptr;
+      return DSEL_ERR_WORKSPACE;
     }
+    w->bytes = bytes;
+    w->used = ++g_ws_clock;
+    *out = w->ptr;
+    return DSEL_OK;
+  }
+  if (on_dev >= kMaxWorkspaces && lru != nullptr) {   // evict: its stream may be gone
+    if (cudaFree(lru->ptr) != cudaSuccess) return DSEL_ERR_CUDA;
+    *lru = g_ws.back();
+    g_ws.pop_back();
   }
   void* p = nullptr;
-  if (cudaMalloc(&p, bytes) != cudaSuccess) return DSEL_ERR_WORKSPACE;
-  g_ws.push_back({dev, stream, p, bytes});
+  if (cudaMallocAsync(&p, bytes, cs) != cudaSuccess) return DSEL_ERR_WORKSPACE;
+  g_ws.push_back({dev, stream, p, bytes, ++g_ws_clock});
   *out = p;
   return DSEL_OK;
 }
@@ -141,6 +173,67 @@ int run_shape(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStre
 }
 
 template <int DT>
+int run_slice(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
+  auto k1 = topk_slice_kernel<DT, kSliceThreads, false>;
+  auto kc = topk_slice_kernel<DT, kSliceThreads, true>;
+  if (!di->slice_attrs_set[DT]) {
+    if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) != cudaSuccess ||
+        cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) != cudaSuccess ||
+        cudaFuncSetAttribute(kc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+      return DSEL_ERR_CUDA;
+    di->slice_attrs_set[DT] = true;
+  }
+  const SliceLayout sl = slice_layout(pl.stages, pl.capacity, elem_bytes(DT));
+  KParams kp = base;
+  kp.off_tab = sl.tab;
+  kp.off_bars = sl.bars;
+  kp.off_cb = sl.cb;
+  kp.off_ci = sl.ci;
+  kp.off_hist = sl.hist;
+  kp.off_ctl = sl.ctl;
+  kp.vpt_cap = pl.stages;
+  kp.capacity = pl.capacity;
+  // geometry of rows of row_stride elements, so that those launches issue their
+  // copies without computing it
+  kp.sl_full = uint32_t((base.row_stride + pl.cluster - 1) / pl.cluster + 15) / 16u * 16u;
+  kp.nch_full = int((int64_t(kp.sl_full) * elem_bytes(DT) + kSliceChunkBytes - 1) / kSliceChunkBytes);
+  kp.pa_full = chunk_stride(uint32_t(kp.nch_full));
+  kp.seg = pl.capacity / (pl.cluster * (kSliceThreads / 32));
+  const int64_t grid = rows * pl.cluster;
+  if (grid > 0x7FFFFFFF) return DSEL_ERR_ROWS;
+  const cudaError_t e = pl.cluster > 1 ? launch_cluster(kc, unsigned(grid), kSliceThreads, pl.cluster, sl.total, st, kp)
+                                       : launch_cluster(k1, unsigned(grid), kSliceThreads, 1, sl.total, st, kp);
+  return e == cudaSuccess ? DSEL_OK : DSEL_ERR_CUDA;
+}
+
+// Largest cluster the slice kernel may launch with on this device: 16 CTAs when
+// such a cluster of the largest slices can be scheduled, else the portable 8.
+int slice_cluster_limit(DevInfo* di) {
+  if (di->slice_cluster != 0) return di->slice_cluster;
+  auto kc = topk_slice_kernel<DSEL_F32, kSliceThreads, true>;
+  int lim = kMaxCluster;
+  if (cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) == cudaSuccess &&
+      cudaFuncSetAttribute(kc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kSliceMaxCluster, 1, 1);
+    cfg.blockDim = dim3(kSliceThreads, 1, 1);
+    cfg.dynamicSmemBytes = uint32_t(di->smem_optin);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kSliceMaxCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, kc, &cfg) == cudaSuccess && nclusters >= 1) lim = kSliceMaxCluster;
+  }
+  cudaGetLastError();   // a refused query leaves no sticky error
+  di->slice_cluster = lim;
+  return lim;
+}
+
+template <int DT>
 int run_resident(const KParams& base, int64_t rows, cudaStream_t st, DevInfo* di) {
   auto rk = topk_resident_kernel<DT>;
   if (!di->res_attrs_set[DT]) {
@@ -165,6 +258,7 @@ int run_resident(const KParams& base, int64_t rows, cudaStream_t st, DevInfo* di
 template <int DT>
 int run(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
   if (pl.kernel == DSEL_KERNEL_RESIDENT) return run_resident<DT>(base, rows, st, di);
+  if (pl.kernel == DSEL_KERNEL_SLICE) return run_slice<DT>(base, pl, rows, st, di);
   if (pl.threads == kThreadsShort) return run_shape<DT, kThreadsShort>(base, pl, rows, st, di);
   if (pl.threads == kThreadsMid) return run_shape<DT, kThreadsMid>(base, pl, rows, st, di);
   if (pl.threads == kThreads) return run_shape<DT, kThreads>(base, pl, rows, st, di);
@@ -196,7 +290,9 @@ DSEL_API const char* dsel_status_string(int status) {
     case DSEL_ERR_NAN_MODE: return "nan_mode must be DSEL_NAN_TRAP or DSEL_NAN_FLAG";
     case DSEL_ERR_ORDER: return "sorted_index must be 0, 1 or 2 (2, value order, needs float32 input)";
     case DSEL_ERR_DEVICE: return "the current device is not an sm_100 GPU";
-    case DSEL_ERR_WORKSPACE: return "could not allocate the split-row workspace";
+    case DSEL_ERR_WORKSPACE:
+      return "could not allocate the split-row workspace (a stream capture cannot allocate it: make the "
+             "first call of this shape on the stream before capturing)";
     case DSEL_ERR_CUDA: return "a CUDA runtime call failed";
     case DSEL_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
     case DSEL_ERR_UNAVAILABLE: return "not available in this build";
@@ -246,6 +342,13 @@ DSEL_API int dsel_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, i
   return make_plan(dtype, rows, row_stride, k, num_sms, smem_optin, max_cluster, out);
 }
 
+DSEL_API int dsel_plan_for(int dtype, int64_t rows, int64_t row_stride, int32_t k, int sorted_index,
+                           int32_t num_sms, int32_t smem_optin, int32_t max_cluster, dsel_plan_t* out) {
+  if (sorted_index < DSEL_ORDER_NONE || sorted_index > DSEL_ORDER_VALUE) return DSEL_ERR_ORDER;
+  return make_plan_ex(dtype, rows, row_stride, k, num_sms, smem_optin, max_cluster,
+                      sorted_index == DSEL_ORDER_VALUE ? 0 : kSliceMaxCluster, out);
+}
+
 DSEL_API int dsel_topk(const void* x, int dtype, int64_t rows, int64_t row_stride, const int32_t* end,
                        int32_t k, int sorted_index, int return_value, int index_dtype, int nan_mode,
                        void* values_out, void* indices_out, void* stream) {
@@ -269,7 +372,8 @@ DSEL_API int dsel_topk(const void* x, int dtype, int64_t rows, int64_t row_strid
   st = device_info(dev, &di);
   if (st != DSEL_OK) return st;
   dsel_plan_t pl;
-  st = make_plan(dtype, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster, &pl);
+  st = make_plan_ex(dtype, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster,
+                    sorted_index == DSEL_ORDER_VALUE ? 0 : slice_cluster_limit(di), &pl);
   if (st != DSEL_OK) return st;
 
   KParams kp = {};
@@ -318,7 +422,7 @@ DSEL_API int dsel_topk_sample(const void* x, int64_t rows, int64_t row_stride, c
   st = device_info(dev, &di);
   if (st != DSEL_OK) return st;
   dsel_plan_t pl;
-  st = make_plan(DSEL_F32, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster, &pl);
+  st = make_plan_ex(DSEL_F32, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster, 0, &pl);
   if (st != DSEL_OK) return st;
 
   KParams kp = {};
@@ -397,8 +501,17 @@ DSEL_API int dsel_topk_noalloc(const void* x, int dtype, int64_t rows, int64_t r
   DevInfo* di = nullptr;
   st = device_info(dev, &di);
   if (st != DSEL_OK) return st;
+  // Set-up, once per device, with that device current, on the first call whatever
+  // its plan: host code only knows a stand-in for the array's name, so ask the
+  // runtime for its device address.
+  if (g_noalloc_scratch_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, dsel_noalloc_scratch) != cudaSuccess || ptr == nullptr) return DSEL_ERR_CUDA;
+    g_noalloc_scratch_addr[dev] = ptr;
+  }
   dsel_plan_t pl;
-  st = make_plan(dtype, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster, &pl);
+  st = make_plan_ex(dtype, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster,
+                    sorted_index == DSEL_ORDER_VALUE ? 0 : slice_cluster_limit(di), &pl);
   if (st != DSEL_OK) return st;
 
   KParams kp = {};
@@ -420,14 +533,6 @@ DSEL_API int dsel_topk_noalloc(const void* x, int dtype, int64_t rows, int64_t r
   kp.capacity = pl.capacity;
   if (pl.groups > 1) {
     if (pl.workspace_bytes > DSEL_NOALLOC_SCRATCH_BYTES) return DSEL_ERR_SCRATCH_LIMIT;
-    // Set-up, once per device, with that device current: host code only knows a
-    // stand-in for the array's name, so ask the runtime for its device address.
-    if (g_noalloc_scratch_addr[dev] == nullptr) {
-      void* ptr = nullptr;
-      if (cudaGetSymbolAddress(&ptr, dsel_noalloc_scratch) != cudaSuccess || ptr == nullptr)
-        return DSEL_ERR_CUDA;
-      g_noalloc_scratch_addr[dev] = ptr;
-    }
     // Nothing in the scratch has to start at zero: the merge launch reads only the
     // slots the streaming launch of the same call has just written.
     char* ws = static_cast<char*>(g_noalloc_scratch_addr[dev]);

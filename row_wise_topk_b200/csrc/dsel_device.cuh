@@ -31,7 +31,10 @@ namespace cg = cooperative_groups;
 namespace dsel {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // bounded waits: 2 s
-constexpr uint32_t kSuspendHintNs = 20000;          // a waiting warp sleeps (woken at completion)
+#ifndef DSEL_SUSPEND_HINT_NS
+#define DSEL_SUSPEND_HINT_NS 20000
+#endif
+constexpr uint32_t kSuspendHintNs = DSEL_SUSPEND_HINT_NS;   // a waiting warp sleeps (woken at completion); 0: no hint
 constexpr int kDigitBits = 8;
 constexpr int kTieMax = 128;                  // radix select: largest bucket finished by direct ranking
 constexpr int kBins = 1 << kDigitBits;
@@ -220,6 +223,16 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
+  if (kSuspendHintNs == 0u) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0u;
+  }
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
@@ -733,10 +746,12 @@ __device__ __noinline__ void bitonic_sort(typename Elem<DT>::bits_t* cb, uint32_
   const int tid = threadIdx.x;
   int M = 1;
   while (M < m) M <<= 1;
+  // padding: index 0xFFFFFFFF and the all-ones pattern (key 0, below every real key,
+  // a negative NaN included), so it sorts after every real entry in either order
 #pragma unroll 1
   for (int i = m + tid; i < M; i += THREADS) {
     ci[i] = 0xFFFFFFFFu;
-    cb[i] = static_cast<typename Elem<DT>::bits_t>(Elem<DT>::kNegInf);
+    cb[i] = static_cast<typename Elem<DT>::bits_t>(~0u);
   }
   __syncthreads();
 #pragma unroll 1

@@ -30,6 +30,11 @@ struct KParams {
   int32_t capacity;         // candidate-buffer slots
   uint32_t off_bars, off_blk, off_cb, off_ci, off_holes, off_ctl;
   uint32_t off_hist, off_tab;   // row-resident kernel: histograms, scan table
+  int32_t vpt_cap;          // slice kernel: chunks of the largest slice (one mbarrier each)
+  uint32_t sl_full;         // slice kernel, rows of row_stride elements: slice length,
+  int32_t nch_full;         //   its chunks,
+  uint32_t pa_full;         //   the chunk visiting stride (coprime with nch_full),
+  int32_t seg;              //   candidate-list entries per (slice, warp) segment
   // sampling step after TopK (fp32 only; token_out == nullptr: no draw)
   const float* u;           // [rows] the caller's uniforms in [0, 1)
   int64_t* token_out;       // [rows] drawn index, or a negative row code
@@ -116,6 +121,20 @@ __device__ __noinline__ void write_sentinel_row(const KParams& p, int64_t row, i
     if (p.index_i64) static_cast<int64_t*>(p.indices_out)[base + i] = code;
     else static_cast<int32_t*>(p.indices_out)[base + i] = code;
     if (p.return_value) static_cast<bits_t*>(p.values_out)[base + i] = static_cast<bits_t>(Elem<DT>::kQNaN);
+  }
+}
+
+// Slots n..k-1 of a short row: index DSEL_IDX_PAD, value -inf.
+template <int DT, int THREADS>
+__device__ void write_short_pad(const KParams& p, int64_t row, int64_t n) {
+  using bits_t = typename Elem<DT>::bits_t;
+  if (p.indices_out == nullptr) return;
+  const int64_t base = row * p.k;
+#pragma unroll 1
+  for (int64_t i = n + threadIdx.x; i < p.k; i += THREADS) {
+    if (p.index_i64) static_cast<int64_t*>(p.indices_out)[base + i] = DSEL_IDX_PAD;
+    else static_cast<int32_t*>(p.indices_out)[base + i] = DSEL_IDX_PAD;
+    if (p.return_value) static_cast<bits_t*>(p.values_out)[base + i] = static_cast<bits_t>(Elem<DT>::kNegInf);
   }
 }
 
@@ -241,24 +260,36 @@ __device__ __noinline__ void sample_draw(const KParams& p, int64_t row, const ui
   }
 }
 
-// Rows no longer than k: the TopK output (every entry in index order, then
-// padding) and, for a sampling call, the draw among the n entries, which are
+// Rows no longer than k: the TopK output -- every entry, in index order, or in
+// value order for DSEL_ORDER_VALUE (value descending, ties by index; such rows skip
+// the NaN check, and a NaN takes its IEEE totalOrder place, which the
+// order-preserving key gives it: sign clear above +inf, sign set below -inf) --
+// then padding; for a sampling call, the draw among the n entries, which are
 // checked for NaN first (the softmax has no meaning with one).
 template <int DT, int THREADS>
 __device__ __noinline__ void finish_short_row(const KParams& p, int64_t row, int64_t n,
                                               typename Elem<DT>::bits_t* cb, uint32_t* ci, Ctl& ctl) {
-  write_short_row<DT, THREADS>(p, row, n);
-  if (DT != DSEL_F32 || p.token_out == nullptr) return;
-  const uint32_t* xr = static_cast<const uint32_t*>(p.x) + row * p.row_stride;
+  const bool sampling = DT == DSEL_F32 && p.token_out != nullptr;
+  if (p.order != DSEL_ORDER_VALUE && !sampling) {
+    write_short_row<DT, THREADS>(p, row, n);
+    return;
+  }
+  using bits_t = typename Elem<DT>::bits_t;
+  const bits_t* xr = static_cast<const bits_t*>(p.x) + row * p.row_stride;
   bool nan = false;
 #pragma unroll 1
   for (int i = threadIdx.x; i < n; i += THREADS) {
-    const uint32_t bits = xr[i];
-    cb[i] = static_cast<typename Elem<DT>::bits_t>(bits);
+    const bits_t bits = xr[i];
+    cb[i] = bits;
     ci[i] = static_cast<uint32_t>(i);
     nan |= Elem<DT>::is_nan(bits);
   }
-  if (__syncthreads_or(nan)) {   // uniform
+  nan = __syncthreads_or(nan) != 0;   // uniform; also: the entries are in place
+  bitonic_sort<DT, THREADS, true>(cb, ci, static_cast<int>(n));
+  write_rows_out<DT, THREADS>(p, row, 0, static_cast<int>(n), cb, ci);
+  write_short_pad<DT, THREADS>(p, row, n);
+  if (!sampling) return;
+  if (nan) {
     if (!p.nan_flag) nan_trap();   // the pages' default NaN policy
     if (threadIdx.x == 0) {
       p.token_out[row] = DSEL_IDX_NAN;
@@ -266,7 +297,6 @@ __device__ __noinline__ void finish_short_row(const KParams& p, int64_t row, int
     }
     return;
   }
-  bitonic_sort<DT, THREADS, true>(cb, ci, static_cast<int>(n));
   sample_draw<THREADS>(p, row, reinterpret_cast<const uint32_t*>(cb), ci, static_cast<int>(n), ctl);
 }
 

@@ -62,6 +62,11 @@ int64_t shape_smem(const dsel_plan_t& p, int64_t stages, int32_t k, int eb) {
 
 int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t num_sms,
               int32_t smem_optin, int32_t max_cluster, dsel_plan_t* out) {
+  return make_plan_ex(dtype, rows, row_stride, k, num_sms, smem_optin, max_cluster, kSliceMaxCluster, out);
+}
+
+int make_plan_ex(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t num_sms,
+                 int32_t smem_optin, int32_t max_cluster, int32_t slice_cluster, dsel_plan_t* out) {
   int st = check_shape(dtype, rows, row_stride, k);
   if (st != DSEL_OK) return st;
   if (out == nullptr || num_sms < 1 || smem_optin < 48 * 1024 || max_cluster < 1)
@@ -70,6 +75,7 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
   const int eb = elem_bytes(dtype);
   dsel_plan_t p{};
   const bool one_per_row = rows >= num_sms;
+  const bool resident_rows = one_per_row && row_stride * eb <= kResRowBytes;
 
   // Rows that fit in shared memory: the row-resident kernel.
   if (one_per_row && row_stride * eb <= kResRowBytes) {
@@ -86,6 +92,46 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
       p.stages = int(ceil_div(row_stride * eb, int64_t(kResThreads) * kVecBytes));
       p.idx_bits = ceil_log2_u64(uint64_t(row_stride));
       p.smem_bytes = int(rl.total);
+      p.workspace_bytes = 0;
+      *out = p;
+      return DSEL_OK;
+    }
+  }
+  // Rows that fit, a few slices each, in the shared memory of one cluster: the
+  // slice kernel.  The fewest slices that fit, or more while the batch leaves SMs
+  // idle (but no slice under kSliceMinElems); the candidate list takes the rest of
+  // the shared memory and must hold at least 2k + 2048 entries.
+  if (slice_cluster >= 1 && !resident_rows) {
+    auto fits = [&](int64_t c) {
+      const int64_t ch = slice_chunks(row_stride, c, eb);
+      return ch <= kSliceMaxChunks && slice_list_cap(ch, smem_optin, eb) >= 2 * int64_t(k) + 2048;
+    };
+    int64_t cmin = 0;
+    for (int64_t c = 1; c <= slice_cluster; ++c) {
+      if (fits(c)) {
+        cmin = c;
+        break;
+      }
+    }
+    if (cmin > 0) {
+      int64_t c = std::max<int64_t>(1, num_sms / std::max<int64_t>(rows, 1));
+      c = std::min<int64_t>({c, slice_cluster, std::max<int64_t>(1, ceil_div(row_stride, kSliceMinElems))});
+      c = std::max(c, cmin);
+      while (c > cmin && !fits(c)) --c;
+      const int64_t ch = slice_chunks(row_stride, c, eb);
+      const int64_t lcap = slice_list_cap(ch, smem_optin, eb);
+      const SliceLayout sl = slice_layout(ch, lcap, eb);
+      p.kernel = DSEL_KERNEL_SLICE;
+      p.threads = kSliceThreads;
+      p.cluster = int(c);
+      p.groups = 1;
+      p.stages = int(ch);
+      p.block = kSliceChunkBytes / eb;
+      p.round = int(round_up(ceil_div(row_stride, c), 16));
+      p.b2 = 0;
+      p.capacity = int(lcap);
+      p.idx_bits = ceil_log2_u64(uint64_t(row_stride));
+      p.smem_bytes = int(sl.total);
       p.workspace_bytes = 0;
       *out = p;
       return DSEL_OK;

@@ -20,6 +20,16 @@ constexpr int kVecBytes = 16;                 // one 128-bit shared-memory load 
 // 32 KB: 16,384 bf16 or 8,192 f32 elements) in shared memory.
 constexpr int kResThreads = 256;
 constexpr int kResRowBytes = 32 * 1024;
+// Slice-resident kernel: one 1024-thread CTA per slice of a row (at most 8 chunks
+// of 16 KB, one 16-byte vector per thread each: 128 KB), the slices of a row in
+// one thread-block cluster.
+constexpr int kSliceThreads = 1024;
+constexpr int kSliceChunkBytes = kSliceThreads * kVecBytes;
+constexpr int kSliceMaxChunks = 8;
+constexpr int kSliceMaxCluster = 16;          // non-portable cluster size (B200 schedules 16)
+constexpr int kSliceMinElems = 8192;          // smallest slice worth its own CTA
+constexpr int kSliceCtlBytes = 6144;          // its control block
+constexpr int kSliceMaxList = 16384;          // candidate-list entries
 // Vectors each thread screens per round (a warp owns whole blocks): 16 for bf16
 // (a 64K-element round, the whole slice of a 131,072-position row split in two),
 // 8 for f32 (16K elements, so that two rounds fit the ring for double buffering).
@@ -135,6 +145,73 @@ inline ResLayout resident_layout(int64_t row_stride, int32_t k, int eb) {
   return l;
 }
 
+// Slice kernel: the slice (chunks of 8 KB), the 16-bit maxima of the sampled
+// vectors (later the bitmap ranks: 1 KB per chunk either way), one mbarrier per
+// chunk, the candidate list (element bits, row index), three 1024-bin histograms
+// and the control block.
+struct SliceLayout {
+  uint32_t tab, bars, cb, ci, hist, ctl, total;
+};
+
+inline SliceLayout slice_layout(int64_t chunks, int64_t lcap, int eb) {
+  auto up = [](int64_t v, int64_t a) { return (v + a - 1) / a * a; };
+  SliceLayout l{};
+  int64_t off = chunks * kSliceChunkBytes;
+  l.tab = uint32_t(off);
+  off += chunks * kSliceThreads * 2;
+  l.bars = uint32_t(off);
+  off += up(chunks * 8, 16);
+  l.cb = uint32_t(off);
+  off += up(lcap * eb, 16);
+  l.ci = uint32_t(off);
+  off += up(lcap * 4, 16);
+  l.hist = uint32_t(off);
+  off += 3 * 1024 * 4;
+  l.ctl = uint32_t(off);
+  off += kSliceCtlBytes;
+  l.total = uint32_t(off);
+  return l;
+}
+
+#ifdef __CUDACC__
+#define DSEL_HOST_DEVICE __host__ __device__
+#else
+#define DSEL_HOST_DEVICE
+#endif
+
+// Visiting stride of n chunks: about 0.618 n, odd, coprime with n (1 for n <= 2).
+// Host and device: the host computes it for rows of row_stride elements, a
+// kernel for a row that `end` shortens.
+DSEL_HOST_DEVICE inline uint32_t chunk_stride(uint32_t n) {
+  if (n <= 2) return 1u;
+  uint32_t a = (n * 618u + 500u) / 1000u | 1u;
+  for (;; a += 2u) {
+    uint32_t x = a, y = n;
+    while (y) {
+      const uint32_t t = x % y;
+      x = y;
+      y = t;
+    }
+    if (x == 1u) break;
+  }
+  return a % n;
+}
+
+// Chunks of a slice of ceil(row_stride / C) elements (rounded up to 16).
+inline int64_t slice_chunks(int64_t row_stride, int64_t C, int eb) {
+  const int64_t sl = ((row_stride + C - 1) / C + 15) / 16 * 16;
+  const int64_t per = kSliceChunkBytes / eb;
+  return (sl + per - 1) / per;
+}
+
+// Candidate-list entries that fit next to `chunks` chunks in `smem` bytes.
+inline int64_t slice_list_cap(int64_t chunks, int64_t smem, int eb) {
+  const int64_t fixed = slice_layout(chunks, 0, eb).total + 64;
+  int64_t l = (smem - fixed) / (eb + 4);
+  l = l < kSliceMaxList ? l : kSliceMaxList;
+  return l / 32 * 32;
+}
+
 // Merge kernel: candidate arrays, hole list and the control block.
 inline SmemLayout merge_layout(int64_t capacity, int64_t holes, int eb) {
   auto up = [](int64_t v, int64_t a) { return (v + a - 1) / a * a; };
@@ -154,6 +231,12 @@ inline SmemLayout merge_layout(int64_t capacity, int64_t holes, int eb) {
 
 int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t num_sms,
               int32_t smem_optin, int32_t max_cluster, dsel_plan_t* out);
+
+// make_plan with control over the slice kernel: `slice_cluster` is the largest
+// cluster the slice kernel may use (0: never use it, as for value order and the
+// sampling step, which the other kernels serve).
+int make_plan_ex(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t num_sms,
+                 int32_t smem_optin, int32_t max_cluster, int32_t slice_cluster, dsel_plan_t* out);
 
 // Argument checks shared by dsel_topk and dsel_plan (host only).
 int check_shape(int dtype, int64_t rows, int64_t row_stride, int32_t k);

@@ -62,18 +62,20 @@ def compare(w: W.Workload, got_idx, got_val, exp: O.OracleResult, order, rows=No
     ei = exp.indices.astype(np.int64)
     ev = exp.values
     for n, r in enumerate(rows):
-        if exp.status[n] in (O.ROW_SELECTED,) and order != T.DSEL_ORDER_INDEX:
-            if order == T.DSEL_ORDER_NONE:
-                perm = np.argsort(gi[n], kind="stable")
-                gi_r = gi[n][perm]
-                gv_r = None if gv is None else gv[n][perm]
-                ei_r, ev_r = ei[n], None if ev is None else ev[n]
-            else:   # value order: expected sequence from the oracle's set
-                dec = O.decode(ev[n] if ev is not None else w.x[r][ei[n]], w.dtype)
-                perm = np.lexsort((ei[n], -dec))
-                ei_r = ei[n][perm]
-                ev_r = None if ev is None else ev[n][perm]
-                gi_r, gv_r = gi[n], None if gv is None else gv[n]
+        if exp.status[n] == O.ROW_SELECTED and order == T.DSEL_ORDER_NONE:
+            perm = np.argsort(gi[n], kind="stable")
+            gi_r = gi[n][perm]
+            gv_r = None if gv is None else gv[n][perm]
+            ei_r, ev_r = ei[n], None if ev is None else ev[n]
+        elif exp.status[n] in (O.ROW_SELECTED, O.ROW_SHORT) and order == T.DSEL_ORDER_VALUE:
+            # value order: the oracle's entries (a short row's real ones; its padding
+            # stays at the end) put in value order by the oracle's value_order
+            m = int((ei[n] >= 0).sum())
+            bits = ev[n][:m] if ev is not None else w.x[r][ei[n][:m]]
+            perm = np.concatenate([O.value_order(bits, ei[n][:m], w.dtype), np.arange(m, ei.shape[1])])
+            ei_r = ei[n][perm]
+            ev_r = None if ev is None else ev[n][perm]
+            gi_r, gv_r = gi[n], None if gv is None else gv[n]
         else:
             gi_r, gv_r = gi[n], None if gv is None else gv[n]
             ei_r, ev_r = ei[n], None if ev is None else ev[n]

@@ -133,7 +133,29 @@ def test_plan_invariants(dtype, rows, stride, k):
     assert st == 0
     eb = 2 if dtype == T.DSEL_BF16 else 4
     assert p["smem_bytes"] <= PEAK["smem_optin"]
-    assert p["kernel"] in (T.DSEL_KERNEL_STREAM, T.DSEL_KERNEL_RESIDENT)
+    assert p["kernel"] in (T.DSEL_KERNEL_STREAM, T.DSEL_KERNEL_RESIDENT, T.DSEL_KERNEL_SLICE)
+    if p["kernel"] == T.DSEL_KERNEL_SLICE:
+        # rows cut into `cluster` slices, each held whole in one CTA's shared memory as
+        # chunks of 8 KB (one 16-byte vector per thread), plus a candidate list
+        assert p["threads"] == 1024 and p["groups"] == 1 and 1 <= p["cluster"] <= 16
+        assert p["round"] % 16 == 0 and p["round"] * p["cluster"] >= stride
+        assert p["block"] * eb == 16384 and p["stages"] == -(-p["round"] // p["block"]) <= 8
+        assert p["capacity"] >= 2 * k + 2048 and p["capacity"] % 32 == 0      # candidate list
+        assert p["smem_bytes"] >= p["stages"] * (16384 + 2048) + p["capacity"] * (eb + 4) + 3 * 4096
+        assert p["b2"] == 0 and p["workspace_bytes"] == 0
+        assert (1 << p["idx_bits"]) >= stride
+        # as few slices as fit (8 chunks and a list of 2k + 2048), or more while the
+        # batch leaves SMs idle (but no slice under 8192 elements)
+        def fits(c):
+            sl = (-(-stride // c) + 15) // 16 * 16
+            ch = -(-sl * eb // 16384)
+            fixed = ch * (16384 + 2048) + -(-ch * 8 // 16) * 16 + 3 * 4096 + 6144 + 64
+            lcap = min(16384, (PEAK["smem_optin"] - fixed) // (eb + 4)) // 32 * 32
+            return ch <= 8 and lcap >= 2 * k + 2048
+        assert fits(p["cluster"])
+        assert p["cluster"] == 1 or not fits(p["cluster"] - 1) or \
+            (rows * p["cluster"] <= PEAK["num_sms"] and p["cluster"] <= -(-stride // 8192))
+        return
     if rows >= PEAK["num_sms"] and stride * eb <= 32 * 1024:
         # rows that fit in shared memory: one 256-thread CTA per row holds the whole row
         assert p["kernel"] == T.DSEL_KERNEL_RESIDENT
@@ -182,15 +204,27 @@ def test_plan_splits():
     p = T.dsel_plan(T.DSEL_BF16, 4096, 16384, 512, **PEAK)[1]
     assert p["kernel"] == T.DSEL_KERNEL_RESIDENT and p["threads"] == 256
     p = T.dsel_plan(T.DSEL_BF16, 4096, 16400, 512, **PEAK)[1]
-    assert p["kernel"] == T.DSEL_KERNEL_STREAM and p["cluster"] == 1 and p["threads"] == 128
+    assert p["kernel"] == T.DSEL_KERNEL_SLICE and p["cluster"] == 1 and p["threads"] == 1024
+    # value order never takes the slice kernel
+    p = T.dsel_plan_for(T.DSEL_F32, 256, 129280, 1024, T.DSEL_ORDER_VALUE, **PEAK)[1]
+    assert p["kernel"] == T.DSEL_KERNEL_STREAM and p["threads"] == 256
+    assert T.dsel_plan_for(T.DSEL_F32, 256, 129280, 1024, T.DSEL_ORDER_INDEX, **PEAK)[1] == \
+        T.dsel_plan(T.DSEL_F32, 256, 129280, 1024, **PEAK)[1]
+    assert T.dsel_plan_for(T.DSEL_F32, 4, 8192, 64, 3, **PEAK)[0] == header_define("DSEL_ERR_ORDER")
     # fewer rows than SMs: never resident
-    assert T.dsel_plan(T.DSEL_BF16, 147, 16384, 512, **PEAK)[1]["kernel"] == T.DSEL_KERNEL_STREAM
-    assert T.dsel_plan(T.DSEL_F32, 256, 129280, 4096, **PEAK)[1]["threads"] == 512
+    assert T.dsel_plan(T.DSEL_BF16, 147, 16384, 512, **PEAK)[1]["kernel"] == T.DSEL_KERNEL_SLICE
+    # rows longer than sixteen 160 KB slices: the streaming kernel
+    assert T.dsel_plan(T.DSEL_F32, 256, 1 << 20, 4096, **PEAK)[1]["kernel"] == T.DSEL_KERNEL_STREAM
     # long rows, k <= 1024, at least as many rows as SMs: 256 threads, two CTAs per SM
-    assert T.dsel_plan(T.DSEL_F32, 256, 129280, 1024, **PEAK)[1]["threads"] == 256
-    # 64 indexer rows: two CTAs per row
+    assert T.dsel_plan(T.DSEL_F32, 256, 1 << 20, 1024, **PEAK)[1]["threads"] == 256
+    # 64 indexer rows: two slices per row, each held in one CTA's shared memory
     p = T.dsel_plan(T.DSEL_BF16, 64, 131072, 512, **PEAK)[1]
-    assert (p["kernel"], p["cluster"], p["groups"]) == (T.DSEL_KERNEL_STREAM, 2, 1)
+    assert (p["kernel"], p["cluster"], p["groups"]) == (T.DSEL_KERNEL_SLICE, 2, 1)
+    # one or eight sampler rows: sixteen slices per row; 256 rows: the fewest slices that fit
+    assert T.dsel_plan(T.DSEL_F32, 1, 129280, 50, **PEAK)[1]["cluster"] == 16
+    assert T.dsel_plan(T.DSEL_F32, 8, 129280, 1024, **PEAK)[1]["cluster"] == 16
+    p = T.dsel_plan(T.DSEL_F32, 256, 129280, 1024, **PEAK)[1]
+    assert (p["kernel"], p["cluster"]) == (T.DSEL_KERNEL_SLICE, 4)
     # a single 2^28 row uses several clusters
     p = T.dsel_plan(T.DSEL_F32, 1, 1 << 28, 1000, **PEAK)[1]
     assert p["groups"] > 1 and p["cluster"] == 8

@@ -148,11 +148,11 @@ def test_torch_wrapper_bf16():
 # the workload families at full size (the bench's launch configuration)
 # --------------------------------------------------------------------------- #
 # --------------------------------------------------------------------------- #
-# the 128-thread shape: at least as many rows as SMs, bf16 rows of one or two rounds
+# many rows of 32-64 KB: one slice per row (no cluster), several waves of CTAs
 # --------------------------------------------------------------------------- #
 SHORT = [
-    # (seed, dtype, rows, stride, k, dist, order): bf16 rows above 32 KB (longer ones
-    # are resident in shared memory), at most two 128-thread rounds
+    # (seed, dtype, rows, stride, k, dist, order): bf16 rows above 32 KB (shorter ones
+    # go to the row-resident kernel), each one slice of the slice kernel
     (301, "bf16", 160, 32768, 1, "normal", 1),
     (302, "bf16", 160, 32768, 512, "ties", 0),
     (303, "bf16", 150, 16400, 4096, "normal", 1),
@@ -163,29 +163,36 @@ SHORT = [
 
 
 @pytest.mark.parametrize("seed,dtype,rows,stride,k,dist,order", SHORT)
-def test_short_row_shape(seed, dtype, rows, stride, k, dist, order):
-    st, plan = T.dsel_plan(T.DSEL_BF16 if dtype == "bf16" else T.DSEL_F32, rows, stride, k,
-                           num_sms=torch.cuda.get_device_properties(0).multi_processor_count)
-    assert st == 0 and plan["threads"] == 128, "the case must use the 128-thread shape"
+def test_one_slice_rows(seed, dtype, rows, stride, k, dist, order):
+    st, plan = T.dsel_plan_for(T.DSEL_BF16 if dtype == "bf16" else T.DSEL_F32, rows, stride, k, order,
+                               num_sms=torch.cuda.get_device_properties(0).multi_processor_count)
+    assert st == 0 and plan["kernel"] == T.DSEL_KERNEL_SLICE and plan["cluster"] == 1, \
+        "the case must use one slice per row"
     w = W.random_small(seed, dtype, rows, stride, k, dist=dist, with_end=(seed % 2 == 0),
                        end_lo=0, sorted_index=1, return_value=1, index_dtype="i64")
     check(w, order=order)
 
 
 MID = [
-    # (seed, dtype, rows, stride, k, dist, order): the 256-thread shape, two CTAs per SM
-    (401, "f32", 150, 65536, 1024, "normal", 1),
-    (402, "f32", 160, 40960, 50, "ties", 0),
+    # (seed, dtype, rows, stride, k, dist, order): value order takes the streaming kernel's
+    # 256-thread shape (two CTAs per SM); index order and no order the slice kernel
+    (401, "f32", 150, 65536, 1024, "normal", 2),
+    (402, "f32", 160, 40960, 50, "ties", 2),
     (403, "bf16", 152, 131072, 512, "ascending", 1),
     (404, "f32", 149, 16400, 700, "equal", 2),
+    (405, "f32", 150, 65536, 1024, "normal", 1),
+    (406, "f32", 160, 40960, 50, "ties", 0),
 ]
 
 
 @pytest.mark.parametrize("seed,dtype,rows,stride,k,dist,order", MID)
 def test_mid_row_shape(seed, dtype, rows, stride, k, dist, order):
-    st, plan = T.dsel_plan(T.DSEL_BF16 if dtype == "bf16" else T.DSEL_F32, rows, stride, k,
-                           num_sms=torch.cuda.get_device_properties(0).multi_processor_count)
-    assert st == 0 and plan["threads"] == 256, "the case must use the 256-thread shape"
+    st, plan = T.dsel_plan_for(T.DSEL_BF16 if dtype == "bf16" else T.DSEL_F32, rows, stride, k, order,
+                               num_sms=torch.cuda.get_device_properties(0).multi_processor_count)
+    if order == T.DSEL_ORDER_VALUE:
+        assert st == 0 and plan["threads"] == 256, "the case must use the 256-thread shape"
+    else:
+        assert st == 0 and plan["kernel"] == T.DSEL_KERNEL_SLICE and plan["cluster"] >= 2
     w = W.random_small(seed, dtype, rows, stride, k, dist=dist, with_end=(seed % 2 == 0),
                        end_lo=0, sorted_index=1, return_value=1, index_dtype="i64")
     check(w, order=order)
@@ -240,3 +247,29 @@ def test_long_rows_nan_flag_full(rows, n):
     if clean:
         exp = expected(w, np.array(clean))
         compare(w, gi, None, O.OracleResult(exp.indices, None, exp.status, False), 1, clean)
+
+
+@pytest.mark.parametrize("rows", [6, 160])
+def test_value_order_short_rows(rows):
+    """Rows no longer than k in value order come back sorted by value, like the
+    selected rows (the oracle's value_order), padding last; they skip the NaN check,
+    so a NaN is listed at its totalOrder place.  6 rows: the streaming kernel; 160
+    rows of 256 B: the row-resident kernel."""
+    rng = np.random.default_rng(31)
+    k, stride = 64, 64
+    pool = np.array([-np.inf, -1.5, -0.0, 0.0, 0.25, 0.25, 3.0, np.inf], dtype=np.float32)
+    f = pool[rng.integers(0, len(pool), size=(rows, stride))]
+    bits = f.view(np.uint32).copy()
+    bits[0, 5] = 0x7FC00000      # +NaN: first in value order
+    bits[1, 9] = 0xFFC00001      # -NaN: last among the real entries
+    end = rng.integers(0, stride + 1, size=rows).astype(np.int32)
+    end[0], end[1] = 40, 64
+    w = W.Workload("short_value_order", "f32", bits, end, k, 2, 1, "i64", nan_mode="flag")
+    st, plan = T.dsel_plan_for(T.DSEL_F32, rows, stride, k, T.DSEL_ORDER_VALUE,
+                               num_sms=torch.cuda.get_device_properties(0).multi_processor_count)
+    assert st == 0 and plan["kernel"] == (T.DSEL_KERNEL_RESIDENT if rows >= 148 else T.DSEL_KERNEL_STREAM)
+    gi, gv = check(w, order=T.DSEL_ORDER_VALUE)
+    assert gi[0, 0] == 5 and gv[0, 0] == 0x7FC00000
+    assert gi[1, 63] == 9 and gv[1, 63] == 0xFFC00001
+    for r in range(rows):
+        assert (gi[r, end[r]:] == T.DSEL_IDX_PAD).all()

@@ -283,3 +283,32 @@ def test_mutant_nan_ignored_is_caught(monkeypatch):
     real_decode = O.decode
     monkeypatch.setattr(O, "decode", lambda b, d: np.nan_to_num(real_decode(b, d)))
     assert nan_flag_failures(O.oracle_topk)
+
+
+# --------------------------------------------------------------------------- #
+# value order (sorted_index = 2) and its reading for short rows with NaN
+# --------------------------------------------------------------------------- #
+def test_value_order_matches_a_stable_library_sort():
+    """NaN-free rows: value descending, ties by index, is numpy's stable sort of -v
+    (a library routine); -0.0 and +0.0 compare equal there too."""
+    rng = np.random.default_rng(21)
+    pool = np.array([-np.inf, -2.0, -0.0, 0.0, 0.5, 3.0, np.inf], dtype=np.float32)
+    for t in range(200):
+        n = int(rng.integers(1, 60))
+        f = pool[rng.integers(0, len(pool), size=n)] if t % 2 else rng.standard_normal(n).astype(np.float32)
+        idx = np.sort(rng.choice(1000, size=n, replace=False))
+        got = O.value_order(f.view(np.uint32), idx, "f32")
+        want = np.argsort(-f.astype(np.float64), kind="stable")
+        assert got.tolist() == want.tolist()
+
+
+def test_value_order_hand_case_with_nan():
+    """A worked case: +NaN payloads rank above +inf (larger payload first), -NaN
+    payloads below -inf (larger payload last), -0.0 == +0.0 tied by index."""
+    f = np.array([1.0, -0.0, 0.0, np.inf, -np.inf, 2.0, 1.0], dtype=np.float32)
+    b = np.concatenate([f.view(np.uint32), np.array([0x7FC00000, 0x7FC00001, 0xFFC00000, 0xFFC00001],
+                                                    dtype=np.uint32)])
+    assert O.value_order(b, np.arange(11), "f32").tolist() == [8, 7, 3, 5, 0, 6, 1, 2, 4, 9, 10]
+    # the index breaks ties, whatever the positions
+    assert O.value_order(b[[6, 0]], np.array([3, 9]), "f32").tolist() == [0, 1]
+    assert O.value_order(b[[6, 0]], np.array([9, 3]), "f32").tolist() == [1, 0]
