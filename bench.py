@@ -39,6 +39,7 @@ KERNEL_SOURCES = ["row_wise_topk_b200/csrc/dsel_device.cuh", "row_wise_topk_b200
                   "row_wise_topk_b200/csrc/dsel_slice.cuh"]
 FALLBACK_HBM_GBS = 6650.0
 SAMPLE_T, SAMPLE_P = 1.0, 0.9      # temperature and top-p of the sample_B_k workloads
+LONG_SPLIT_N = 1 << 28             # the long_split_k row: 2^28 float32 positions (1 GiB)
 
 
 def make_workload(name: str) -> W.Workload:
@@ -54,6 +55,8 @@ def make_workload(name: str) -> W.Workload:
         w = W.sampler_logits(int(b), int(k))
         w.name = "topk_sample_" + w.name + f"_t{SAMPLE_T}_p{SAMPLE_P}"
         return w
+    if name.startswith("long_split"):     # long_split_k: one 2^28 row (the reference arm's view)
+        return W.long_rows(1, LONG_SPLIT_N, int(name.split("_")[2]), "uniform")
     if name.startswith("long"):           # long_1_1000 (1 x 2^28) or long_16_4096 (16 x 2^24)
         _, r, k = name.split("_")
         r = int(r)
@@ -572,8 +575,7 @@ def run_ours(args, w, world, rank, local, pg):
         "data": "synthetic", "config": workload_config(args, w, world),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
-                     "kernel": ("topk_resident_kernel" if plan.get("kernel") == T.DSEL_KERNEL_RESIDENT
-                                else "topk_stream_kernel" + ("+topk_merge_kernel" if launches_per_step > 1 else "")),
+                     "kernel": kernel_name(T, plan, launches_per_step),
                      "launch_ms": round(kern_ms, 5),
                      "launch_ms_isolated": {"mean": round(statistics.mean(per_step_ms), 5),
                                             "median": round(statistics.median(per_step_ms), 5),
@@ -585,6 +587,141 @@ def run_ours(args, w, world, rank, local, pg):
         "clocks": clocks,
         "plan": {k_: plan[k_] for k_ in ("kernel", "threads", "cluster", "groups", "stages", "smem_bytes")},
         "input_copies": n_copies,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def kernel_name(T, plan, launches_per_step):
+    if plan.get("kernel") == T.DSEL_KERNEL_RESIDENT:
+        return "topk_resident_kernel"
+    if plan.get("kernel") == T.DSEL_KERNEL_SLICE:
+        return "topk_slice_kernel"
+    return "topk_stream_kernel" + ("+topk_merge_kernel" if launches_per_step > 1 else "")
+
+
+def run_long_split(args, world, rank, local, pg):
+    """One 2^28-element float32 row split over the ranks (columns), TopK of the whole
+    row through ``sharded.topk_row_split``: a local TopK per shard, one NCCL
+    all-gather of the k candidates per rank, and the final TopK of the stacked
+    candidates, timed end to end per step (strong scaling: the row is fixed, each
+    rank holds 1 / N of it).  Each rank's shard is drawn on the host from its own
+    seeded generator (U[-1, 1], the long-row workload's distribution)."""
+    import torch
+    import row_wise_topk_b200 as T
+    from row_wise_topk_b200 import sharded
+
+    k = int(args.workload.split("_")[2])
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    n = LONG_SPLIT_N
+    if n % (world * 16):
+        raise SystemExit("the long_split row must split into shards of whole 16-element units")
+    shard_len = n // world
+    rng = np.random.default_rng(4 + rank)
+    host = torch.from_numpy(rng.uniform(-1.0, 1.0, size=(1, shard_len)).astype(np.float32)).pin_memory()
+    x = host.to(dev)
+    group = pg.group.WORLD if pg is not None else None
+
+    def step():
+        return sharded.topk_row_split(x, k, shard_len=shard_len, group=group, sorted_index=T.DSEL_ORDER_INDEX,
+                                      return_value=True, index_dtype=torch.int64, nan_mode="trap")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record()
+    step()
+    p1.record()
+    torch.cuda.synchronize(dev)
+    est_ms = max(p0.elapsed_time(p1), 1e-3)
+    steps = int(max(args.steps, -(-args.min_seconds * 1000.0 // est_ms)))
+    steps = int(max_over_ranks(float(steps), pg, dev))
+    sampler = ClockSampler(physical_gpu_index(local))
+    sampler.start()
+    time.sleep(0.3)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.mark("t0")
+    t0.record()
+    for _ in range(steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize(dev)
+    sampler.mark("t1")
+    if pg is not None:
+        pg.barrier()
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), pg, dev)
+    time.sleep(0.2)
+    clocks = sampler.stop()
+
+    # the dominant kernel: this rank's local TopK of its shard, timed alone
+    be = sharded.CudaBackend()
+    reps = max(3, min(50, steps))
+    l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    l0.record()
+    for _ in range(reps):
+        be.local_topk(x, k, "trap")
+    l1.record()
+    torch.cuda.synchronize(dev)
+    local_ms = l0.elapsed_time(l1) / reps
+    plan = T.dsel_plan_for(T.DSEL_F32, 1, shard_len, k, T.DSEL_ORDER_INDEX,
+                           num_sms=torch.cuda.get_device_properties(dev).multi_processor_count)[1]
+    local_launches = 1 + (1 if plan["groups"] > 1 else 0)
+    shard_bytes = shard_len * 4 + k * (4 + 8)
+    peak, peak_kind = hbm_peak()
+    achieved = shard_bytes / (local_ms / 1e3) / 1e9
+
+    # end to end: the shard from pinned host memory, the split TopK, the result to the host
+    host_i = torch.empty((1, k), dtype=torch.int64).pin_memory()
+    host_v = torch.empty((1, k), dtype=torch.float32).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    torch.cuda.synchronize(dev)
+    if pg is not None:
+        pg.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        x.copy_(host, non_blocking=True)
+        v, i = step()
+        host_i.copy_(i, non_blocking=True)
+        host_v.copy_(v, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg, dev) / e2e_steps
+    if rank != 0:
+        return
+    total = n * 4 + k * (4 + 8)   # the row read once, the k (value, index) pairs written
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        wsub = W.long_rows(1, 1 << 24, k, "uniform")
+        gbs1, rps1, nrows1, secs1 = cpu_oracle_throughput(wsub, args.cpu_seconds)
+        cpu = {"value": round(gbs1, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{nrows1} rows of 2^24 float32 (1/16 of the row), U[-1, 1], k = {k} "
+                         f"({secs1:.1f} s, one thread, numpy)"}
+    line = {
+        "metric": METRIC, "value": round(total * steps / (elapsed_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+        "n_gpus": world, "steps": steps, "steps_requested": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(elapsed_ms / steps, 5), "timed_ms": round(elapsed_ms, 3),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": f"long_split_f32_1x{n}_k{k}", "rows": 1, "row_length": n, "k": k,
+                   "shard_len": shard_len, "sorted_index": 1, "return_value": 1, "index_dtype": "i64",
+                   "parallelism": f"row split over {world} rank(s): local TopK, NCCL all-gather, final TopK",
+                   "l2": "the 1 GiB row (1 / N per rank) exceeds L2 at N <= 8"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None, "peak_source": peak_kind,
+                     "kernel": kernel_name(T, plan, local_launches) + " (local shard TopK)",
+                     "launch_ms": round(local_ms / local_launches, 5)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(total / (e2e_ms / 1e3) / 1e9, 3), "unit": "GB/s",
+                "h2d_bytes_per_step": shard_len * 4, "d2h_bytes_per_step": k * (4 + 8),
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": (local_launches + 3) * steps,   # local TopK, stack, final TopK, index take
+        "clocks": clocks,
+        "plan": {k_: plan[k_] for k_ in ("kernel", "threads", "cluster", "groups", "stages", "smem_bytes")},
     }
     print(json.dumps(line), flush=True)
 
@@ -604,7 +741,17 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local, pg = dist_setup(args)
-    w = make_workload(args.workload)
+    if args.impl == "ours" and args.workload.startswith("long_split"):
+        try:
+            run_long_split(args, world, rank, local, pg)
+        finally:
+            if pg is not None:
+                pg.destroy_process_group()
+        return
+    if args.impl == "reference" and rank != 0:
+        w = None   # only rank 0 runs the reference arm
+    else:
+        w = make_workload(args.workload)
     try:
         if args.impl == "reference":
             run_reference(args, w, world, rank)

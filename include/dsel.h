@@ -140,11 +140,12 @@ typedef struct {
                             SMs and rows of at most 32 KB, one 256-thread CTA per row holding the
                             whole row in shared memory (block = the 4 KB bulk-copy chunk,
                             round = row_stride, stages = chunks per row, b2 = 0), or
-                            DSEL_KERNEL_SLICE: rows cut into `cluster` slices of at most 160 KB,
-                            one 512-thread CTA per slice holding it whole in shared memory, the
+                            DSEL_KERNEL_SLICE: rows cut into `cluster` slices of at most 128 KB,
+                            one 256-thread CTA per slice holding it whole in shared memory, the
                             slices of a row in one cluster (round = slice elements, block =
-                            elements per warp block, stages = 16-byte vectors per thread,
-                            b2 = capacity = 0); index order and unspecified order only */
+                            elements per 16 KB bulk-copy chunk, stages = chunks per slice,
+                            capacity = candidate-list entries of each CTA, b2 = 0); index
+                            order and unspecified order only */
 } dsel_plan_t;
 
 #define DSEL_KERNEL_STREAM 0

@@ -23,7 +23,7 @@ struct DevInfo {
   int major = 0;
   bool attrs_set[2][3] = {{false, false, false}, {false, false, false}};   // [dtype][shape]
   bool res_attrs_set[2] = {false, false};                                  // [dtype], resident kernel
-  bool slice_attrs_set[2] = {false, false};                                // [dtype], slice kernel
+  bool slice_attrs_set[4] = {false, false, false, false};                  // [dtype][shape], slice kernel
   int slice_cluster = 0;   // largest cluster the slice kernel launches with (16 when schedulable, else 8)
 };
 
@@ -172,16 +172,17 @@ int run_shape(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStre
   return DSEL_OK;
 }
 
-template <int DT>
-int run_slice(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
-  auto k1 = topk_slice_kernel<DT, kSliceThreads, false>;
-  auto kc = topk_slice_kernel<DT, kSliceThreads, true>;
-  if (!di->slice_attrs_set[DT]) {
+template <int DT, int THREADS>
+int run_slice_shape(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
+  auto k1 = topk_slice_kernel<DT, THREADS, false>;
+  auto kc = topk_slice_kernel<DT, THREADS, true>;
+  const int slot = DT * 2 + (THREADS == kSliceThreadsLarge ? 1 : 0);
+  if (!di->slice_attrs_set[slot]) {
     if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) != cudaSuccess ||
         cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) != cudaSuccess ||
         cudaFuncSetAttribute(kc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
       return DSEL_ERR_CUDA;
-    di->slice_attrs_set[DT] = true;
+    di->slice_attrs_set[slot] = true;
   }
   const SliceLayout sl = slice_layout(pl.stages, pl.capacity, elem_bytes(DT));
   KParams kp = base;
@@ -189,6 +190,7 @@ int run_slice(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStre
   kp.off_bars = sl.bars;
   kp.off_cb = sl.cb;
   kp.off_ci = sl.ci;
+  kp.off_cv = sl.cv;
   kp.off_hist = sl.hist;
   kp.off_ctl = sl.ctl;
   kp.vpt_cap = pl.stages;
@@ -198,25 +200,32 @@ int run_slice(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStre
   kp.sl_full = uint32_t((base.row_stride + pl.cluster - 1) / pl.cluster + 15) / 16u * 16u;
   kp.nch_full = int((int64_t(kp.sl_full) * elem_bytes(DT) + kSliceChunkBytes - 1) / kSliceChunkBytes);
   kp.pa_full = chunk_stride(uint32_t(kp.nch_full));
-  kp.seg = pl.capacity / (pl.cluster * (kSliceThreads / 32));
+  kp.seg = pl.capacity / (THREADS / 32);   // each CTA's list, one segment per warp
   const int64_t grid = rows * pl.cluster;
   if (grid > 0x7FFFFFFF) return DSEL_ERR_ROWS;
-  const cudaError_t e = pl.cluster > 1 ? launch_cluster(kc, unsigned(grid), kSliceThreads, pl.cluster, sl.total, st, kp)
-                                       : launch_cluster(k1, unsigned(grid), kSliceThreads, 1, sl.total, st, kp);
+  const cudaError_t e = pl.cluster > 1 ? launch_cluster(kc, unsigned(grid), THREADS, pl.cluster, sl.total, st, kp)
+                                       : launch_cluster(k1, unsigned(grid), THREADS, 1, sl.total, st, kp);
   return e == cudaSuccess ? DSEL_OK : DSEL_ERR_CUDA;
+}
+
+template <int DT>
+int run_slice(const KParams& base, const dsel_plan_t& pl, int64_t rows, cudaStream_t st, DevInfo* di) {
+  if (pl.threads == kSliceThreadsLarge) return run_slice_shape<DT, kSliceThreadsLarge>(base, pl, rows, st, di);
+  if (pl.threads == kSliceThreadsSmall) return run_slice_shape<DT, kSliceThreadsSmall>(base, pl, rows, st, di);
+  return DSEL_ERR_DEVICE;
 }
 
 // Largest cluster the slice kernel may launch with on this device: 16 CTAs when
 // such a cluster of the largest slices can be scheduled, else the portable 8.
 int slice_cluster_limit(DevInfo* di) {
   if (di->slice_cluster != 0) return di->slice_cluster;
-  auto kc = topk_slice_kernel<DSEL_F32, kSliceThreads, true>;
+  auto kc = topk_slice_kernel<DSEL_F32, kSliceThreadsLarge, true>;
   int lim = kMaxCluster;
   if (cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) == cudaSuccess &&
       cudaFuncSetAttribute(kc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kSliceMaxCluster, 1, 1);
-    cfg.blockDim = dim3(kSliceThreads, 1, 1);
+    cfg.blockDim = dim3(kSliceThreadsLarge, 1, 1);
     cfg.dynamicSmemBytes = uint32_t(di->smem_optin);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;

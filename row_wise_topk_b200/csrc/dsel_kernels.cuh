@@ -30,6 +30,7 @@ struct KParams {
   int32_t capacity;         // candidate-buffer slots
   uint32_t off_bars, off_blk, off_cb, off_ci, off_holes, off_ctl;
   uint32_t off_hist, off_tab;   // row-resident kernel: histograms, scan table
+  uint32_t off_cv;              // slice kernel: candidate-vector list
   int32_t vpt_cap;          // slice kernel: chunks of the largest slice (one mbarrier each)
   uint32_t sl_full;         // slice kernel, rows of row_stride elements: slice length,
   int32_t nch_full;         //   its chunks,

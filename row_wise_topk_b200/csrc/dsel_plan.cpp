@@ -113,7 +113,10 @@ int make_plan_ex(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t
         break;
       }
     }
-    if (cmin > 0) {
+    // one wave only: a CTA holds its SM from the first copy to the last write, so
+    // batches needing several waves of slices go to the streaming kernel, whose
+    // two CTAs per SM overlap one row's tail with the next row's loads
+    if (cmin > 0 && rows * cmin <= num_sms) {
       int64_t c = std::max<int64_t>(1, num_sms / std::max<int64_t>(rows, 1));
       c = std::min<int64_t>({c, slice_cluster, std::max<int64_t>(1, ceil_div(row_stride, kSliceMinElems))});
       c = std::max(c, cmin);
@@ -122,7 +125,7 @@ int make_plan_ex(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t
       const int64_t lcap = slice_list_cap(ch, smem_optin, eb);
       const SliceLayout sl = slice_layout(ch, lcap, eb);
       p.kernel = DSEL_KERNEL_SLICE;
-      p.threads = kSliceThreads;
+      p.threads = slice_threads(ch);
       p.cluster = int(c);
       p.groups = 1;
       p.stages = int(ch);

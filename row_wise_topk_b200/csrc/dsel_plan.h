@@ -20,15 +20,23 @@ constexpr int kVecBytes = 16;                 // one 128-bit shared-memory load 
 // 32 KB: 16,384 bf16 or 8,192 f32 elements) in shared memory.
 constexpr int kResThreads = 256;
 constexpr int kResRowBytes = 32 * 1024;
-// Slice-resident kernel: one 1024-thread CTA per slice of a row (at most 8 chunks
-// of 16 KB, one 16-byte vector per thread each: 128 KB), the slices of a row in
-// one thread-block cluster.
-constexpr int kSliceThreads = 1024;
-constexpr int kSliceChunkBytes = kSliceThreads * kVecBytes;
+// Slice-resident kernel: one CTA per slice of a row (at most 8 chunks of 16 KB:
+// 128 KB), the slices of a row in one thread-block cluster.  512 threads (two
+// 16-byte vectors per thread and chunk) for slices of four chunks or more, whose
+// per-vector passes need the warps to hide their latency; 256 threads (four
+// vectors per thread and chunk) for smaller slices, where the fixed per-CTA work
+// dominates.
+constexpr int kSliceThreadsLarge = 512;
+constexpr int kSliceThreadsSmall = 256;
+constexpr int kSliceLargeFromChunks = 4;
+constexpr int slice_threads(int64_t chunks) {
+  return chunks >= kSliceLargeFromChunks ? kSliceThreadsLarge : kSliceThreadsSmall;
+}
+constexpr int kSliceChunkBytes = 16384;
 constexpr int kSliceMaxChunks = 8;
 constexpr int kSliceMaxCluster = 16;          // non-portable cluster size (B200 schedules 16)
 constexpr int kSliceMinElems = 8192;          // smallest slice worth its own CTA
-constexpr int kSliceCtlBytes = 6144;          // its control block
+constexpr int kSliceCtlBytes = 1024;          // its control block
 constexpr int kSliceMaxList = 16384;          // candidate-list entries
 // Vectors each thread screens per round (a warp owns whole blocks): 16 for bf16
 // (a 64K-element round, the whole slice of a 131,072-position row split in two),
@@ -145,12 +153,13 @@ inline ResLayout resident_layout(int64_t row_stride, int32_t k, int eb) {
   return l;
 }
 
-// Slice kernel: the slice (chunks of 8 KB), the 16-bit maxima of the sampled
-// vectors (later the bitmap ranks: 1 KB per chunk either way), one mbarrier per
-// chunk, the candidate list (element bits, row index), three 1024-bin histograms
-// and the control block.
+// Slice kernel: the slice (chunks of 16 KB), the 16-bit maxima of its vectors
+// (later the bitmap ranks: 2 KB per chunk either way), one mbarrier per chunk, the
+// CTA's candidate lists (elements: bits and row index; vectors: half as many
+// indices), a 4096-bin histogram of the vector maxima and a 1024-bin one of the
+// candidates, and the control block.
 struct SliceLayout {
-  uint32_t tab, bars, cb, ci, hist, ctl, total;
+  uint32_t tab, bars, cb, ci, cv, hist, ctl, total;
 };
 
 inline SliceLayout slice_layout(int64_t chunks, int64_t lcap, int eb) {
@@ -158,15 +167,17 @@ inline SliceLayout slice_layout(int64_t chunks, int64_t lcap, int eb) {
   SliceLayout l{};
   int64_t off = chunks * kSliceChunkBytes;
   l.tab = uint32_t(off);
-  off += chunks * kSliceThreads * 2;
+  off += chunks * (kSliceChunkBytes / kVecBytes) * 2;   // a 16-bit summary per vector
   l.bars = uint32_t(off);
   off += up(chunks * 8, 16);
   l.cb = uint32_t(off);
   off += up(lcap * eb, 16);
   l.ci = uint32_t(off);
   off += up(lcap * 4, 16);
+  l.cv = uint32_t(off);   // candidate vectors: half as many entries as the element list
+  off += up(lcap / 2 * 4, 16);
   l.hist = uint32_t(off);
-  off += 3 * 1024 * 4;
+  off += (4096 + 1024 + 512) * 4;   // and their coarse sums
   l.ctl = uint32_t(off);
   off += kSliceCtlBytes;
   l.total = uint32_t(off);
@@ -207,7 +218,7 @@ inline int64_t slice_chunks(int64_t row_stride, int64_t C, int eb) {
 // Candidate-list entries that fit next to `chunks` chunks in `smem` bytes.
 inline int64_t slice_list_cap(int64_t chunks, int64_t smem, int eb) {
   const int64_t fixed = slice_layout(chunks, 0, eb).total + 64;
-  int64_t l = (smem - fixed) / (eb + 4);
+  int64_t l = (smem - fixed) / (eb + 4 + 2);
   l = l < kSliceMaxList ? l : kSliceMaxList;
   return l / 32 * 32;
 }

@@ -1,36 +1,36 @@
 // Slice-resident TopK: the rows of a batch are cut into slices that fit in shared
 // memory, one CTA per slice, and the slices of one row form a thread-block
-// cluster whose rank-0 CTA leads.  Every CTA loads its whole slice with bulk
-// copies (all in flight at once), so the row is read exactly once.  The method is
-// the threshold filter of "DeepSeek releases DeepSelect, a TopK kernel for sparse
-// attention and sampling" (method paragraph), laid out for the order in which the
-// data lands:
+// cluster.  Every CTA loads its whole slice with bulk copies (all in flight at
+// once), so the row is read exactly once.  The method is the threshold filter of
+// "DeepSeek releases DeepSelect, a TopK kernel for sparse attention and sampling"
+// (method paragraph), laid out for the order in which the data lands:
 //
 //   A. threshold from a sample: the chunks are visited in a per-slice
-//      pseudo-random order, and the first ns to arrive are a random sample of the
+//      pseudo-random order, and the first ns of them are a random sample of the
 //      slice.  Either every CTA takes T_c, a lower edge of the k-th largest vector
 //      maximum of its own sample (k vectors hold an element >= T_c: a valid
-//      threshold for the whole row, found with no cluster barrier), or, when that
-//      would let too many candidates through, the CTAs take the k'-th largest,
-//      k' = ceil(k / C), and the cluster uses T = min_c T_c (C slices with k'
-//      such vectors each: again at least k), one cluster barrier;
-//   B. filter: every chunk, as it lands, is screened against T (one packed
-//      compare per 16-byte vector); the survivors go straight into the leader's
-//      candidate list through distributed shared memory;
-//   C. exact finish, by the leader alone after one cluster barrier (the other
-//      CTAs leave): histogram levels over the candidates' keys and a ranking of the
-//      boundary bin's members by (key, index) give the composite boundary (K*, I*),
-//      the k-th entry of the row in the order value descending, index ascending.
-//      An entry is selected when (key, index) ranks at or before (K*, I*); index
-//      order comes from a bitmap of the row.
+//      threshold for the whole row) and the cluster keeps the largest, or, when
+//      that would need too large a sample, the CTAs take the k'-th largest,
+//      k' = ceil(k / C), and the cluster keeps the smallest (C slices with k'
+//      such vectors each: again at least k).  One cluster barrier;
+//   B. filter: every vector is screened against T with packed compares (about
+//      ten instructions per 16-byte vector); the survivors go into the CTA's own
+//      candidate list, one segment per warp, and into a histogram of their keys;
+//   C. exact finish, shared by the cluster: the CTAs sum their histograms through
+//      distributed shared memory and refine the bin that holds the k-th entry
+//      (one cluster barrier per extra level) down to the boundary key K*, or to a
+//      bin that is selected whole.  Each CTA then counts its entries above K* and
+//      equal to it; after one more barrier every CTA knows how many entries each
+//      slice contributes, so it ranks its own selection in index order from a
+//      bitmap of its slice and writes it at its offset.  The entries equal to K*
+//      are taken in index order across the slices (the composite (value, index)
+//      order: value descending, lower index first among equals).
 //
-// When the list overflows an exact fallback runs on the resident slices (every
-// CTA): histogram levels down to a single key, then ranks in index order from
-// bitmaps.  The code runs once per launch, so every instruction it executes is
-// fetched cold: loops stay rolled, and bin searches run in one warp (the others
-// wait at a barrier) instead of every warp reading the whole histogram.  No wait
-// depends on another CTA except the hardware cluster barriers; the bulk-copy
-// waits are bounded.
+// When a candidate list overflows an exact fallback runs on the resident slices
+// (every CTA): histogram levels down to a single key, then ranks in index order
+// from bitmaps.  No wait depends on another CTA except the hardware cluster
+// barriers; the bulk-copy waits are bounded.  A CTA that has read a peer's shared
+// memory arrives at a last cluster barrier before it leaves.
 #pragma once
 
 #include "dsel_resident.cuh"
@@ -38,38 +38,54 @@
 namespace dsel {
 
 constexpr int kSlBins = 1024;
-constexpr int kSlMembers = 256;   // boundary members ranked directly
-constexpr int kSlChunk = kSliceThreads * kVecBytes;   // bytes per chunk: one vector per thread
+constexpr int kSlVBins = 4096;   // vector-maximum histogram: fixed bins of 16 key summaries
+constexpr int kSlChunk = kSliceChunkBytes;                   // bytes per chunk
+constexpr int kSlChunkVecs = kSliceChunkBytes / kVecBytes;   // 16-byte vectors per chunk
 
 struct __align__(16) SliceCtl {
   uint32_t w_a[kWarpsMax];
   uint32_t w_b[kWarpsMax];
   int w_c[kWarpsMax];
   int bin, before, cnt;      // a bin search, broadcast to the CTA
-  uint32_t t_key;            // this slice's threshold, broadcast to the CTA
-  int m_n;                   // boundary members collected in m_w
-  uint32_t kstar, istar;
+  int bin2, before2, cnt2;   // the fine stage of a two-stage search
+  // published to the cluster: the peers read these after a cluster barrier
   int flags;                 // bit 0: NaN seen, bit 1: list overflow, bit 2: a wait gave up
-  // the leader's copy is updated by every CTA of the cluster (remote atomics)
-  uint32_t t_max;            // largest slice threshold (each one valid alone)
-  uint32_t t_min;            // smallest slice threshold (each valid for k / C)
-  uint32_t top;              // largest sampled key
-  uint32_t kmax;             // largest key of the row
-  // read by the peers in the exact fallback
-  int x_sel;
-  int x_cnt;
-  uint32_t x_istar;
-  int segcnt[kSliceMaxCluster * (kSliceThreads / 32)];   // entries of each (slice, warp) list segment
-  unsigned long long m_w[kSlMembers];   // boundary members (key << 32 | ~index)
+  uint32_t kmax;             // largest key of this slice
+  int x_a;                   // entries selected above the boundary key
+  int x_t;                   // entries equal to the boundary key
+  int x_sel, x_cnt;          // exact fallback: selected / tied entries of this slice
+  uint32_t x_istar;          // the last selected tie (row index)
+  int n_list;                // entries in this CTA's candidate list
+#ifdef DSEL_STATS
+  unsigned long long marks[32];   // phase timestamps, written out when the CTA ends
+#endif
 };
 
-// Phase timestamps of thread 0 (%globaltimer, ns) in counter builds only:
-// g_stats[cta][i] for i = 0..15.
-__device__ __forceinline__ void sl_mark(int i) {
+// Phase timestamps of thread 0 (%globaltimer, ns) in counter builds only, kept
+// in shared memory (a global store before a cluster barrier would make the
+// barrier's release wait for it) and written to g_stats[cta][i] when the CTA ends.
+__device__ __forceinline__ void sl_mark(SliceCtl& ctl, int i) {
 #ifdef DSEL_STATS
-  if (threadIdx.x == 0 && blockIdx.x < kStatsCtas) g_stats[blockIdx.x * kStatsFields + i] = global_ns();
+  if (threadIdx.x == 0) ctl.marks[i] = global_ns();
 #else
+  (void)ctl;
   (void)i;
+#endif
+}
+
+__device__ __forceinline__ void sl_marks_out(SliceCtl& ctl) {
+#ifdef DSEL_STATS
+  if (threadIdx.x == 0 && blockIdx.x < kStatsCtas) {
+    ctl.marks[11] = global_ns();
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i) g_stats[blockIdx.x * kStatsFields + i] = ctl.marks[i];
+    if (blockIdx.x < kStatsCtas / 2) {   // per-chunk times in the upper half
+#pragma unroll 1
+      for (int i = 0; i < 16; ++i) g_stats[(kStatsCtas / 2 + blockIdx.x) * kStatsFields + i] = ctl.marks[16 + i];
+    }
+  }
+#else
+  (void)ctl;
 #endif
 }
 
@@ -79,8 +95,8 @@ __device__ __forceinline__ void sl_sync(cg::cluster_group& cluster) {
   else __syncthreads();
 }
 
-// Split cluster barrier: arrive (release) early, wait (acquire) only where the
-// ordering is needed.
+// Split cluster barrier: arrive (release) once this CTA is done reading its
+// peers' shared memory, wait (acquire) just before it leaves.
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
@@ -125,6 +141,162 @@ __device__ __forceinline__ void cluster_hist_sum(const int* h, int* hs, int C, c
   __syncthreads();
 }
 
+// NB consecutive ints of shared memory at p (16-, 8- or 4-byte loads).
+template <int NB>
+__device__ __forceinline__ void load_run(const int* p, int (&c)[NB]) {
+  if constexpr (NB % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < NB / 4; ++i) {
+      const int4 v = reinterpret_cast<const int4*>(p)[i];
+      c[4 * i] = v.x;
+      c[4 * i + 1] = v.y;
+      c[4 * i + 2] = v.z;
+      c[4 * i + 3] = v.w;
+    }
+  } else if constexpr (NB == 2) {
+    const int2 v = *reinterpret_cast<const int2*>(p);
+    c[0] = v.x;
+    c[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < NB; ++i) c[i] = p[i];
+  }
+}
+
+// This thread's run of NB consecutive bins of a histogram (bins NB t .. NB t +
+// NB - 1), summed over the cluster's CTAs: the caller has passed a cluster
+// barrier after the histograms were complete.
+template <bool CLUSTER, int NB>
+__device__ __forceinline__ void hist_sum_run(const int* h, int (&c)[NB], int C, cg::cluster_group& cluster) {
+  const int* hp = h + threadIdx.x * NB;
+  load_run<NB>(hp, c);
+  if (CLUSTER) {
+#pragma unroll 1
+    for (int r = 1; r < C; ++r) {
+      int v[NB];
+      load_run<NB>(cluster.map_shared_rank(hp, (static_cast<int>(cluster.block_rank()) + r) % C), v);
+#pragma unroll
+      for (int i = 0; i < NB; ++i) c[i] += v[i];
+    }
+  }
+}
+
+// Bin of the need-th largest entry of a histogram held as consecutive runs of NB
+// bins per thread (bin 0 the largest keys): a CTA-wide scan, two CTA barriers.
+// bin = -1 when the histogram holds fewer than `need` entries.
+template <int THREADS, int NB>
+__device__ __forceinline__ BinHit cta_find_bin(const int (&c)[NB], int need, SliceCtl& ctl) {
+  constexpr int NW = THREADS / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int s = 0;
+#pragma unroll
+  for (int i = 0; i < NB; ++i) s += c[i];
+  const int incl = warp_incl_scan(s, lane);
+  if (lane == 31) ctl.w_c[warp] = incl;
+  __syncthreads();
+  int total;
+  const int base = warp_prefix_of<NW>(ctl.w_c, warp, lane, total) + incl - s;
+  BinHit r;
+  if (total < need) {   // uniform in the CTA
+    __syncthreads();
+    r.bin = -1;
+    r.before = 0;
+    r.cnt = 0;
+    return r;
+  }
+  if (base < need && need <= base + s) {   // exactly one thread
+    int found = -1, before = base, cnt = 0;
+#pragma unroll
+    for (int i = 0; i < NB; ++i) {
+      if (found < 0) {
+        if (before + c[i] >= need) {
+          found = i;
+          cnt = c[i];
+        } else {
+          before += c[i];
+        }
+      }
+    }
+    ctl.bin = NB * tid + found;
+    ctl.before = before;
+    ctl.cnt = cnt;
+  }
+  __syncthreads();
+  r.bin = ctl.bin;
+  r.before = ctl.before;
+  r.cnt = ctl.cnt;
+  return r;
+}
+
+// Coarse sums of a histogram kept beside it for the two-stage search:
+// coarse[i] = fine[16 i] + ... + fine[16 i + 15], i < ncb.  The caller has made
+// the fine histogram complete with a CTA barrier, and publishes both with a
+// cluster barrier.
+template <int THREADS>
+__device__ __forceinline__ void coarse_sums(const int* fine, int* coarse, int ncb) {
+#pragma unroll 1
+  for (int i = threadIdx.x; i < ncb; i += THREADS) {
+    const int4* f4 = reinterpret_cast<const int4*>(fine + 16 * i);
+    int sum = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int4 v = f4[q];
+      sum += v.x + v.y + v.z + v.w;
+    }
+    coarse[i] = sum;
+  }
+}
+
+// Element i of an int array summed over the cluster's CTAs, four loads in flight.
+template <bool CLUSTER>
+__device__ __forceinline__ int cluster_sum_at(const int* a, int i, int C, cg::cluster_group& cluster) {
+  if (!CLUSTER) return a[i];
+  const int me = static_cast<int>(cluster.block_rank());
+  int sum = 0;
+#pragma unroll 1
+  for (int r0 = 0; r0 < C; r0 += 4) {
+    int v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int r = r0 + q;
+      v[q] = r < C ? cluster.map_shared_rank(a, r + me < C ? r + me : r + me - C)[i] : 0;
+    }
+    sum += v[0] + v[1] + v[2] + v[3];
+  }
+  return sum;
+}
+
+// Bin of the need-th largest entry of a histogram of 16 * ncb bins (bin 0 the
+// largest keys), summed over the cluster, in two stages: the coarse sums (ncb <=
+// THREADS bins of 16) locate the coarse bin, whose 16 fine bins then locate the
+// bin.  The caller has passed a cluster barrier after publishing both arrays.
+// Four CTA barriers; bin = -1 when the histogram holds fewer than `need` entries.
+template <int THREADS, bool CLUSTER>
+__device__ __forceinline__ BinHit cluster_find_bin(const int* fine, const int* coarse, int ncb, int need, int C,
+                                                   SliceCtl& ctl, cg::cluster_group& cluster) {
+  const int tid = threadIdx.x;
+  int c[1] = {tid < ncb ? cluster_sum_at<CLUSTER>(coarse, tid, C, cluster) : 0};
+  const BinHit cb = cta_find_bin<THREADS, 1>(c, need, ctl);
+  if (cb.bin < 0) return cb;   // uniform in the CTA
+  const int need2 = need - cb.before;
+  if (tid < 32) {   // one warp: the coarse bin's 16 fine bins
+    const int f = tid < 16 ? cluster_sum_at<CLUSTER>(fine, 16 * cb.bin + tid, C, cluster) : 0;
+    const int incl = warp_incl_scan(f, tid);
+    const int j = __ffs(__ballot_sync(0xffffffffu, tid < 16 && incl >= need2)) - 1;
+    if (tid == j) {
+      ctl.bin2 = 16 * cb.bin + j;
+      ctl.before2 = cb.before + incl - f;
+      ctl.cnt2 = f;
+    }
+  }
+  __syncthreads();
+  BinHit r;
+  r.bin = ctl.bin2;
+  r.before = ctl.before2;
+  r.cnt = ctl.cnt2;
+  return r;
+}
+
 // Exclusive prefix over the cluster's slices of a per-slice count published in
 // ctl.x_*: the caller has passed a cluster barrier after publishing it.
 __device__ __forceinline__ int slices_before(const SliceCtl& ctl, const int SliceCtl::*field, int crank,
@@ -163,44 +335,6 @@ __device__ __forceinline__ int bitmap_rank(const uint32_t* bm, const uint32_t* p
   return static_cast<int>(pre[i >> 5]) + __popc(bm[i >> 5] & ((1u << (i & 31u)) - 1u));
 }
 
-// Bitmap rank over a whole row with a coarse prefix: bp[b] = set bits in the
-// blocks of 32 words before block b.  After the bits are set and a CTA barrier;
-// two CTA barriers.  Returns the total.
-template <int THREADS>
-__device__ __noinline__ int row_bitmap_prefix(const uint32_t* bm, int* bp, int words, SliceCtl& ctl) {
-  constexpr int NW = THREADS / 32;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int blocks = (words + 31) / 32;
-#pragma unroll 1
-  for (int b = warp; b < blocks; b += NW) {   // one warp per block: its total
-    const int w = b * 32 + lane;
-    const int c = static_cast<int>(__reduce_add_sync(0xffffffffu, w < words ? __popc(bm[w]) : 0u));
-    if (lane == 0) bp[b] = c;
-  }
-  __syncthreads();
-  if (warp == 0) {   // exclusive scan of the block totals, 32 blocks at a time
-    int run = 0;
-#pragma unroll 1
-    for (int b0 = 0; b0 < blocks; b0 += 32) {
-      const int b = b0 + lane;
-      const int c = b < blocks ? bp[b] : 0;
-      const int incl = warp_incl_scan(c, lane);
-      if (b < blocks) bp[b] = run + incl - c;
-      run += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) ctl.w_c[0] = run;
-  }
-  __syncthreads();
-  return ctl.w_c[0];
-}
-
-__device__ __forceinline__ int row_bitmap_rank(const uint32_t* bm, const int* bp, uint32_t i) {
-  int r = bp[i >> 10];
-#pragma unroll 1
-  for (uint32_t w = (i >> 10) << 5; w < (i >> 5); ++w) r += __popc(bm[w]);
-  return r + __popc(bm[i >> 5] & ((1u << (i & 31u)) - 1u));
-}
-
 // Everything a CTA of the slice kernel knows about its slice.
 struct SliceGeom {
   int64_t row;
@@ -212,10 +346,19 @@ struct SliceGeom {
 
 // Exact fallback on the resident slice: histogram levels over the keys >= lo_k
 // down to a single key K*, then the ties at K* and the selected entries ranked in
-// index order through bitmaps.  Runs on every CTA of the cluster together.
+// index order through bitmaps.  Runs on every CTA of the cluster together and
+// ends with a cluster barrier.  The slice lies in shared memory as one flat array
+// of 16-byte vectors.
 template <int DT, int THREADS, bool CLUSTER>
-__device__ __noinline__ void slice_exact(const KParams& p, unsigned char* smem, const SliceGeom& g, uint32_t lo_k,
-                                         uint32_t kmax_row, cg::cluster_group& cluster) {
+__device__ __noinline__ void slice_exact(const KParams& p, unsigned char* smem, int64_t row, uint32_t slice_lo,
+                                         uint32_t n_sl, int C, int crank, uint32_t lo_k, uint32_t kmax_row,
+                                         cg::cluster_group& cluster) {
+  SliceGeom g;   // rebuilt from values: a reference argument would keep the caller's copy in local memory
+  g.row = row;
+  g.lo = slice_lo;
+  g.n_sl = n_sl;
+  g.C = C;
+  g.crank = crank;
   using E = Elem<DT>;
   using bits_t = typename E::bits_t;
   constexpr int PV = E::kPerVec;
@@ -225,13 +368,12 @@ __device__ __noinline__ void slice_exact(const KParams& p, unsigned char* smem, 
   uint32_t* bm = reinterpret_cast<uint32_t*>(smem + p.off_tab);   // bitmap, then its prefix
   const int words = static_cast<int>((g.n_sl + 31u) / 32u);
   uint32_t* pre = bm + words;
+  const int nvec = static_cast<int>((g.n_sl + PV - 1u) / PV);
   const int k = p.k;
-  auto load_vec = [&](int c) -> uint4 {
-    return *reinterpret_cast<const uint4*>(smem + static_cast<size_t>(c) * kSlChunk + tid * kVecBytes);
-  };
-  auto valid_of = [&](int c) -> int { return static_cast<int>(g.n_sl) - (c * THREADS + tid) * PV; };
+  auto load_vec = [&](int v) -> uint4 { return *reinterpret_cast<const uint4*>(smem + static_cast<size_t>(v) * kVecBytes); };
+  auto valid_of = [&](int v) -> int { return static_cast<int>(g.n_sl) - v * PV; };
 
-  // the peers may still read this CTA's histograms and list: meet first, then clear
+  // the peers may still read this CTA's control block: meet first, then clear
   sl_sync<CLUSTER>(cluster);
 #pragma unroll 1
   for (int i = tid; i < 3 * kSlBins / 4; i += THREADS) reinterpret_cast<int4*>(hist)[i] = make_int4(0, 0, 0, 0);
@@ -246,11 +388,9 @@ __device__ __noinline__ void slice_exact(const KParams& p, unsigned char* smem, 
     int* h = hist + (level & 1) * kSlBins;
     const int s = res_shift(hi_k - lo_k);
 #pragma unroll 1
-    for (int c = 0; c < g.nch; ++c) {
-      const int valid = valid_of(c);
-      if (valid <= 0) continue;
-      const uint4 x = load_vec(c);
-      uint32_t m = res_mask_ge<DT>(x, lo_k, valid);
+    for (int v = tid; v < nvec; v += THREADS) {
+      const uint4 x = load_vec(v);
+      uint32_t m = res_mask_ge<DT>(x, lo_k, valid_of(v));
 #pragma unroll 1
       while (m != 0u) {
         const int e = __ffs(m) - 1;
@@ -297,13 +437,11 @@ __device__ __noinline__ void slice_exact(const KParams& p, unsigned char* smem, 
     for (int i = tid; i < 2 * words; i += THREADS) bm[i] = 0u;
     __syncthreads();
 #pragma unroll 1
-    for (int c = 0; c < g.nch; ++c) {
-      const int valid = valid_of(c);
-      if (valid <= 0) continue;
+    for (int v = tid; v < nvec; v += THREADS) {
       uint32_t gt;
-      const uint32_t eq = masks(load_vec(c), valid, gt);
+      const uint32_t eq = masks(load_vec(v), valid_of(v), gt);
       if (eq != 0u) {
-        const uint32_t b0 = static_cast<uint32_t>(c * THREADS + tid) * PV;   // PV divides 32: one word
+        const uint32_t b0 = static_cast<uint32_t>(v) * PV;   // PV divides 32: one word
         atomicOr(&bm[b0 >> 5], eq << (b0 & 31u));
       }
     }
@@ -347,12 +485,10 @@ __device__ __noinline__ void slice_exact(const KParams& p, unsigned char* smem, 
   for (int i = tid; i < 2 * words; i += THREADS) bm[i] = 0u;
   __syncthreads();
 #pragma unroll 1
-  for (int c = 0; c < g.nch; ++c) {
-    const int valid = valid_of(c);
-    if (valid <= 0) continue;
+  for (int v = tid; v < nvec; v += THREADS) {
     uint32_t gt;
-    uint32_t eq = masks(load_vec(c), valid, gt);
-    const uint32_t b0 = static_cast<uint32_t>(c * THREADS + tid) * PV;
+    uint32_t eq = masks(load_vec(v), valid_of(v), gt);
+    const uint32_t b0 = static_cast<uint32_t>(v) * PV;
     uint32_t keep = gt;
 #pragma unroll 1
     while (eq != 0u) {
@@ -372,13 +508,11 @@ __device__ __noinline__ void slice_exact(const KParams& p, unsigned char* smem, 
   }
   const int64_t obase = g.row * static_cast<int64_t>(k);
 #pragma unroll 1
-  for (int c = 0; c < g.nch; ++c) {
-    const int valid = valid_of(c);
-    if (valid <= 0) continue;
-    const uint32_t b0 = static_cast<uint32_t>(c * THREADS + tid) * PV;
+  for (int v = tid; v < nvec; v += THREADS) {
+    const uint32_t b0 = static_cast<uint32_t>(v) * PV;
     uint32_t m = (bm[b0 >> 5] >> (b0 & 31u)) & ((1u << PV) - 1u);
     if (m == 0u) continue;
-    const uint4 x = load_vec(c);
+    const uint4 x = load_vec(v);
 #pragma unroll 1
     while (m != 0u) {
       const int e = __ffs(m) - 1;
@@ -392,141 +526,7 @@ __device__ __noinline__ void slice_exact(const KParams& p, unsigned char* smem, 
       }
     }
   }
-  if (CLUSTER) cluster.sync();   // the peers read this CTA's counts above: leave together
-}
-
-// The leader's candidate list: C * NW segments of `seg` entries, segment s
-// (slice s / NW, warp s % NW) holding segcnt[s] entries.  Visits every entry,
-// warp w taking segments w, w + NW, ... and its lanes the entries side by side;
-// f(i, valid) runs in every lane, with the same trip count across the warp.
-template <int THREADS, typename F>
-__device__ __forceinline__ void for_list(const int* segcnt, int nseg, int seg, F&& f) {
-  constexpr int NW = THREADS / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll 1
-  for (int s = warp; s < nseg; s += NW) {
-    const int cnt = segcnt[s];
-#pragma unroll 1
-    for (int j0 = 0; j0 < cnt; j0 += 32) {
-      const int j = j0 + lane;
-      f(s * seg + j, j < cnt);
-    }
-  }
-}
-
-// The leader's exact finish when the boundary bin is too big to rank directly:
-// histogram levels over the list entries with keys in [lo_k, hi_k] (the `need`-th
-// largest of them is the boundary), one warp searching, until the boundary bin is
-// one key or holds at most kSlMembers entries, which are ranked by (key, index);
-// many entries of one key are ranked by index through the bitmap `bm` of the row,
-// which is zero on entry and left for the caller to clear.  `h2` is two free
-// histograms.  The result is the composite boundary (K*, I*).
-template <int DT, int THREADS>
-__device__ __noinline__ void list_boundary(const KParams& p, const SliceGeom& g, const typename Elem<DT>::bits_t* lbits,
-                                           const uint32_t* lidx, const int* segcnt, int nseg, uint32_t lo_k,
-                                           uint32_t hi_k, int need, int* h2, uint32_t* bm, SliceCtl& ctl,
-                                           uint32_t& kstar, uint32_t& istar) {
-  using E = Elem<DT>;
-  constexpr int NW = THREADS / 32;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int seg = p.seg;
-  const uint32_t below = (1u << lane) - 1u;
-#pragma unroll 1
-  for (int i = tid; i < 2 * kSlBins / 4; i += THREADS) reinterpret_cast<int4*>(h2)[i] = make_int4(0, 0, 0, 0);
-  __syncthreads();
-#pragma unroll 1
-  for (int level = 0;; ++level) {
-    int* h = h2 + (level & 1) * kSlBins;
-    const int s = res_shift(hi_k - lo_k);
-    for_list<THREADS>(segcnt, nseg, seg, [&](int i, bool valid) {
-      if (valid) {
-        const uint32_t kk = E::key(lbits[i]);
-        if (kk >= lo_k && kk <= hi_k) atomicAdd(&h[(hi_k - kk) >> s], 1);
-      }
-    });
-    __syncthreads();
-    if (warp == 0) {
-      const BinHit bh = res_find_bin(h, need, lane);
-      if (lane == 0) {
-        ctl.bin = bh.bin;
-        ctl.before = bh.before;
-        ctl.cnt = bh.cnt;
-      }
-    }
-    {   // the other level buffer is read by nobody any more: clear it for the next level
-      int4* z = reinterpret_cast<int4*>(h2 + ((level + 1) & 1) * kSlBins);
-#pragma unroll 1
-      for (int i = tid; i < kSlBins / 4; i += THREADS) z[i] = make_int4(0, 0, 0, 0);
-    }
-    __syncthreads();
-    const int bin = ctl.bin, cnt = ctl.cnt;
-    need -= ctl.before;
-    const uint32_t bhi = hi_k - (static_cast<uint32_t>(bin) << s);
-    const uint32_t blo = res_bin_lo(hi_k, lo_k, bin, s);
-    if (s == 0 && cnt == need) {   // every entry of the boundary key is selected
-      kstar = bhi;
-      istar = 0xFFFFFFFFu;
-      return;
-    }
-    auto member = [&](int i) -> bool {
-      const uint32_t kk = E::key(lbits[i]);
-      return kk >= blo && kk <= bhi;
-    };
-    if (cnt <= kSlMembers) {   // rank the members by (key, index); slots from per-warp counts
-      int mine = 0;
-      for_list<THREADS>(segcnt, nseg, seg, [&](int i, bool valid) { mine += valid && member(i) ? 1 : 0; });
-      mine = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(mine)));
-      if (lane == 0) ctl.w_c[warp] = mine;
-      __syncthreads();
-      int M;
-      int pos = warp_prefix_of<NW>(ctl.w_c, warp, lane, M);
-      if (mine != 0) {   // warp-uniform
-        for_list<THREADS>(segcnt, nseg, seg, [&](int i, bool valid) {
-          const bool m = valid && member(i);
-          const unsigned bal = __ballot_sync(0xffffffffu, m);
-          const int at = pos + __popc(bal & below);
-          if (m && at < kSlMembers)
-            ctl.m_w[at] = (static_cast<unsigned long long>(E::key(lbits[i])) << 32) | (~lidx[i]);
-          pos += __popc(bal);
-        });
-      }
-      __syncthreads();
-      M = min(M, kSlMembers);
-#pragma unroll 1
-      for (int j = tid; j < M; j += THREADS) {
-        const unsigned long long wj = ctl.m_w[j];
-        int r = 0;
-#pragma unroll 4
-        for (int i = 0; i < M; ++i) r += ctl.m_w[i] > wj ? 1 : 0;
-        if (r == need - 1) {
-          ctl.kstar = static_cast<uint32_t>(wj >> 32);
-          ctl.istar = ~static_cast<uint32_t>(wj);
-        }
-      }
-      __syncthreads();
-      kstar = ctl.kstar;
-      istar = ctl.istar;
-      return;
-    }
-    if (s == 0) {   // many entries of the boundary key: the need-th of them in index order
-      kstar = bhi;
-      const int words = static_cast<int>((g.n + 31u) / 32u);
-      int* bp = reinterpret_cast<int*>(bm + words);
-      for_list<THREADS>(segcnt, nseg, seg, [&](int i, bool valid) {
-        if (valid && E::key(lbits[i]) == kstar) atomicOr(&bm[lidx[i] >> 5], 1u << (lidx[i] & 31u));
-      });
-      __syncthreads();
-      row_bitmap_prefix<THREADS>(bm, bp, words, ctl);
-      for_list<THREADS>(segcnt, nseg, seg, [&](int i, bool valid) {
-        if (valid && E::key(lbits[i]) == kstar && row_bitmap_rank(bm, bp, lidx[i]) == need - 1) ctl.istar = lidx[i];
-      });
-      __syncthreads();
-      istar = ctl.istar;
-      return;
-    }
-    lo_k = blo;
-    hi_k = bhi;
-  }
+  if (CLUSTER) cluster.sync();   // the peers have read this CTA's counts
 }
 
 __device__ __forceinline__ uint32_t cluster_id_x() {
@@ -535,22 +535,37 @@ __device__ __forceinline__ uint32_t cluster_id_x() {
   return r;
 }
 
+// One of VT 16-byte vectors held in registers, picked by a run-time index.
+template <int VT>
+__device__ __forceinline__ uint4 pick(const uint4 (&xs)[VT], int i) {
+  if constexpr (VT == 1) {
+    return xs[0];
+  } else if constexpr (VT == 2) {
+    return i == 0 ? xs[0] : xs[1];
+  } else {
+    static_assert(VT == 4, "one, two or four vectors per thread and chunk");
+    return i < 2 ? (i == 0 ? xs[0] : xs[1]) : (i == 2 ? xs[2] : xs[3]);
+  }
+}
+
 // One CTA per slice; clusters of C CTAs along x hold the C slices of one row.
-// The slice lands in shared memory as chunks of one 16-byte vector per thread:
-// thread t's vector of chunk c is slice vector c * THREADS + t, so (chunk, thread,
-// element) is index order and every thread holds an even share of any index range.
+// The slice lands in shared memory as one flat array of 16-byte vectors, in
+// chunks of kSlChunkVecs vectors; thread t screens vectors t, t + THREADS, ... of
+// each chunk, so its loads are conflict-free and every thread holds an even share
+// of any index range.
 template <int DT, int THREADS, bool CLUSTER>
 __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem, cg::cluster_group& cluster) {
   using E = Elem<DT>;
   using bits_t = typename E::bits_t;
   constexpr int NW = THREADS / 32;
   constexpr int PV = E::kPerVec;
-  constexpr int CE = THREADS * PV;   // elements per chunk
+  constexpr int VT = kSlChunkVecs / THREADS;   // vectors per thread and chunk
+  constexpr int CE = kSlChunkVecs * PV;        // elements per chunk
+  static_assert(VT * THREADS == kSlChunkVecs && VT * PV <= 32, "one 32-bit candidate mask per chunk");
+  static_assert(kSliceMaxChunks <= NW, "one warp issues each chunk");
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bars);
-  int* hist = reinterpret_cast<int*>(smem + p.off_hist);   // [3][kSlBins]: candidates, sample, spare
-  uint16_t* vkm = reinterpret_cast<uint16_t*>(smem + p.off_tab) + threadIdx.x;   // [sample chunk][THREADS]
-  bits_t* lbits = reinterpret_cast<bits_t*>(smem + p.off_cb);     // candidate list (leader): element bits
-  uint32_t* lidx = reinterpret_cast<uint32_t*>(smem + p.off_ci);  //                          row index
+  int* hist = reinterpret_cast<int*>(smem + p.off_hist);   // kSlVBins + kSlBins bins
+  uint16_t* vkm = reinterpret_cast<uint16_t*>(smem + p.off_tab);   // every vector's key summary
   SliceCtl& ctl = *reinterpret_cast<SliceCtl*>(smem + p.off_ctl);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t below = (1u << lane) - 1u;
@@ -561,30 +576,30 @@ __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem
   const bool leader = g.crank == 0;
   const int k = p.k;
   const int seg = p.seg;
-  sl_mark(0);
+  bits_t* wbits = reinterpret_cast<bits_t*>(smem + p.off_cb) + warp * seg;     // this warp's list segment
+  uint32_t* widx = reinterpret_cast<uint32_t*>(smem + p.off_ci) + warp * seg;
+#ifdef DSEL_STATS
+  if (tid < 32) ctl.marks[tid] = 0ull;
+#endif
+  sl_mark(ctl, 0);
 
 #pragma unroll 1
-  for (int i = tid; i < 3 * kSlBins / 4; i += THREADS) reinterpret_cast<int4*>(hist)[i] = make_int4(0, 0, 0, 0);
+  for (int i = tid; i < (kSlVBins + kSlBins) / 4; i += THREADS) reinterpret_cast<int4*>(hist)[i] = make_int4(0, 0, 0, 0);
   if (tid == 0) {
     ctl.flags = 0;
-    ctl.t_max = 0u;
-    ctl.t_min = 0xFFFFFFFFu;
-    ctl.top = 0u;
     ctl.kmax = 0u;
+    ctl.x_a = 0;
+    ctl.x_t = 0;
+    ctl.n_list = 0;
   }
   if (tid < p.vpt_cap) {
     mbar_init(smem_u32(&bars[tid]), 1);
     fence_mbar_init();
   }
   __syncthreads();
-  // the leader's counters and histogram are initialised: peers may update them
-  // after the wait half of this barrier.  (Arriving here, before any copy is
-  // issued: a cluster-scope release after a bulk copy waits for the copy to land.)
-  // Every CTA of the row arrives, and waits below unless the row is short.
-  if (CLUSTER) cluster_arrive();
   // the set-up above touched shared memory only: it may overlap the previous launch
   grid_dependency_wait();
-  sl_mark(1);
+  sl_mark(ctl, 1);
 
   // ---- the slice, and its copies issued first ----
   uint32_t sl, pa;
@@ -634,16 +649,12 @@ __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem
     bulk_g2s(smem_u32(smem + static_cast<size_t>(c) * kSlChunk), rowp + static_cast<size_t>(g.lo + e0) * E::kBytes,
              bytes, bar);
   }
-#ifdef DSEL_STATS
-  if (tid == 0 && blockIdx.x < 8) g_trace[blockIdx.x * 32 + 16] = static_cast<long long>(global_ns());
-#endif
   grid_launch_dependents();
-  sl_mark(2);
+  sl_mark(ctl, 2);
 
-  auto load_vec = [&](int c) -> uint4 {
-    return *reinterpret_cast<const uint4*>(smem + static_cast<size_t>(c) * kSlChunk + tid * kVecBytes);
-  };
-  auto valid_of = [&](int c) -> int { return static_cast<int>(g.n_sl) - (c * THREADS + tid) * PV; };
+  auto vec_of = [&](int c, int i) -> int { return c * kSlChunkVecs + i * THREADS + tid; };
+  auto load_vec = [&](int v) -> uint4 { return *reinterpret_cast<const uint4*>(smem + static_cast<size_t>(v) * kVecBytes); };
+  auto valid_of = [&](int v) -> int { return static_cast<int>(g.n_sl) - v * PV; };
   bool late = false;
   auto wait_chunk = [&](int c) {
     if (!mbar_wait(smem_u32(&bars[c]), 0u)) late = true;
@@ -653,321 +664,344 @@ __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem
     return static_cast<int>(t >= static_cast<uint32_t>(g.nch) ? t - static_cast<uint32_t>(g.nch) : t);
   };
 
-  // ---- A. threshold from the first ns chunks of the visiting order ----
-  // Candidates expected past a threshold taken from a fraction f of the row:
-  // about 1.3 k / f.  Each slice's own k-th (each valid alone; the cluster keeps
-  // the largest) while C slices' worth of candidates fit half the list with at most
-  // half the slice as sample; otherwise per-slice k' = ceil(k / C) thresholds and
-  // the cluster keeps the smallest (C slices with k' such vectors: at least k).
-  const int lcap = p.capacity;
-  auto chunks_for = [&](int64_t kk, int64_t slices) -> int {     // sample chunks for a list of lcap / 2
-    const int64_t by_list = (13 * slices * kk * nch_full + 5 * lcap - 1) / (5 * lcap);
-    const int64_t by_k = (2 * kk + THREADS - 1) / THREADS;
-    const int64_t q = (nch_full + 3) / 4;
-    return static_cast<int>(by_list > by_k ? (by_list > q ? by_list : q) : (by_k > q ? by_k : q));
-  };
-  const int ns_local = chunks_for(k, g.C);
-  const bool local = !CLUSTER || 2 * ns_local <= nch_full;
-  const int kq = local ? k : (k + g.C - 1) / g.C;
-  const int ns = min(g.nch, local ? ns_local : chunks_for(k, 1));
-  uint32_t tmax = 0u, tmin16 = 0xFFFFu;
-  int tn = 0;
+  // ---- A. as each chunk lands: every vector's largest key, summarised in 16 bits,
+  //      and a histogram of those summaries over fixed bins of 16 summaries
+  //      (bin 0 = the largest), the same bins in every CTA of the cluster ----
+  int* hv = hist;                  // [kSlVBins]: vector maxima
+  int* hc = hist + kSlVBins;       // [kSlBins]: candidate keys
   bool tnan = false;
-  {
-    int c = static_cast<int>(pc);
-#pragma unroll 1
-    for (int j = 0; j < ns; ++j, c = next_chunk(c)) {
-      wait_chunk(c);
-#ifdef DSEL_STATS
-      if (tid == 0 && blockIdx.x < 8) g_trace[blockIdx.x * 32 + j] = static_cast<long long>(global_ns());
-#endif
-      uint32_t s16 = 0u;
-      const int valid = valid_of(c);
-      if (valid > 0) {
-        uint32_t key = 0u;
-        if (vec_max_valid<DT>(load_vec(c), valid, key)) {
-          tnan = true;
-        } else {
-          s16 = key16<DT>(key);
-          tmax = max(tmax, key);
-          tmin16 = min(tmin16, s16);
-          ++tn;
-        }
-      }
-      vkm[j * THREADS] = static_cast<uint16_t>(s16);
-    }
-  }
-  sl_mark(3);
-  tmax = __reduce_max_sync(0xffffffffu, tmax);
-  tmin16 = __reduce_min_sync(0xffffffffu, tmin16);
-  tn = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(tn)));
-  if (lane == 0) {
-    ctl.w_a[warp] = tmax;
-    ctl.w_b[warp] = tmin16;
-    ctl.w_c[warp] = tn;
-  }
-  __syncthreads();
-  const uint32_t smax = __reduce_max_sync(0xffffffffu, lane < NW ? ctl.w_a[lane] : 0u);
-  const uint32_t smin = __reduce_min_sync(0xffffffffu, lane < NW ? ctl.w_b[lane] : 0xFFFFu);
-  const int sn = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(lane < NW ? ctl.w_c[lane] : 0)));
-  uint32_t t_row = 0u;
-  if (sn >= kq) {   // uniform in the CTA
-    // bins 16 times narrower than the summaries' range needs, the last one open
-    // below: the top sixteenth of the range, where the kq-th largest usually lies
-    const uint32_t top16 = key16<DT>(smax);
-    const int s = max(0, res_shift(top16 - smin) - 4);
-    int* h = hist + kSlBins;
-#pragma unroll 4
-    for (int j = 0; j < ns; ++j) {
-      const uint32_t m = vkm[j * THREADS];
-      if (m != 0u) atomicAdd(&h[min((top16 - m) >> s, static_cast<uint32_t>(kSlBins - 1))], 1);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      const BinHit bh = res_find_bin(h, kq, lane);
-      if (lane == 0) {
-        const uint32_t t16 = bh.bin == kSlBins - 1 ? smin : res_bin_lo(top16, smin, bh.bin, s);
-        ctl.t_key = DT == DSEL_BF16 ? t16 : (t16 << 16);
-      }
-    }
-    __syncthreads();
-    t_row = ctl.t_key;
-  }
-  uint32_t top = smax;   // bins of the candidate histogram count down from here
-  SliceCtl* lctl = CLUSTER ? cluster.map_shared_rank(&ctl, 0) : &ctl;
-  if (CLUSTER) {   // the cluster's threshold and top, through the leader
-    cluster_wait();   // the leader's counters are initialised
-    if (tid == 0) {
-      if (local) atomicMax(&lctl->t_max, t_row);
-      else atomicMin(&lctl->t_min, t_row);
-      atomicMax(&lctl->top, smax);
-    }
-#ifdef DSEL_STATS
-    if (tid == 0 && blockIdx.x < 8) g_trace[blockIdx.x * 32 + 18] = static_cast<long long>(global_ns());
-#endif
-    cluster.sync();
-#ifdef DSEL_STATS
-    if (tid == 0 && blockIdx.x < 8) g_trace[blockIdx.x * 32 + 19] = static_cast<long long>(global_ns());
-#endif
-    if (lane == 0) {
-      t_row = local ? lctl->t_max : lctl->t_min;
-      top = lctl->top;
-    }
-    t_row = __shfl_sync(0xffffffffu, t_row, 0);
-    top = __shfl_sync(0xffffffffu, top, 0);
-  }
-  top = max(top, t_row);
-  const int sb = res_shift(top - t_row);   // one key per bin for bfloat16 when the range allows
-  sl_mark(4);
-
-  // ---- B. filter every chunk against T: this warp's segment of the leader's
-  //      list, and this CTA's histogram of the candidates' keys ----
-  const int sid = g.crank * NW + warp;
-  bits_t* rbits = (CLUSTER ? cluster.map_shared_rank(lbits, 0) : lbits) + sid * seg;
-  uint32_t* ridx = (CLUSTER ? cluster.map_shared_rank(lidx, 0) : lidx) + sid * seg;
-  int* hc = hist;   // candidates, bins counting down from top (keys above top share bin 0)
-  const uint32_t t16 = key16<DT>(t_row);
-  uint32_t kmax_sl = tmax;   // largest key of the slice
-  int wrun = 0;              // entries of this warp's segment (warp-uniform)
+  uint32_t kmax_c = 0u;            // largest key of the slice
   {
     int c = static_cast<int>(pc);
 #pragma unroll 1
     for (int j = 0; j < g.nch; ++j, c = next_chunk(c)) {
-      const int valid = valid_of(c);
-      bool cand = false;
-      uint4 x = make_uint4(0u, 0u, 0u, 0u);
-      if (j < ns) {
-        const uint32_t sm = vkm[j * THREADS];
-        cand = valid > 0 && sm >= t16 && sm != 0u;
-        if (cand) x = load_vec(c);
-      } else {
-        wait_chunk(c);
+      wait_chunk(c);
 #ifdef DSEL_STATS
-        if (tid == 0 && blockIdx.x < 8) g_trace[blockIdx.x * 32 + j] = static_cast<long long>(global_ns());
+      if (tid == 0) ctl.marks[24 + j] = global_ns();
 #endif
+#pragma unroll
+      for (int i = 0; i < VT; ++i) {
+        const int v = vec_of(c, i);
+        const int valid = valid_of(v);
+        uint32_t s16 = 0u;
         if (valid > 0) {
-          x = load_vec(c);
           uint32_t key = 0u;
-          if (vec_max_valid<DT>(x, valid, key)) {
+          if (vec_max_valid<DT>(load_vec(v), valid, key)) {
             tnan = true;
           } else {
-            kmax_sl = max(kmax_sl, key);
-            cand = key >= t_row;
+            s16 = key16<DT>(key);
+            kmax_c = max(kmax_c, key);
+            atomicAdd(&hv[kSlVBins - 1 - static_cast<int>(s16 >> 4)], 1);
           }
         }
+        vkm[v] = static_cast<uint16_t>(s16);   // 0: no element (NaN or past the end)
       }
-      uint32_t m = cand ? res_mask_ge<DT>(x, t_row, valid) : 0u;
-      const uint32_t g0 = g.lo + static_cast<uint32_t>(c * THREADS + tid) * PV;
-#pragma unroll 1
-      while (__any_sync(0xffffffffu, m != 0u)) {   // one candidate per lane per step
-        const bool has = m != 0u;
-        const unsigned bal = __ballot_sync(0xffffffffu, has);
-        if (has) {
-          const int e = __ffs(m) - 1;
-          m &= m - 1u;
-          const int pos = wrun + __popc(bal & below);
-          const uint32_t b = vec_elem_dyn<DT>(x, e);
-          const uint32_t kk = E::key(b);
-          atomicAdd(&hc[kk >= top ? 0u : (top - kk) >> sb], 1);
-          if (pos < seg) {
-            rbits[pos] = static_cast<bits_t>(b);
-            ridx[pos] = g0 + static_cast<uint32_t>(e);
-          }
-        }
-        wrun += __popc(bal);
-      }
-#ifdef DSEL_STATS
-      if (tid == 0 && blockIdx.x < 8 && j < 8) g_trace[blockIdx.x * 32 + 20 + j] = static_cast<long long>(global_ns());
-#endif
     }
   }
-  sl_mark(5);
   {
-    const int f = (__any_sync(0xffffffffu, tnan) ? 1 : 0) | (wrun > seg ? 2 : 0) |
-                  (__any_sync(0xffffffffu, late) ? 4 : 0);
-    const uint32_t wk = __reduce_max_sync(0xffffffffu, kmax_sl);
+    const int f = (__any_sync(0xffffffffu, tnan) ? 1 : 0) | (__any_sync(0xffffffffu, late) ? 4 : 0);
+    const uint32_t wk = __reduce_max_sync(0xffffffffu, kmax_c);
     if (lane == 0) {
-      lctl->segcnt[sid] = min(wrun, seg);
-      // the flags go to every CTA's own copy: after the barrier below each reads
-      // its own (the leader may be gone before a peer could read the leader's)
-      if (f) {
-        if (CLUSTER) {
-#pragma unroll 1
-          for (int r = 0; r < g.C; ++r) atomicOr(&cluster.map_shared_rank(&ctl, r)->flags, f);
-        } else {
-          atomicOr(&ctl.flags, f);
-        }
-      }
-      atomicMax(&lctl->kmax, wk);
+      if (f) atomicOr(&ctl.flags, f);
+      atomicMax(&ctl.kmax, wk);
     }
   }
-  if (CLUSTER && !leader) {   // this CTA's candidate histogram joins the leader's
-    __syncthreads();
-    int* lh = cluster.map_shared_rank(hc, 0);
-#pragma unroll 1
-    for (int b = tid; b < kSlBins; b += THREADS) {
-      const int v = hc[b];
-      if (v) atomicAdd(&lh[b], v);
-    }
+  int* hvc = hist + kSlVBins + kSlBins;   // coarse sums: vector maxima [256], candidates [64], levels [2][64]
+  int* hcc = hvc + kSlVBins / 16;
+  __syncthreads();
+  coarse_sums<THREADS>(hv, hvc, kSlVBins / 16);
+  sl_mark(ctl, 3);
+  sl_sync<CLUSTER>(cluster);   // every CTA's vector-maximum histogram, flags and largest key are final
+  sl_mark(ctl, 4);
+  if ((ctl.flags & 4) && tid < g.nch) mbar_wait(smem_u32(&bars[tid]), 0u);   // a copy may still be landing
+  int flags;
+  uint32_t top;   // the row's largest key
+  if (CLUSTER) {
+    const SliceCtl* pr = cluster.map_shared_rank(&ctl, lane < g.C ? lane : 0);
+    flags = static_cast<int>(__reduce_or_sync(0xffffffffu, lane < g.C ? static_cast<unsigned>(pr->flags) : 0u));
+    top = __reduce_max_sync(0xffffffffu, lane < g.C ? pr->kmax : 0u);
+  } else {
+    flags = ctl.flags;
+    top = ctl.kmax;
   }
-  if (late && tid < g.nch) mbar_wait(smem_u32(&bars[tid]), 0u);   // a copy may still be landing
-  sl_sync<CLUSTER>(cluster);   // the row's candidates are in the leader's list and histogram
-  sl_mark(6);
-  const int flags = ctl.flags;
   if ((flags & 1) && !p.nan_flag) nan_trap();   // the pages' default NaN policy
   if (flags & 1) {   // flag mode: the row's NaN sentinel
     if (leader) write_sentinel_row<DT, THREADS>(p, g.row, DSEL_IDX_NAN);
+    if (CLUSTER) cluster.sync();   // the peers have read this CTA's control block
     return;
+  }
+  // T: the lowest summary of the bin that holds the k-th largest vector maximum of
+  // the row (at least k vectors hold an element >= T: a valid threshold), or 0
+  // when the row has fewer than k vectors
+  uint32_t t16 = 0u;
+  {
+    const BinHit bh = cluster_find_bin<THREADS, CLUSTER>(hv, hvc, kSlVBins / 16, k, g.C, ctl, cluster);
+    if (bh.bin >= 0) t16 = static_cast<uint32_t>(kSlVBins - 1 - bh.bin) << 4;
+  }
+  const uint32_t t_row = DT == DSEL_BF16 ? t16 : (t16 << 16);
+  const int sb = res_shift(top - t_row);   // one key per bin for bfloat16 when the range allows
+  sl_mark(ctl, 5);
+
+  // ---- B. filter, dense in two steps: the vectors whose summary reaches T into
+  //      this warp's vector list (one ballot per vector slot), then their elements
+  //      >= T into this warp's element list and the CTA's histogram of candidate
+  //      keys (bins counting down from top), 32 vectors per warp step ----
+  const uint32_t tb = E::bits_of_key(t_row);
+  const uint32_t tv2 = DT == DSEL_BF16 ? (tb | (tb << 16)) : tb;   // T as packed element bits
+  const int segv = seg / 2;
+  uint32_t* wvec = reinterpret_cast<uint32_t*>(smem + p.off_cv) + warp * segv;
+  int vrun = 0;   // vectors of this warp's vector list (warp-uniform)
+#pragma unroll 1
+  for (int c = 0; c < g.nch; ++c) {
+    uint32_t sm[VT];
+#pragma unroll
+    for (int i = 0; i < VT; ++i) sm[i] = vkm[vec_of(c, i)];
+#pragma unroll
+    for (int i = 0; i < VT; ++i) {
+      const bool cand = sm[i] >= t16 && sm[i] != 0u;
+      const unsigned bal = __ballot_sync(0xffffffffu, cand);
+      const int pos = vrun + __popc(bal & below);
+      if (cand && pos < segv) wvec[pos] = static_cast<uint32_t>(vec_of(c, i));
+      vrun += __popc(bal);
+    }
+  }
+  const int vcnt = min(vrun, segv);
+  int wrun = 0;   // entries of this warp's element list (warp-uniform)
+#pragma unroll 1
+  for (int j0 = 0; j0 < vcnt; j0 += 32) {
+    const int j = j0 + lane;
+    uint32_t m = 0u, v = 0u;
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (j < vcnt) {
+      v = wvec[j];
+      x = load_vec(static_cast<int>(v));
+      m = candidate_mask<DT>(x, tv2);
+      const int valid = valid_of(static_cast<int>(v));
+      if (valid < PV) m &= (1u << valid) - 1u;
+    }
+    const int cnt = __popc(m);
+    const int incl = warp_incl_scan(cnt, lane);
+    int pos = wrun + incl - cnt;
+#pragma unroll 1
+    while (m != 0u) {
+      const int e = __ffs(m) - 1;
+      m &= m - 1u;
+      const uint32_t b = vec_elem_dyn<DT>(x, e);
+      atomicAdd(&hc[(top - E::key(b)) >> sb], 1);
+      if (pos < seg) {
+        wbits[pos] = static_cast<bits_t>(b);
+        widx[pos] = g.lo + v * PV + static_cast<uint32_t>(e);
+      }
+      ++pos;
+    }
+    wrun += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  sl_mark(ctl, 6);
+  const int wcnt = min(wrun, seg);   // this warp's entries
+  if (lane == 0) {
+    if (wrun > seg || vrun > segv) atomicOr(&ctl.flags, 2);
+    atomicAdd(&ctl.n_list, wcnt);
+  }
+  __syncthreads();
+  coarse_sums<THREADS>(hc, hcc, kSlBins / 16);
+  sl_sync<CLUSTER>(cluster);   // every CTA's candidate histogram and list are final
+  if (CLUSTER) {
+    const SliceCtl* pr = cluster.map_shared_rank(&ctl, lane < g.C ? lane : 0);
+    flags = static_cast<int>(__reduce_or_sync(0xffffffffu, lane < g.C ? static_cast<unsigned>(pr->flags) : 0u));
+  } else {
+    flags = ctl.flags;
   }
   if (flags & 2) {   // a segment overflowed: every CTA selects exactly on its resident slice
-    slice_exact<DT, THREADS, CLUSTER>(p, smem, g, t_row, lctl->kmax, cluster);
+    slice_exact<DT, THREADS, CLUSTER>(p, smem, g.row, g.lo, g.n_sl, g.C, g.crank, t_row, top, cluster);
     return;
   }
-  if (!leader) return;   // the leader finishes the row alone
 
-  // ---- C. the boundary bin, from the summed histogram (one warp searches) ----
-  const int nseg = g.C * NW;
+  // ---- C. the boundary: histogram levels summed over the cluster ----
+  auto for_mine = [&](auto&& f) {   // this warp's entries, side by side in its lanes
+#pragma unroll 1
+    for (int j = lane; j < wcnt; j += 32) f(E::key(wbits[j]), widx[j]);
+  };
+  uint32_t lo = t_row, hi = top;
+  int s = sb, need = k;
+  const int* h = hc;
+  const int* hcs = hcc;
+  bool all_bin;   // the boundary bin is selected whole: every key >= kb
+  uint32_t kb;    // else the boundary key K*: every key > K*, and ties in index order
+#pragma unroll 1
+  for (int level = 0;; ++level) {
+    const BinHit bh = cluster_find_bin<THREADS, CLUSTER>(h, hcs, kSlBins / 16, need, g.C, ctl, cluster);
+    if (bh.bin < 0) {   // cannot happen (the bins hold the row's entries >= lo): select from lo
+      all_bin = true;
+      kb = lo;
+      break;
+    }
+    need -= bh.before;
+    const uint32_t bhi = hi - (static_cast<uint32_t>(bh.bin) << s);
+    const uint32_t blo = res_bin_lo(hi, lo, bh.bin, s);
+    if (bh.cnt == need || blo == bhi) {
+      all_bin = bh.cnt == need;
+      kb = blo;
+      break;
+    }
+    lo = blo;
+    hi = bhi;
+    s = res_shift(hi - lo);
+    // levels 1, 2, ... alternate between two buffers in the vector-maximum
+    // histogram's space: every CTA read their previous contents before the last
+    // cluster barrier
+    int* hn = hist + (level & 1) * kSlBins;
+    int* hnc = hcc + kSlBins / 16 * (1 + (level & 1));
+#pragma unroll 1
+    for (int i = tid; i < kSlBins / 4; i += THREADS) reinterpret_cast<int4*>(hn)[i] = make_int4(0, 0, 0, 0);
+    __syncthreads();
+    for_mine([&](uint32_t kk, uint32_t) {
+      if (kk >= lo && kk <= hi) atomicAdd(&hn[(hi - kk) >> s], 1);
+    });
+    __syncthreads();
+    coarse_sums<THREADS>(hn, hnc, kSlBins / 16);
+    sl_sync<CLUSTER>(cluster);   // the level's histograms are complete
+    h = hn;
+    hcs = hnc;
+  }
+  sl_mark(ctl, 7);
 #ifdef DSEL_STATS
-  if (tid == 0 && blockIdx.x < kStatsCtas) {   // list length, sample chunks, mode, chunks
-    int tot = 0;
-    for (int s2 = 0; s2 < nseg; ++s2) tot += ctl.segcnt[s2];
-    g_stats[blockIdx.x * kStatsFields + 12] = static_cast<unsigned long long>(tot);
-    g_stats[blockIdx.x * kStatsFields + 13] = static_cast<unsigned long long>(ns);
-    g_stats[blockIdx.x * kStatsFields + 14] = local ? 1ull : 0ull;
-    g_stats[blockIdx.x * kStatsFields + 15] = static_cast<unsigned long long>(g.nch);
+  if (tid == 0) {   // threshold summary, list entries
+    ctl.marks[14] = static_cast<unsigned long long>(t16);
+    ctl.marks[15] = static_cast<unsigned long long>(ctl.n_list);
   }
 #endif
-  if (warp == 0) {
-    const BinHit bh = res_find_bin(hc, k, lane);
-    if (lane == 0) {
-      ctl.bin = bh.bin;
-      ctl.before = bh.before;
-      ctl.cnt = bh.cnt;
-    }
-  }
-  __syncthreads();
-  const int bin = ctl.bin, bcnt = ctl.cnt;
-  const int need = k - ctl.before;   // entries of the boundary bin to select (1..bcnt)
-  const uint32_t bhi = bin == 0 ? 0xFFFFFFFFu : top - (static_cast<uint32_t>(bin) << sb);
-  const uint32_t blo = res_bin_lo(top, t_row, bin, sb);
-  // row bitmaps in the leader's dead slice: selected entries, then the block prefix
-  uint32_t* bm = reinterpret_cast<uint32_t*>(smem);
-  const int words = static_cast<int>((g.n + 31u) / 32u);
-  int* bp = reinterpret_cast<int*>(bm + words);
+
+  // ---- this slice's share, and per-block counts for the index-order ranks ----
+  // Block b (32 consecutive vectors of the slice) belongs to warp b % NW, and each
+  // warp's list is in index order, so an entry's rank among this slice's entries
+  // of a kind (above the boundary, or equal to it) is the count in earlier blocks
+  // plus the warp's running count since the block's first entry.
+  const int nblk = g.nch * (kSlChunkVecs / 32);
+  int* ba = reinterpret_cast<int*>(smem + p.off_tab);   // [nblk] entries above the boundary, per block
+  int* bt = ba + nblk;                                   // [nblk] entries equal to the boundary key
+  int* sa = bt + nblk;                                   // [nblk] the owning warp's running counts at
+  int* st = sa + nblk;                                   //        the block's first entry
 #pragma unroll 1
-  for (int w = tid; w < words; w += THREADS) bm[w] = 0u;
+  for (int i = tid; i < 2 * nblk; i += THREADS) ba[i] = 0;
   __syncthreads();
-  const bool all_bin = bcnt == need;   // every member of the boundary bin is selected
-  if (!all_bin && bcnt > kSlMembers) {   // heavy ties or a coarse bin: exact levels over the list
-    uint32_t kstar = 0u, istar = 0u;
-    list_boundary<DT, THREADS>(p, g, lbits, lidx, ctl.segcnt, nseg, blo, bhi == 0xFFFFFFFFu ? ctl.kmax : bhi,
-                               need, hist + kSlBins, bm, ctl, kstar, istar);
+  auto kinds = [&](uint32_t kk, bool& a, bool& t) {
+    a = all_bin ? kk >= kb : kk > kb;
+    t = !all_bin && kk == kb;
+  };
+  auto block_of = [&](uint32_t gi) -> int { return static_cast<int>((gi - g.lo) / static_cast<uint32_t>(PV * 32)); };
+  {
+    int ra = 0, rt = 0, last = -1;   // running counts and block (warp-uniform)
 #pragma unroll 1
-    for (int w = tid; w < words; w += THREADS) bm[w] = 0u;
-    __syncthreads();
-    for_list<THREADS>(ctl.segcnt, nseg, seg, [&](int i, bool valid) {
-      const uint32_t kk = E::key(lbits[i]);
-      if (valid && (kk > kstar || (kk == kstar && lidx[i] <= istar))) atomicOr(&bm[lidx[i] >> 5], 1u << (lidx[i] & 31u));
-    });
-  } else {
-    // entries above the boundary bin (and the whole bin when all of it is selected)
-    // go into the bitmap; the bin's members are counted per warp
-    const uint32_t sel_lo = all_bin ? blo : (bhi == 0xFFFFFFFFu ? 0xFFFFFFFFu : bhi + 1u);
-    int mine = 0;
-    for_list<THREADS>(ctl.segcnt, nseg, seg, [&](int i, bool valid) {
+    for (int j0 = 0; j0 < wcnt; j0 += 32) {
+      const int j = j0 + lane;
+      const bool valid = j < wcnt;
+      bool a = false, t = false;
+      int b = -1;
       if (valid) {
-        const uint32_t kk = E::key(lbits[i]);
-        if (kk >= sel_lo && (sel_lo != 0xFFFFFFFFu || all_bin)) atomicOr(&bm[lidx[i] >> 5], 1u << (lidx[i] & 31u));
-        else if (!all_bin && kk >= blo) ++mine;
+        const uint32_t gi = widx[j];
+        kinds(E::key(wbits[j]), a, t);
+        b = block_of(gi);
       }
-    });
-    if (!all_bin) {   // rank the members by (key, index): the first `need` are selected
-      mine = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(mine)));
-      if (lane == 0) ctl.w_c[warp] = mine;
-      __syncthreads();
-      int M;
-      int pos = warp_prefix_of<NW>(ctl.w_c, warp, lane, M);
-      if (mine != 0) {   // warp-uniform
-        for_list<THREADS>(ctl.segcnt, nseg, seg, [&](int i, bool valid) {
-          const uint32_t kk = valid ? E::key(lbits[i]) : 0u;
-          const bool m = valid && kk >= blo && kk < sel_lo;
-          const unsigned bal = __ballot_sync(0xffffffffu, m);
-          if (m) ctl.m_w[pos + __popc(bal & below)] = (static_cast<unsigned long long>(kk) << 32) | (~lidx[i]);
-          pos += __popc(bal);
-        });
+      const unsigned am = __ballot_sync(0xffffffffu, a), tm = __ballot_sync(0xffffffffu, t);
+      const int prev = __shfl_up_sync(0xffffffffu, b, 1);
+      if (valid && b != (lane == 0 ? last : prev)) {   // the block's first entry in this warp's list
+        sa[b] = ra + __popc(am & below);
+        st[b] = rt + __popc(tm & below);
       }
-      __syncthreads();
-#pragma unroll 1
-      for (int j = tid; j < M; j += THREADS) {
-        const unsigned long long wj = ctl.m_w[j];
-        int r = 0;
-#pragma unroll 4
-        for (int i = 0; i < M; ++i) r += ctl.m_w[i] > wj ? 1 : 0;
-        if (r < need) {
-          const uint32_t gi = ~static_cast<uint32_t>(wj);
-          atomicOr(&bm[gi >> 5], 1u << (gi & 31u));
-        }
-      }
+      if (a) atomicAdd(&ba[b], 1);
+      if (t) atomicAdd(&bt[b], 1);
+      ra += __popc(am);
+      rt += __popc(tm);
+      last = __shfl_sync(0xffffffffu, b, 31);
+    }
+    if (lane == 0) {
+      if (ra) atomicAdd(&ctl.x_a, ra);
+      if (rt) atomicAdd(&ctl.x_t, rt);
     }
   }
-  __syncthreads();
-  row_bitmap_prefix<THREADS>(bm, bp, words, ctl);
-  sl_mark(7);
+  sl_sync<CLUSTER>(cluster);   // every slice's counts are published
+  int off, my_ties;
+  {
+    const SliceCtl* pr = CLUSTER ? cluster.map_shared_rank(&ctl, lane < g.C ? lane : 0) : &ctl;
+    const int ar = lane < g.C ? pr->x_a : 0;
+    const int tr = lane < g.C ? pr->x_t : 0;
+    const int tin = warp_incl_scan(tr, lane);
+    const int take = min(max(need - (tin - tr), 0), tr);   // ties slice `lane` contributes
+    const int sel = ar + take;
+    const int sin = warp_incl_scan(sel, lane);
+    off = __shfl_sync(0xffffffffu, sin - sel, g.crank);
+    my_ties = __shfl_sync(0xffffffffu, take, g.crank);
+  }
+  if (CLUSTER) cluster_arrive();   // done with the peers' shared memory
+  sl_mark(ctl, 10);
+
+  // exclusive prefix over the blocks of both counts (nblk <= 8 * 32 <= THREADS... or
+  // several blocks per thread)
+  {
+    constexpr int NW2 = THREADS / 32;
+    const int per = (nblk + THREADS - 1) / THREADS;
+    const int b0 = min(nblk, tid * per), b1 = min(nblk, b0 + per);
+    int xa = 0, xt = 0;
+#pragma unroll 1
+    for (int b = b0; b < b1; ++b) {
+      xa += ba[b];
+      xt += bt[b];
+    }
+    const int ia = warp_incl_scan(xa, lane), it = warp_incl_scan(xt, lane);
+    if (lane == 31) {
+      ctl.w_a[warp] = static_cast<uint32_t>(ia);
+      ctl.w_b[warp] = static_cast<uint32_t>(it);
+    }
+    __syncthreads();
+    int ta, tt;
+    int ra = warp_prefix_of<NW2>(reinterpret_cast<const int*>(ctl.w_a), warp, lane, ta) + ia - xa;
+    int rt = warp_prefix_of<NW2>(reinterpret_cast<const int*>(ctl.w_b), warp, lane, tt) + it - xt;
+#pragma unroll 1
+    for (int b = b0; b < b1; ++b) {
+      const int ca = ba[b], ct = bt[b];
+      ba[b] = ra;
+      bt[b] = rt;
+      ra += ca;
+      rt += ct;
+    }
+    __syncthreads();
+  }
+  sl_mark(ctl, 8);
 
   // ---- output: every selected entry at its rank in index order ----
-  const int64_t obase = g.row * static_cast<int64_t>(k);
-  for_list<THREADS>(ctl.segcnt, nseg, seg, [&](int i, bool valid) {
-    if (!valid) return;
-    const uint32_t gi = lidx[i];
-    if (!((bm[gi >> 5] >> (gi & 31u)) & 1u)) return;
-    const int pos = row_bitmap_rank(bm, bp, gi);
-    if (pos < k) {
-      if (p.index_i64) static_cast<int64_t*>(p.indices_out)[obase + pos] = static_cast<int64_t>(gi);
-      else static_cast<int32_t*>(p.indices_out)[obase + pos] = static_cast<int32_t>(gi);
-      if (p.return_value) static_cast<bits_t*>(p.values_out)[obase + pos] = lbits[i];
+  {
+    const int64_t obase = g.row * static_cast<int64_t>(k);
+    int ra = 0, rt = 0;
+#pragma unroll 1
+    for (int j0 = 0; j0 < wcnt; j0 += 32) {
+      const int j = j0 + lane;
+      bool a = false, t = false;
+      uint32_t gi = 0u, kk = 0u;
+      if (j < wcnt) {
+        gi = widx[j];
+        kk = E::key(wbits[j]);
+        kinds(kk, a, t);
+      }
+      const unsigned am = __ballot_sync(0xffffffffu, a), tm = __ballot_sync(0xffffffffu, t);
+      if (a || t) {
+        const int b = block_of(gi);
+        const int rank_a = ba[b] + ra + __popc(am & below) - sa[b];   // above entries before this one
+        const int rank_t = bt[b] + rt + __popc(tm & below) - st[b];   // boundary-key entries before it
+        if (a || rank_t < my_ties) {
+          const int pos = off + rank_a + min(rank_t, my_ties);
+          if (pos < k) {
+            if (p.index_i64) static_cast<int64_t*>(p.indices_out)[obase + pos] = static_cast<int64_t>(gi);
+            else static_cast<int32_t*>(p.indices_out)[obase + pos] = static_cast<int32_t>(gi);
+            if (p.return_value) static_cast<bits_t*>(p.values_out)[obase + pos] = wbits[j];
+          }
+        }
+      }
+      ra += __popc(am);
+      rt += __popc(tm);
     }
-  });
-  sl_mark(9);
+  }
+  sl_mark(ctl, 9);
+  if (CLUSTER) cluster_wait();   // the peers are done with this CTA's shared memory
 }
 
 template <int DT, int THREADS, bool CLUSTER>
@@ -975,7 +1009,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_slice_kernel(const __grid_con
   extern __shared__ __align__(1024) unsigned char smem[];
   cg::cluster_group cluster = cg::this_cluster();
   slice_body<DT, THREADS, CLUSTER>(p, smem, cluster);
-  sl_mark(11);
+  sl_marks_out(*reinterpret_cast<SliceCtl*>(smem + p.off_ctl));
 }
 
 }  // namespace dsel

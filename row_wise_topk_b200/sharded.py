@@ -48,6 +48,8 @@ class CudaBackend:
         import torch
         import torch.distributed as dist
 
+        if not dist.is_initialized():   # a single process: the gather is the identity
+            return values.unsqueeze(0), indices.unsqueeze(0)
         world = dist.get_world_size(group)
         vg = torch.empty((world,) + tuple(values.shape), dtype=values.dtype, device=values.device)
         ig = torch.empty((world,) + tuple(indices.shape), dtype=indices.dtype, device=indices.device)

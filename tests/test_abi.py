@@ -136,12 +136,13 @@ def test_plan_invariants(dtype, rows, stride, k):
     assert p["kernel"] in (T.DSEL_KERNEL_STREAM, T.DSEL_KERNEL_RESIDENT, T.DSEL_KERNEL_SLICE)
     if p["kernel"] == T.DSEL_KERNEL_SLICE:
         # rows cut into `cluster` slices, each held whole in one CTA's shared memory as
-        # chunks of 8 KB (one 16-byte vector per thread), plus a candidate list
-        assert p["threads"] == 1024 and p["groups"] == 1 and 1 <= p["cluster"] <= 16
+        # chunks of 16 KB, plus the CTA's candidate lists; 512 threads from 4 chunks
+        assert p["threads"] == (512 if p["stages"] >= 4 else 256)
+        assert p["groups"] == 1 and 1 <= p["cluster"] <= 16
         assert p["round"] % 16 == 0 and p["round"] * p["cluster"] >= stride
         assert p["block"] * eb == 16384 and p["stages"] == -(-p["round"] // p["block"]) <= 8
         assert p["capacity"] >= 2 * k + 2048 and p["capacity"] % 32 == 0      # candidate list
-        assert p["smem_bytes"] >= p["stages"] * (16384 + 2048) + p["capacity"] * (eb + 4) + 3 * 4096
+        assert p["smem_bytes"] >= p["stages"] * (16384 + 2048) + p["capacity"] * (eb + 4) + 5 * 4096
         assert p["b2"] == 0 and p["workspace_bytes"] == 0
         assert (1 << p["idx_bits"]) >= stride
         # as few slices as fit (8 chunks and a list of 2k + 2048), or more while the
@@ -149,8 +150,8 @@ def test_plan_invariants(dtype, rows, stride, k):
         def fits(c):
             sl = (-(-stride // c) + 15) // 16 * 16
             ch = -(-sl * eb // 16384)
-            fixed = ch * (16384 + 2048) + -(-ch * 8 // 16) * 16 + 3 * 4096 + 6144 + 64
-            lcap = min(16384, (PEAK["smem_optin"] - fixed) // (eb + 4)) // 32 * 32
+            fixed = ch * (16384 + 2048) + -(-ch * 8 // 16) * 16 + 5632 * 4 + 1024 + 64
+            lcap = min(16384, (PEAK["smem_optin"] - fixed) // (eb + 6)) // 32 * 32
             return ch <= 8 and lcap >= 2 * k + 2048
         assert fits(p["cluster"])
         assert p["cluster"] == 1 or not fits(p["cluster"] - 1) or \
@@ -204,7 +205,12 @@ def test_plan_splits():
     p = T.dsel_plan(T.DSEL_BF16, 4096, 16384, 512, **PEAK)[1]
     assert p["kernel"] == T.DSEL_KERNEL_RESIDENT and p["threads"] == 256
     p = T.dsel_plan(T.DSEL_BF16, 4096, 16400, 512, **PEAK)[1]
-    assert p["kernel"] == T.DSEL_KERNEL_SLICE and p["cluster"] == 1 and p["threads"] == 1024
+    assert p["kernel"] == T.DSEL_KERNEL_STREAM and p["threads"] == 128
+    # the slice kernel only when one wave of slices covers the batch
+    p = T.dsel_plan(T.DSEL_BF16, 64, 131072, 512, **PEAK)[1]
+    assert p["kernel"] == T.DSEL_KERNEL_SLICE and p["cluster"] * 64 <= PEAK["num_sms"]
+    p = T.dsel_plan(T.DSEL_F32, 256, 129280, 1024, **PEAK)[1]
+    assert p["kernel"] == T.DSEL_KERNEL_STREAM
     # value order never takes the slice kernel
     p = T.dsel_plan_for(T.DSEL_F32, 256, 129280, 1024, T.DSEL_ORDER_VALUE, **PEAK)[1]
     assert p["kernel"] == T.DSEL_KERNEL_STREAM and p["threads"] == 256
@@ -213,18 +219,19 @@ def test_plan_splits():
     assert T.dsel_plan_for(T.DSEL_F32, 4, 8192, 64, 3, **PEAK)[0] == header_define("DSEL_ERR_ORDER")
     # fewer rows than SMs: never resident
     assert T.dsel_plan(T.DSEL_BF16, 147, 16384, 512, **PEAK)[1]["kernel"] == T.DSEL_KERNEL_SLICE
-    # rows longer than sixteen 160 KB slices: the streaming kernel
+    # rows longer than sixteen 128 KB slices: the streaming kernel
     assert T.dsel_plan(T.DSEL_F32, 256, 1 << 20, 4096, **PEAK)[1]["kernel"] == T.DSEL_KERNEL_STREAM
     # long rows, k <= 1024, at least as many rows as SMs: 256 threads, two CTAs per SM
     assert T.dsel_plan(T.DSEL_F32, 256, 1 << 20, 1024, **PEAK)[1]["threads"] == 256
     # 64 indexer rows: two slices per row, each held in one CTA's shared memory
     p = T.dsel_plan(T.DSEL_BF16, 64, 131072, 512, **PEAK)[1]
     assert (p["kernel"], p["cluster"], p["groups"]) == (T.DSEL_KERNEL_SLICE, 2, 1)
-    # one or eight sampler rows: sixteen slices per row; 256 rows: the fewest slices that fit
+    # one or eight sampler rows: sixteen slices per row; 256 rows (several waves of
+    # slices): the streaming kernel
     assert T.dsel_plan(T.DSEL_F32, 1, 129280, 50, **PEAK)[1]["cluster"] == 16
     assert T.dsel_plan(T.DSEL_F32, 8, 129280, 1024, **PEAK)[1]["cluster"] == 16
     p = T.dsel_plan(T.DSEL_F32, 256, 129280, 1024, **PEAK)[1]
-    assert (p["kernel"], p["cluster"]) == (T.DSEL_KERNEL_SLICE, 4)
+    assert p["kernel"] == T.DSEL_KERNEL_STREAM
     # a single 2^28 row uses several clusters
     p = T.dsel_plan(T.DSEL_F32, 1, 1 << 28, 1000, **PEAK)[1]
     assert p["groups"] > 1 and p["cluster"] == 8

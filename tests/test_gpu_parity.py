@@ -55,26 +55,38 @@ def test_option_grid(dtype, order, rv, idt):
     check(w, order=order, return_value=rv, index_dtype=idt)
 
 
+SPLIT = [
+    # (dtype, rows, row_stride, k): rows longer than one cluster's slices; the longest
+    # span several clusters whose partial results the merge kernel combines
+    ("f32", 1, 1 << 20, 4096),
+    ("f32", 2, 1 << 19, 1000),
+    ("f32", 1, 1 << 22, 512),
+    ("bf16", 1, 1 << 22, 512),
+    ("bf16", 3, 1 << 21, 2000),
+]
+
+
 @pytest.mark.parametrize("dist", ["ascending", "equal", "ties"])
-@pytest.mark.parametrize("rows,stride,k", [(1, 1 << 20, 4096), (2, 1 << 19, 1000), (1, 1 << 22, 512)])
-def test_split_rows(dist, rows, stride, k):
+@pytest.mark.parametrize("dtype,rows,stride,k", SPLIT)
+def test_split_rows(dist, dtype, rows, stride, k):
     """few long rows: cluster split and, for the longest, several clusters + merge"""
-    w = W.random_small(11, "f32", rows, stride, k, dist=dist, sorted_index=1)
+    w = W.random_small(11, dtype, rows, stride, k, dist=dist, sorted_index=1)
     check(w, order=T.DSEL_ORDER_INDEX)
-    check(w, order=T.DSEL_ORDER_VALUE)
+    if dtype == "f32":   # value order is float32 only
+        check(w, order=T.DSEL_ORDER_VALUE)
     check(w, order=T.DSEL_ORDER_NONE)
 
 
-def test_plans_cover_split_and_merge():
-    st, p = T.dsel_plan(T.DSEL_F32, 1, 1 << 22, 512)
-    assert st == 0 and p["groups"] > 1
-    st, p = T.dsel_plan(T.DSEL_F32, 2, 1 << 19, 1000)
-    assert st == 0 and p["cluster"] > 1
+@pytest.mark.parametrize("dtype,rows,stride,k", [("f32", 1, 1 << 22, 512), ("bf16", 1, 1 << 22, 512),
+                                                  ("bf16", 3, 1 << 21, 2000)])
+def test_plans_cover_split_and_merge(dtype, rows, stride, k):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    dt = T.DSEL_BF16 if dtype == "bf16" else T.DSEL_F32
+    for order in (T.DSEL_ORDER_INDEX, T.DSEL_ORDER_NONE):
+        st, p = T.dsel_plan_for(dt, rows, stride, k, order, num_sms=sms)
+        assert st == 0 and p["kernel"] == T.DSEL_KERNEL_STREAM and p["groups"] > 1
 
 
-# --------------------------------------------------------------------------- #
-# edge cases
-# --------------------------------------------------------------------------- #
 def test_all_rows_short():
     w = W.random_small(3, "bf16", 10, 16, 4096, dist="normal")
     check(w, order=1)
@@ -148,17 +160,17 @@ def test_torch_wrapper_bf16():
 # the workload families at full size (the bench's launch configuration)
 # --------------------------------------------------------------------------- #
 # --------------------------------------------------------------------------- #
-# many rows of 32-64 KB: one slice per row (no cluster), several waves of CTAs
+# up to one wave of rows of 32-64 KB: one slice per row (no cluster)
 # --------------------------------------------------------------------------- #
 SHORT = [
     # (seed, dtype, rows, stride, k, dist, order): bf16 rows above 32 KB (shorter ones
-    # go to the row-resident kernel), each one slice of the slice kernel
-    (301, "bf16", 160, 32768, 1, "normal", 1),
-    (302, "bf16", 160, 32768, 512, "ties", 0),
-    (303, "bf16", 150, 16400, 4096, "normal", 1),
-    (304, "bf16", 300, 20480, 512, "ties", 1),
-    (305, "bf16", 150, 24576, 64, "ascending", 0),
-    (306, "bf16", 160, 30000 // 16 * 16, 2000, "equal", 1),
+    # go to the row-resident kernel), each one slice of the slice kernel, one CTA per SM
+    (301, "bf16", 148, 32768, 1, "normal", 1),
+    (302, "bf16", 140, 32768, 512, "ties", 0),
+    (303, "bf16", 100, 16400, 4096, "normal", 1),
+    (304, "bf16", 120, 20480, 512, "ties", 1),
+    (305, "bf16", 148, 24576, 64, "ascending", 0),
+    (306, "bf16", 97, 30000 // 16 * 16, 2000, "equal", 1),
 ]
 
 
@@ -175,13 +187,16 @@ def test_one_slice_rows(seed, dtype, rows, stride, k, dist, order):
 
 MID = [
     # (seed, dtype, rows, stride, k, dist, order): value order takes the streaming kernel's
-    # 256-thread shape (two CTAs per SM); index order and no order the slice kernel
-    (401, "f32", 150, 65536, 1024, "normal", 2),
-    (402, "f32", 160, 40960, 50, "ties", 2),
-    (403, "bf16", 152, 131072, 512, "ascending", 1),
-    (404, "f32", 149, 16400, 700, "equal", 2),
-    (405, "f32", 150, 65536, 1024, "normal", 1),
-    (406, "f32", 160, 40960, 50, "ties", 0),
+    # 256-thread shape (two CTAs per SM); index order and no order the slice kernel, a
+    # cluster per row, one wave of CTAs
+    (401, "f32", 70, 65536, 1024, "normal", 2),
+    (402, "f32", 72, 40960, 50, "ties", 2),
+    (403, "bf16", 64, 131072, 512, "ascending", 1),
+    (404, "f32", 49, 16400, 700, "equal", 2),
+    (405, "f32", 70, 65536, 1024, "normal", 1),
+    (406, "f32", 74, 40960, 50, "ties", 0),
+    (407, "f32", 37, 129280, 1024, "ties", 1),
+    (408, "bf16", 9, 131072, 2000, "normal", 0),
 ]
 
 
@@ -190,9 +205,10 @@ def test_mid_row_shape(seed, dtype, rows, stride, k, dist, order):
     st, plan = T.dsel_plan_for(T.DSEL_BF16 if dtype == "bf16" else T.DSEL_F32, rows, stride, k, order,
                                num_sms=torch.cuda.get_device_properties(0).multi_processor_count)
     if order == T.DSEL_ORDER_VALUE:
-        assert st == 0 and plan["threads"] == 256, "the case must use the 256-thread shape"
+        assert st == 0 and plan["kernel"] == T.DSEL_KERNEL_STREAM, "value order takes the streaming kernel"
     else:
         assert st == 0 and plan["kernel"] == T.DSEL_KERNEL_SLICE and plan["cluster"] >= 2
+        assert rows * plan["cluster"] <= torch.cuda.get_device_properties(0).multi_processor_count
     w = W.random_small(seed, dtype, rows, stride, k, dist=dist, with_end=(seed % 2 == 0),
                        end_lo=0, sorted_index=1, return_value=1, index_dtype="i64")
     check(w, order=order)

@@ -12,7 +12,9 @@ of the visit is (a*j + c) mod nb, a the first odd number coprime to nb at or
 above 0.618*nb, c a hash of the row), so the sample over-represents the row's
 top: the seeded T lands among the 2048 high values while k = 3000, so fewer than
 k candidates reach it and the first pass cannot be certified.  A counter build of the library,
-when present, confirms that those rows took the second pass.
+when present, confirms that those rows took the second pass.  The streaming kernel takes
+these rows under value order; under index order the slice kernel takes them, and the
+same rows check its own sample (the first chunks to land) against the oracle.
 """
 import json
 import math
@@ -62,9 +64,12 @@ def adversarial_rows(rows=150, n=8 * 16384, seed=5):
 
 
 def test_plan_is_one_cta_per_multi_round_row():
-    st, p = T.dsel_plan(T.DSEL_F32, 150, 8 * 16384, 3000,
-                        num_sms=torch.cuda.get_device_properties(0).multi_processor_count)
-    assert st == 0 and p["threads"] == 512 and p["cluster"] == 1 and p["groups"] == 1
+    # value order keeps these rows on the streaming kernel (index order takes the
+    # slice kernel, which has no rounds)
+    st, p = T.dsel_plan_for(T.DSEL_F32, 150, 8 * 16384, 3000, T.DSEL_ORDER_VALUE,
+                            num_sms=torch.cuda.get_device_properties(0).multi_processor_count)
+    assert st == 0 and p["kernel"] == T.DSEL_KERNEL_STREAM
+    assert p["threads"] == 512 and p["cluster"] == 1 and p["groups"] == 1
     assert p["block"] == 1024 and p["round"] == 16384
 
 
@@ -96,10 +101,12 @@ import workloads as W
 from gpu_util import run_gpu
 from test_gpu_sampled_seed import adversarial_rows
 x = adversarial_rows()
-w = W.Workload("adv", "f32", W.f32_bits(x), None, 3000, sorted_index=1, return_value=1, index_dtype="i64")
+w = W.Workload("adv", "f32", W.f32_bits(x), None, 3000, sorted_index=T.DSEL_ORDER_VALUE, return_value=1,
+               index_dtype="i64")
 run_gpu(w)
 stats = T.dsel_debug_stats(w.rows)
 w2 = W.sampler_logits(160, 1024, seed=13)
+w2.sorted_index = T.DSEL_ORDER_VALUE
 run_gpu(w2)
 stats2 = T.dsel_debug_stats(w2.rows)
 print(json.dumps({"adv": [s[7] for s in stats], "iid": [s[7] for s in stats2]}))
