@@ -57,10 +57,11 @@ def make_workload(name: str) -> W.Workload:
         return w
     if name.startswith("long_split"):     # long_split_k: one 2^28 row (the reference arm's view)
         return W.long_rows(1, LONG_SPLIT_N, int(name.split("_")[2]), "uniform")
-    if name.startswith("long"):           # long_1_1000 (1 x 2^28) or long_16_4096 (16 x 2^24)
-        _, r, k = name.split("_")
-        r = int(r)
-        return W.long_rows(r, (1 << 28) if r == 1 else (1 << 24), int(k), "uniform")
+    if name.startswith("long"):           # long_1_1000 (1 x 2^28), long_16_4096 (16 x 2^24),
+        parts = name.split("_")           # long_16_4096_22 (16 x 2^22: a reduced case for profiling)
+        r, k = int(parts[1]), int(parts[2])
+        n = (1 << int(parts[3])) if len(parts) > 3 else ((1 << 28) if r == 1 else (1 << 24))
+        return W.long_rows(r, n, k, "uniform")
     if name == "pr1":
         return W.pr1_duplicates()
     raise SystemExit(f"unknown workload {name}")

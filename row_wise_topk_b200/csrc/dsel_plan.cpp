@@ -113,10 +113,10 @@ int make_plan_ex(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t
         break;
       }
     }
-    // one wave only: a CTA holds its SM from the first copy to the last write, so
-    // batches needing several waves of slices go to the streaming kernel, whose
-    // two CTAs per SM overlap one row's tail with the next row's loads
-    if (cmin > 0 && rows * cmin <= num_sms) {
+    // a few waves at most: a CTA holds its SM from the first copy to the last
+    // write, so batches needing many waves of slices go to the streaming kernel,
+    // whose two CTAs per SM overlap one row's tail with the next row's loads
+    if (cmin > 0 && rows * cmin <= kSliceMaxWaves * int64_t(num_sms)) {
       int64_t c = std::max<int64_t>(1, num_sms / std::max<int64_t>(rows, 1));
       c = std::min<int64_t>({c, slice_cluster, std::max<int64_t>(1, ceil_div(row_stride, kSliceMinElems))});
       c = std::max(c, cmin);

@@ -36,6 +36,7 @@ constexpr int kSliceChunkBytes = 16384;
 constexpr int kSliceMaxChunks = 8;
 constexpr int kSliceMaxCluster = 16;          // non-portable cluster size (B200 schedules 16)
 constexpr int kSliceMinElems = 8192;          // smallest slice worth its own CTA
+constexpr int kSliceMaxWaves = 4;             // batches of more slices than this many SM waves stream
 constexpr int kSliceCtlBytes = 1024;          // its control block
 constexpr int kSliceMaxList = 16384;          // candidate-list entries
 // Vectors each thread screens per round (a warp owns whole blocks): 16 for bf16

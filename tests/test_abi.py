@@ -206,9 +206,11 @@ def test_plan_splits():
     assert p["kernel"] == T.DSEL_KERNEL_RESIDENT and p["threads"] == 256
     p = T.dsel_plan(T.DSEL_BF16, 4096, 16400, 512, **PEAK)[1]
     assert p["kernel"] == T.DSEL_KERNEL_STREAM and p["threads"] == 128
-    # the slice kernel only when one wave of slices covers the batch
+    # the slice kernel only while at most four waves of slices cover the batch
     p = T.dsel_plan(T.DSEL_BF16, 64, 131072, 512, **PEAK)[1]
     assert p["kernel"] == T.DSEL_KERNEL_SLICE and p["cluster"] * 64 <= PEAK["num_sms"]
+    p = T.dsel_plan(T.DSEL_F32, 64, 129280, 4096, **PEAK)[1]
+    assert p["kernel"] == T.DSEL_KERNEL_SLICE and p["cluster"] * 64 <= 4 * PEAK["num_sms"]
     p = T.dsel_plan(T.DSEL_F32, 256, 129280, 1024, **PEAK)[1]
     assert p["kernel"] == T.DSEL_KERNEL_STREAM
     # value order never takes the slice kernel
