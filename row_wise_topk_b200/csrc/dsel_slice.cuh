@@ -61,12 +61,14 @@ struct __align__(16) SliceCtl {
 #endif
 };
 
-// Phase timestamps of thread 0 (%globaltimer, ns) in counter builds only, kept
-// in shared memory (a global store before a cluster barrier would make the
-// barrier's release wait for it) and written to g_stats[cta][i] when the CTA ends.
+// Phase timestamps of thread 0 in counter builds only: the SM's cycle counter
+// (cheap to read), kept in shared memory (a global store before a cluster barrier
+// would make the barrier's release wait for it) and written to g_stats[cta][i]
+// when the CTA ends.  Cycles count from the CTA's own start: compare durations
+// within a CTA.
 __device__ __forceinline__ void sl_mark(SliceCtl& ctl, int i) {
 #ifdef DSEL_STATS
-  if (threadIdx.x == 0) ctl.marks[i] = global_ns();
+  if (threadIdx.x == 0) ctl.marks[i] = static_cast<unsigned long long>(clock64());
 #else
   (void)ctl;
   (void)i;
@@ -76,7 +78,7 @@ __device__ __forceinline__ void sl_mark(SliceCtl& ctl, int i) {
 __device__ __forceinline__ void sl_marks_out(SliceCtl& ctl) {
 #ifdef DSEL_STATS
   if (threadIdx.x == 0 && blockIdx.x < kStatsCtas) {
-    ctl.marks[11] = global_ns();
+    ctl.marks[11] = static_cast<unsigned long long>(clock64());
 #pragma unroll 1
     for (int i = 0; i < 16; ++i) g_stats[blockIdx.x * kStatsFields + i] = ctl.marks[i];
     if (blockIdx.x < kStatsCtas / 2) {   // per-chunk times in the upper half
@@ -677,7 +679,7 @@ __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem
     for (int j = 0; j < g.nch; ++j, c = next_chunk(c)) {
       wait_chunk(c);
 #ifdef DSEL_STATS
-      if (tid == 0) ctl.marks[24 + j] = global_ns();
+      if (tid == 0) ctl.marks[24 + j] = static_cast<unsigned long long>(clock64());
 #endif
 #pragma unroll
       for (int i = 0; i < VT; ++i) {

@@ -6,8 +6,9 @@ Run with the counter build selected, for example::
 
 It replays a CUDA graph of back-to-back calls on one workload (the shapes of
 ``bench.py``), then reads the phase timestamps that thread 0 of every CTA of the
-last launch kept (``%globaltimer``, ns) and prints, per phase, the median and the
-maximum over CTAs of the time since the CTA passed its grid-dependency wait:
+last launch kept (the SM's cycle counter, converted at the device's clock rate)
+and prints, per phase, the median and the maximum over CTAs of the time since the
+CTA passed its grid-dependency wait:
 
 - issue: the slice's bulk copies issued;
 - landed: the last chunk of the slice arrived and its vector maxima were counted;
@@ -35,6 +36,19 @@ import numpy as np
 PHASES = [(2, "issue"), (3, "landed"), (4, "sync #1"), (5, "threshold"), (6, "filter"), (7, "boundary"),
           (10, "counts"), (8, "ranks"), (9, "written")]
 STATS_CTAS = 8192
+
+
+def sm_clock_ghz(default: float = 1.965) -> float:
+    """The current SM clock of GPU 0 from NVML (the B200's 1965 MHz when unavailable)."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByIndex(0)
+        mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+        pynvml.nvmlShutdown()
+        return mhz / 1000.0 if mhz > 0 else default
+    except Exception:
+        return default
 
 
 def main(argv=None):
@@ -90,15 +104,16 @@ def main(argv=None):
     allst = np.array(T.dsel_debug_stats(STATS_CTAS), dtype=np.int64)
     marks, chunks = allst[:n], allst[STATS_CTAS // 2:STATS_CTAS // 2 + n]
     t0 = marks[:, 1]   # each CTA's grid-dependency wait
+    ghz = sm_clock_ghz()   # cycles per ns
     print(f"{w.name}: plan {plan['threads']} threads, clusters of {plan['cluster']}, {plan['stages']} chunks "
           f"per slice; {per_launch_us:.2f} us per launch in a graph of back-to-back launches; {n} CTAs")
     print(f"{'phase':<10} {'median us':>10} {'max us':>10}   (since each CTA's dependency wait)")
     for i, nm in PHASES:
-        d = [(marks[c, i] - t0[c]) / 1000.0 for c in range(n) if marks[c, i] > 0]
+        d = [(marks[c, i] - t0[c]) / ghz / 1000.0 for c in range(n) if marks[c, i] > 0]
         if d:
             print(f"{nm:<10} {statistics.median(d):>10.2f} {max(d):>10.2f}")
     for c in range(min(n, 4)):
-        land = [round(float(v - t0[c]) / 1000.0, 2) for v in chunks[c, 8:16] if v > 0]
+        land = [round(float(v - t0[c]) / ghz / 1000.0, 2) for v in chunks[c, 8:16] if v > 0]
         print(f"cta {c}: chunks landed at {land} us; threshold summary {int(marks[c, 14])}, "
               f"list entries {int(marks[c, 15])}")
 
