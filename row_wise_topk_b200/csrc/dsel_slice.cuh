@@ -5,32 +5,36 @@
 // "DeepSeek releases DeepSelect, a TopK kernel for sparse attention and sampling"
 // (method paragraph), laid out for the order in which the data lands:
 //
-//   A. threshold from a sample: the chunks are visited in a per-slice
-//      pseudo-random order, and the first ns of them are a random sample of the
-//      slice.  Either every CTA takes T_c, a lower edge of the k-th largest vector
-//      maximum of its own sample (k vectors hold an element >= T_c: a valid
-//      threshold for the whole row) and the cluster keeps the largest, or, when
-//      that would need too large a sample, the CTAs take the k'-th largest,
-//      k' = ceil(k / C), and the cluster keeps the smallest (C slices with k'
-//      such vectors each: again at least k).  One cluster barrier;
-//   B. filter: every vector is screened against T with packed compares (about
-//      ten instructions per 16-byte vector); the survivors go into the CTA's own
-//      candidate list, one segment per warp, and into a histogram of their keys;
-//   C. exact finish, shared by the cluster: the CTAs sum their histograms through
-//      distributed shared memory and refine the bin that holds the k-th entry
-//      (one cluster barrier per extra level) down to the boundary key K*, or to a
-//      bin that is selected whole.  Each CTA then counts its entries above K* and
-//      equal to it; after one more barrier every CTA knows how many entries each
-//      slice contributes, so it ranks its own selection in index order from a
-//      bitmap of its slice and writes it at its offset.  The entries equal to K*
-//      are taken in index order across the slices (the composite (value, index)
-//      order: value descending, lower index first among equals).
+//   A. threshold from the vector maxima: as each chunk lands, every 16-byte
+//      vector's largest key goes, as a 16-bit summary, into a table and into a
+//      histogram of fixed bins (16 summaries each, so every CTA of the cluster
+//      has the same bins).  After one cluster barrier the CTAs sum the histograms
+//      through distributed shared memory (coarse sums first, then the 16 fine
+//      bins of one coarse bin) and take T, the lower edge of the bin that holds
+//      the row's k-th largest vector maximum: at least k vectors hold an element
+//      >= T, so T is a valid threshold, and it is the tightest one these bins give;
+//   B. filter, dense in two steps: the vectors whose summary reaches T go into
+//      this warp's vector list (one ballot per vector slot), then their elements
+//      >= T, 32 vectors per warp step, into this warp's element list (which stays
+//      in index order) and the CTA's histogram of candidate keys;
+//   C. exact finish, shared by the cluster: after one cluster barrier the CTAs
+//      sum their candidate histograms the same way and refine the bin that holds
+//      the k-th entry (one cluster barrier per extra level) down to the boundary
+//      key K*, or to a bin that is selected whole.  Each CTA then counts its
+//      entries above K* and equal to it per block of 32 vectors; after one more
+//      cluster barrier every CTA knows how many entries each slice contributes, so
+//      it writes its own selection at its offset, ranked in index order from the
+//      block counts.  The entries equal to K* are taken in index order across the
+//      slices (the composite (value, index) order: value descending, lower index
+//      first among equals).
 //
 // When a candidate list overflows an exact fallback runs on the resident slices
 // (every CTA): histogram levels down to a single key, then ranks in index order
 // from bitmaps.  No wait depends on another CTA except the hardware cluster
-// barriers; the bulk-copy waits are bounded.  A CTA that has read a peer's shared
-// memory arrives at a last cluster barrier before it leaves.
+// barriers, which every CTA of a cluster passes equally often (each path is
+// chosen from cluster-wide values); the bulk-copy waits are bounded.  A CTA that
+// has read a peer's shared memory arrives at a last cluster barrier before it
+// leaves.
 #pragma once
 
 #include "dsel_resident.cuh"
