@@ -147,93 +147,6 @@ __device__ __forceinline__ void cluster_hist_sum(const int* h, int* hs, int C, c
   __syncthreads();
 }
 
-// NB consecutive ints of shared memory at p (16-, 8- or 4-byte loads).
-template <int NB>
-__device__ __forceinline__ void load_run(const int* p, int (&c)[NB]) {
-  if constexpr (NB % 4 == 0) {
-#pragma unroll
-    for (int i = 0; i < NB / 4; ++i) {
-      const int4 v = reinterpret_cast<const int4*>(p)[i];
-      c[4 * i] = v.x;
-      c[4 * i + 1] = v.y;
-      c[4 * i + 2] = v.z;
-      c[4 * i + 3] = v.w;
-    }
-  } else if constexpr (NB == 2) {
-    const int2 v = *reinterpret_cast<const int2*>(p);
-    c[0] = v.x;
-    c[1] = v.y;
-  } else {
-#pragma unroll
-    for (int i = 0; i < NB; ++i) c[i] = p[i];
-  }
-}
-
-// This thread's run of NB consecutive bins of a histogram (bins NB t .. NB t +
-// NB - 1), summed over the cluster's CTAs: the caller has passed a cluster
-// barrier after the histograms were complete.
-template <bool CLUSTER, int NB>
-__device__ __forceinline__ void hist_sum_run(const int* h, int (&c)[NB], int C, cg::cluster_group& cluster) {
-  const int* hp = h + threadIdx.x * NB;
-  load_run<NB>(hp, c);
-  if (CLUSTER) {
-#pragma unroll 1
-    for (int r = 1; r < C; ++r) {
-      int v[NB];
-      load_run<NB>(cluster.map_shared_rank(hp, (static_cast<int>(cluster.block_rank()) + r) % C), v);
-#pragma unroll
-      for (int i = 0; i < NB; ++i) c[i] += v[i];
-    }
-  }
-}
-
-// Bin of the need-th largest entry of a histogram held as consecutive runs of NB
-// bins per thread (bin 0 the largest keys): a CTA-wide scan, two CTA barriers.
-// bin = -1 when the histogram holds fewer than `need` entries.
-template <int THREADS, int NB>
-__device__ __forceinline__ BinHit cta_find_bin(const int (&c)[NB], int need, SliceCtl& ctl) {
-  constexpr int NW = THREADS / 32;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int s = 0;
-#pragma unroll
-  for (int i = 0; i < NB; ++i) s += c[i];
-  const int incl = warp_incl_scan(s, lane);
-  if (lane == 31) ctl.w_c[warp] = incl;
-  __syncthreads();
-  int total;
-  const int base = warp_prefix_of<NW>(ctl.w_c, warp, lane, total) + incl - s;
-  BinHit r;
-  if (total < need) {   // uniform in the CTA
-    __syncthreads();
-    r.bin = -1;
-    r.before = 0;
-    r.cnt = 0;
-    return r;
-  }
-  if (base < need && need <= base + s) {   // exactly one thread
-    int found = -1, before = base, cnt = 0;
-#pragma unroll
-    for (int i = 0; i < NB; ++i) {
-      if (found < 0) {
-        if (before + c[i] >= need) {
-          found = i;
-          cnt = c[i];
-        } else {
-          before += c[i];
-        }
-      }
-    }
-    ctl.bin = NB * tid + found;
-    ctl.before = before;
-    ctl.cnt = cnt;
-  }
-  __syncthreads();
-  r.bin = ctl.bin;
-  r.before = ctl.before;
-  r.cnt = ctl.cnt;
-  return r;
-}
-
 // Coarse sums of a histogram kept beside it for the two-stage search:
 // coarse[i] = fine[16 i] + ... + fine[16 i + 15], i < ncb.  The caller has made
 // the fine histogram complete with a CTA barrier, and publishes both with a
@@ -276,22 +189,55 @@ __device__ __forceinline__ int cluster_sum_at(const int* a, int i, int C, cg::cl
 // largest keys), summed over the cluster, in two stages: the coarse sums (ncb <=
 // THREADS bins of 16) locate the coarse bin, whose 16 fine bins then locate the
 // bin.  The caller has passed a cluster barrier after publishing both arrays.
-// Four CTA barriers; bin = -1 when the histogram holds fewer than `need` entries.
+// Two CTA barriers; bin = -1 when the histogram holds fewer than `need` entries.
+// With `fx`, every warp also reads the cluster's flags (OR) and largest key (max)
+// into fx[0], fx[1], those loads overlapping the search's own.
 template <int THREADS, bool CLUSTER>
 __device__ __forceinline__ BinHit cluster_find_bin(const int* fine, const int* coarse, int ncb, int need, int C,
-                                                   SliceCtl& ctl, cg::cluster_group& cluster) {
-  const int tid = threadIdx.x;
-  int c[1] = {tid < ncb ? cluster_sum_at<CLUSTER>(coarse, tid, C, cluster) : 0};
-  const BinHit cb = cta_find_bin<THREADS, 1>(c, need, ctl);
-  if (cb.bin < 0) return cb;   // uniform in the CTA
-  const int need2 = need - cb.before;
-  if (tid < 32) {   // one warp: the coarse bin's 16 fine bins
-    const int f = tid < 16 ? cluster_sum_at<CLUSTER>(fine, 16 * cb.bin + tid, C, cluster) : 0;
-    const int incl = warp_incl_scan(f, tid);
-    const int j = __ffs(__ballot_sync(0xffffffffu, tid < 16 && incl >= need2)) - 1;
-    if (tid == j) {
-      ctl.bin2 = 16 * cb.bin + j;
-      ctl.before2 = cb.before + incl - f;
+                                                   SliceCtl& ctl, cg::cluster_group& cluster,
+                                                   uint32_t* fx = nullptr) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  uint32_t f_or = 0u, k_max = 0u;
+  if (fx != nullptr && lane < C) {
+    const SliceCtl* pr = CLUSTER ? cluster.map_shared_rank(&ctl, lane) : &ctl;
+    f_or = static_cast<uint32_t>(pr->flags);
+    k_max = pr->kmax;
+  }
+  const int c = tid < ncb ? cluster_sum_at<CLUSTER>(coarse, tid, C, cluster) : 0;
+  if (fx != nullptr) {
+    fx[0] = __reduce_or_sync(0xffffffffu, f_or);
+    fx[1] = __reduce_max_sync(0xffffffffu, k_max);
+  }
+  // the coarse bins, one per thread: a CTA-wide scan finds the one that holds the
+  // need-th entry; the warp holding it then reads that bin's 16 fine bins before
+  // the second barrier
+  constexpr int NW = THREADS / 32;
+  const int warp = tid >> 5;
+  const int incl = warp_incl_scan(c, lane);
+  if (lane == 31) ctl.w_c[warp] = incl;
+  __syncthreads();
+  int total;
+  const int base = warp_prefix_of<NW>(ctl.w_c, warp, lane, total) + incl - c;
+  if (total < need) {   // uniform in the CTA
+    __syncthreads();
+    BinHit r;
+    r.bin = -1;
+    r.before = 0;
+    r.cnt = 0;
+    return r;
+  }
+  const unsigned wb = __ballot_sync(0xffffffffu, base < need && need <= base + c);
+  if (wb != 0u) {   // this warp holds the coarse bin (thread `src` of it)
+    const int src = __ffs(wb) - 1;
+    const int cb = __shfl_sync(0xffffffffu, tid, src);
+    const int cbefore = __shfl_sync(0xffffffffu, base, src);
+    const int need2 = need - cbefore;
+    const int f = lane < 16 ? cluster_sum_at<CLUSTER>(fine, 16 * cb + lane, C, cluster) : 0;
+    const int fincl = warp_incl_scan(f, lane);
+    const int j = __ffs(__ballot_sync(0xffffffffu, lane < 16 && fincl >= need2)) - 1;
+    if (lane == j) {
+      ctl.bin2 = 16 * cb + j;
+      ctl.before2 = cbefore + fincl - f;
       ctl.cnt2 = f;
     }
   }
@@ -720,29 +666,25 @@ __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem
   sl_sync<CLUSTER>(cluster);   // every CTA's vector-maximum histogram, flags and largest key are final
   sl_mark(ctl, 4);
   if ((ctl.flags & 4) && tid < g.nch) mbar_wait(smem_u32(&bars[tid]), 0u);   // a copy may still be landing
+  // T: the lowest summary of the bin that holds the k-th largest vector maximum of
+  // the row (at least k vectors hold an element >= T: a valid threshold), or 0
+  // when the row has fewer than k vectors.  The same step reads the cluster's
+  // flags and largest key.
+  uint32_t t16 = 0u;
   int flags;
   uint32_t top;   // the row's largest key
-  if (CLUSTER) {
-    const SliceCtl* pr = cluster.map_shared_rank(&ctl, lane < g.C ? lane : 0);
-    flags = static_cast<int>(__reduce_or_sync(0xffffffffu, lane < g.C ? static_cast<unsigned>(pr->flags) : 0u));
-    top = __reduce_max_sync(0xffffffffu, lane < g.C ? pr->kmax : 0u);
-  } else {
-    flags = ctl.flags;
-    top = ctl.kmax;
+  {
+    uint32_t fx[2];
+    const BinHit bh = cluster_find_bin<THREADS, CLUSTER>(hv, hvc, kSlVBins / 16, k, g.C, ctl, cluster, fx);
+    if (bh.bin >= 0) t16 = static_cast<uint32_t>(kSlVBins - 1 - bh.bin) << 4;
+    flags = static_cast<int>(fx[0]);
+    top = fx[1];
   }
   if ((flags & 1) && !p.nan_flag) nan_trap();   // the pages' default NaN policy
   if (flags & 1) {   // flag mode: the row's NaN sentinel
     if (leader) write_sentinel_row<DT, THREADS>(p, g.row, DSEL_IDX_NAN);
     if (CLUSTER) cluster.sync();   // the peers have read this CTA's control block
     return;
-  }
-  // T: the lowest summary of the bin that holds the k-th largest vector maximum of
-  // the row (at least k vectors hold an element >= T: a valid threshold), or 0
-  // when the row has fewer than k vectors
-  uint32_t t16 = 0u;
-  {
-    const BinHit bh = cluster_find_bin<THREADS, CLUSTER>(hv, hvc, kSlVBins / 16, k, g.C, ctl, cluster);
-    if (bh.bin >= 0) t16 = static_cast<uint32_t>(kSlVBins - 1 - bh.bin) << 4;
   }
   const uint32_t t_row = DT == DSEL_BF16 ? t16 : (t16 << 16);
   const int sb = res_shift(top - t_row);   // one key per bin for bfloat16 when the range allows
@@ -811,15 +753,11 @@ __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem
   __syncthreads();
   coarse_sums<THREADS>(hc, hcc, kSlBins / 16);
   sl_sync<CLUSTER>(cluster);   // every CTA's candidate histogram and list are final
-  if (CLUSTER) {
-    const SliceCtl* pr = cluster.map_shared_rank(&ctl, lane < g.C ? lane : 0);
-    flags = static_cast<int>(__reduce_or_sync(0xffffffffu, lane < g.C ? static_cast<unsigned>(pr->flags) : 0u));
-  } else {
-    flags = ctl.flags;
-  }
-  if (flags & 2) {   // a segment overflowed: every CTA selects exactly on its resident slice
-    slice_exact<DT, THREADS, CLUSTER>(p, smem, g.row, g.lo, g.n_sl, g.C, g.crank, t_row, top, cluster);
-    return;
+  {   // the block counters of the ranking (in the dead summary table); the search's
+      // barriers order this before the count pass (the fallback clears its own bitmaps)
+    int* bz = reinterpret_cast<int*>(smem + p.off_tab);
+#pragma unroll 1
+    for (int i = tid; i < 2 * g.nch * (kSlChunkVecs / 32); i += THREADS) bz[i] = 0;
   }
 
   // ---- C. the boundary: histogram levels summed over the cluster ----
@@ -835,7 +773,13 @@ __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem
   uint32_t kb;    // else the boundary key K*: every key > K*, and ties in index order
 #pragma unroll 1
   for (int level = 0;; ++level) {
-    const BinHit bh = cluster_find_bin<THREADS, CLUSTER>(h, hcs, kSlBins / 16, need, g.C, ctl, cluster);
+    uint32_t fx[2];
+    const BinHit bh = cluster_find_bin<THREADS, CLUSTER>(h, hcs, kSlBins / 16, need, g.C, ctl, cluster,
+                                                         level == 0 ? fx : nullptr);
+    if (level == 0 && (fx[0] & 2u)) {   // a list overflowed (uniform): exact selection on the resident slices
+      slice_exact<DT, THREADS, CLUSTER>(p, smem, g.row, g.lo, g.n_sl, g.C, g.crank, t_row, top, cluster);
+      return;
+    }
     if (bh.bin < 0) {   // cannot happen (the bins hold the row's entries >= lo): select from lo
       all_bin = true;
       kb = lo;
@@ -887,9 +831,6 @@ __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem
   int* bt = ba + nblk;                                   // [nblk] entries equal to the boundary key
   int* sa = bt + nblk;                                   // [nblk] the owning warp's running counts at
   int* st = sa + nblk;                                   //        the block's first entry
-#pragma unroll 1
-  for (int i = tid; i < 2 * nblk; i += THREADS) ba[i] = 0;
-  __syncthreads();
   auto kinds = [&](uint32_t kk, bool& a, bool& t) {
     a = all_bin ? kk >= kb : kk > kb;
     t = !all_bin && kk == kb;
