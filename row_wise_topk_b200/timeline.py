@@ -1,4 +1,5 @@
-"""Phase timeline of the slice kernel, from the counter build of the library.
+"""Phase timeline of the slice kernel (or the streaming kernel's counters), from the
+counter build of the library.
 
 Run with the counter build selected, for example::
 
@@ -23,7 +24,11 @@ CTA passed its grid-dependency wait:
 
 Also printed: the chunk arrival times of the first CTAs and, per CTA, the
 threshold summary and the candidate-list length.  The counter build only adds
-timestamps kept in shared memory and written out when each CTA ends.
+timestamps kept in shared memory and written out when each CTA ends.  For a
+workload that takes the streaming kernel it prints that kernel's counters
+instead: time in the stream of rounds (and in block waits and compactions), in
+the final phase, rounds, compactions, candidates appended, vectors given the
+exact test and restarted passes.
 """
 from __future__ import annotations
 
@@ -51,6 +56,38 @@ def sm_clock_ghz(default: float = 1.965) -> float:
         return default
 
 
+def stream_counters(T, w, plan, per_launch_us, ghz):
+    """The streaming kernel's per-CTA counters of the last launch: medians over CTAs."""
+    n = min(w.rows * plan["cluster"] * plan["groups"], STATS_CTAS)
+    st = np.array(T.dsel_debug_stats(n), dtype=np.int64)
+    us = lambda c: c / ghz / 1000.0
+    print(f"{w.name}: streaming kernel, {plan['threads']} threads, clusters of {plan['cluster']}, "
+          f"{plan['groups']} cluster(s) per row; {per_launch_us:.2f} us per launch in a graph of back-to-back "
+          f"launches; {n} CTAs (medians over CTAs)")
+    rows = [("stream phase (rounds) us", us(st[:, 0])), ("  of it waiting for blocks us", us(st[:, 14])),
+            ("  of it compacting us", us(st[:, 2])), ("final phase us", us(st[:, 1])), ("total us", us(st[:, 15])),
+            ("rounds", st[:, 6]), ("compactions", st[:, 3]), ("candidates appended", st[:, 4]),
+            ("vectors given the exact test", st[:, 5]), ("passes restarted (uncertified seed)", st[:, 7])]
+    for name, v in rows:
+        print(f"{name:<38} {statistics.median(v.tolist()):>12.2f} {max(v.tolist()):>12.2f} (max)")
+    # per-round steps of CTA 0 (lane 0 of each warp): [warp][round][event], cycles since its start
+    import ctypes
+    buf = (ctypes.c_uint64 * (16 * 12 * 10))()
+    if T.lib.dsel_debug_stats(ctypes.cast(buf, ctypes.c_void_p), -1, None) != 0:
+        return
+    tr = np.array(buf[:], dtype=np.uint64).astype(np.int64).reshape(16, 12, 10)
+    steps = [(0, 8, "wait"), (8, 1, "screen"), (7, 2, "exact test + append"), (2, 3, "refill + count barrier"),
+             (3, 4, "overflow"), (4, 5, "compaction")]
+    print("CTA 0, rounds 1..9, median over warps (us):")
+    print("round " + " ".join(f"{nm:>22}" for _, _, nm in steps))
+    for r in range(1, 10):
+        cols = []
+        for a, b, _ in steps:
+            d = [tr[wp, r, b] - tr[wp, r, a] for wp in range(16) if tr[wp, r, a] > 0 and tr[wp, r, b] > 0]
+            cols.append(f"{us(statistics.median(d)):>22.2f}" if d else f"{'-':>22}")
+        print(f"{r:>5} " + " ".join(cols))
+
+
 def main(argv=None):
     import torch
 
@@ -71,8 +108,8 @@ def main(argv=None):
     dt = T.DSEL_BF16 if w.dtype == "bf16" else T.DSEL_F32
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     st, plan = T.dsel_plan_for(dt, w.rows, w.row_stride, w.k, w.sorted_index, num_sms=sms)
-    if plan["kernel"] != T.DSEL_KERNEL_SLICE:
-        raise SystemExit(f"{w.name} does not take the slice kernel (plan {plan})")
+    if plan["kernel"] not in (T.DSEL_KERNEL_SLICE, T.DSEL_KERNEL_STREAM):
+        raise SystemExit(f"{w.name} takes neither the slice nor the streaming kernel (plan {plan})")
     s = torch.cuda.Stream()
 
     def call(i):
@@ -100,11 +137,14 @@ def main(argv=None):
     torch.cuda.synchronize()
     per_launch_us = e0.elapsed_time(e1) / 24 * 1000.0
 
+    ghz = sm_clock_ghz()   # cycles per ns
+    if plan["kernel"] == T.DSEL_KERNEL_STREAM:
+        stream_counters(T, w, plan, per_launch_us, ghz)
+        return
     n = min(w.rows * plan["cluster"], STATS_CTAS // 2)
     allst = np.array(T.dsel_debug_stats(STATS_CTAS), dtype=np.int64)
     marks, chunks = allst[:n], allst[STATS_CTAS // 2:STATS_CTAS // 2 + n]
     t0 = marks[:, 1]   # each CTA's grid-dependency wait
-    ghz = sm_clock_ghz()   # cycles per ns
     print(f"{w.name}: plan {plan['threads']} threads, clusters of {plan['cluster']}, {plan['stages']} chunks "
           f"per slice; {per_launch_us:.2f} us per launch in a graph of back-to-back launches; {n} CTAs")
     print(f"{'phase':<10} {'median us':>10} {'max us':>10}   (since each CTA's dependency wait)")
