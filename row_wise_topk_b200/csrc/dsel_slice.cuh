@@ -114,6 +114,33 @@ __device__ __forceinline__ uint32_t key16(uint32_t key) {
   return DT == DSEL_BF16 ? key : (key >> 16);
 }
 
+// Largest key of a whole vector, without a NaN test: NaN-propagating packed
+// maxima, folded into the thread's running accumulator `nacc`, which is tested once
+// when the slice is done (a row with a NaN is flagged whole, so the key of a vector
+// holding one is never used).
+template <int DT>
+__device__ __forceinline__ uint32_t vec_max_key_fast(const uint4& x, uint32_t& nacc) {
+  using E = Elem<DT>;
+  if (DT == DSEL_BF16) {
+    const uint32_t m2 = bf16x2_max_nan(bf16x2_max_nan(x.x, x.y), bf16x2_max_nan(x.z, x.w));
+    nacc = bf16x2_max_nan(nacc, m2);
+    const uint32_t m1 = bf16x2_max_nan(m2, __byte_perm(m2, 0u, 0x1032u));   // both halves: the larger
+    return E::key(m1 & 0xFFFFu);
+  } else {
+    const float m = f32_max_nan(f32_max_nan(__uint_as_float(x.x), __uint_as_float(x.y)),
+                                f32_max_nan(__uint_as_float(x.z), __uint_as_float(x.w)));
+    nacc = __float_as_uint(f32_max_nan(__uint_as_float(nacc), m));
+    return E::key(__float_as_uint(m));
+  }
+}
+
+// True when the accumulator of vec_max_key_fast saw a NaN.
+template <int DT>
+__device__ __forceinline__ bool nacc_is_nan(uint32_t nacc) {
+  using E = Elem<DT>;
+  return DT == DSEL_BF16 ? (E::is_nan(nacc & 0xFFFFu) || E::is_nan(nacc >> 16)) : E::is_nan(nacc);
+}
+
 // Largest key of the first `valid` elements of a vector (all of them when valid
 // >= PV); true on a NaN among them.
 template <int DT>
@@ -622,6 +649,7 @@ __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem
   int* hv = hist;                  // [kSlVBins]: vector maxima
   int* hc = hist + kSlVBins;       // [kSlBins]: candidate keys
   bool tnan = false;
+  uint32_t nacc = 0u;              // NaN-propagating maximum of every whole vector
   uint32_t kmax_c = 0u;            // largest key of the slice
   {
     int c = static_cast<int>(pc);
@@ -636,7 +664,12 @@ __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem
         const int v = vec_of(c, i);
         const int valid = valid_of(v);
         uint32_t s16 = 0u;
-        if (valid > 0) {
+        if (valid >= PV) {
+          const uint32_t key = vec_max_key_fast<DT>(load_vec(v), nacc);
+          s16 = key16<DT>(key);
+          kmax_c = max(kmax_c, key);
+          atomicAdd(&hv[kSlVBins - 1 - static_cast<int>(s16 >> 4)], 1);
+        } else if (valid > 0) {   // the slice's last vector, cut short
           uint32_t key = 0u;
           if (vec_max_valid<DT>(load_vec(v), valid, key)) {
             tnan = true;
@@ -646,10 +679,11 @@ __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem
             atomicAdd(&hv[kSlVBins - 1 - static_cast<int>(s16 >> 4)], 1);
           }
         }
-        vkm[v] = static_cast<uint16_t>(s16);   // 0: no element (NaN or past the end)
+        vkm[v] = static_cast<uint16_t>(s16);   // 0: no element (past the end, or a cut vector with a NaN)
       }
     }
   }
+  tnan |= nacc_is_nan<DT>(nacc);
   {
     const int f = (__any_sync(0xffffffffu, tnan) ? 1 : 0) | (__any_sync(0xffffffffu, late) ? 4 : 0);
     const uint32_t wk = __reduce_max_sync(0xffffffffu, kmax_c);
