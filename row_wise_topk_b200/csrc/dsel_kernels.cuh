@@ -1360,6 +1360,7 @@ __global__ void __launch_bounds__(THREADS, kThreads / THREADS) topk_stream_kerne
           if (bit < 64) pend.w[0] |= static_cast<uint64_t>(kb) << bit;
           else pend.w[1] |= static_cast<uint64_t>(kb) << (bit - 64);
         }
+        DSEL_TR(r, 6);
         // one reservation per warp for the round: a scan and one shared atomic
         const int mine = pend.count();
         const int incl = warp_incl_scan(mine, lane);

@@ -635,9 +635,27 @@ __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem
   auto load_vec = [&](int v) -> uint4 { return *reinterpret_cast<const uint4*>(smem + static_cast<size_t>(v) * kVecBytes); };
   auto valid_of = [&](int v) -> int { return static_cast<int>(g.n_sl) - v * PV; };
   bool late = false;
+#ifdef DSEL_STATS
+  int st_tries = 0;   // try_wait calls of this thread (counter builds)
+  auto wait_chunk = [&](int c) {
+    const uint32_t bar = smem_u32(&bars[c]);
+    ++st_tries;
+    if (mbar_try_wait(bar, 0u)) return;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, 0u)) {
+      ++st_tries;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        atomicExch(&g_device_status, DSEL_ERR_DEVICE_TIMEOUT);
+        late = true;
+        return;
+      }
+    }
+  };
+#else
   auto wait_chunk = [&](int c) {
     if (!mbar_wait(smem_u32(&bars[c]), 0u)) late = true;
   };
+#endif
   auto next_chunk = [&](int c) -> int {   // the chunk after c in the visiting order
     const uint32_t t = static_cast<uint32_t>(c) + pa;
     return static_cast<int>(t >= static_cast<uint32_t>(g.nch) ? t - static_cast<uint32_t>(g.nch) : t);
@@ -684,6 +702,9 @@ __device__ __forceinline__ void slice_body(const KParams& p, unsigned char* smem
     }
   }
   tnan |= nacc_is_nan<DT>(nacc);
+#ifdef DSEL_STATS
+  if (lane == 0) atomicAdd(&ctl.marks[13], static_cast<unsigned long long>(st_tries));   // per warp (lane 0)
+#endif
   {
     const int f = (__any_sync(0xffffffffu, tnan) ? 1 : 0) | (__any_sync(0xffffffffu, late) ? 4 : 0);
     const uint32_t wk = __reduce_max_sync(0xffffffffu, kmax_c);

@@ -76,15 +76,15 @@ def stream_counters(T, w, plan, per_launch_us, ghz):
     if T.lib.dsel_debug_stats(ctypes.cast(buf, ctypes.c_void_p), -1, None) != 0:
         return
     tr = np.array(buf[:], dtype=np.uint64).astype(np.int64).reshape(16, 12, 10)
-    steps = [(0, 8, "wait"), (8, 1, "screen"), (7, 2, "exact test + append"), (2, 3, "refill + count barrier"),
-             (3, 4, "overflow"), (4, 5, "compaction")]
+    steps = [(0, 8, "wait"), (8, 1, "screen"), (7, 6, "exact test"), (6, 2, "append"),
+             (2, 3, "refill + count barrier"), (3, 4, "overflow"), (4, 5, "compaction")]
     print("CTA 0, rounds 1..9, median over warps (us):")
-    print("round " + " ".join(f"{nm:>22}" for _, _, nm in steps))
+    print("round " + " ".join(f"{nm:>14}" for _, _, nm in steps))
     for r in range(1, 10):
         cols = []
         for a, b, _ in steps:
             d = [tr[wp, r, b] - tr[wp, r, a] for wp in range(16) if tr[wp, r, a] > 0 and tr[wp, r, b] > 0]
-            cols.append(f"{us(statistics.median(d)):>22.2f}" if d else f"{'-':>22}")
+            cols.append(f"{us(statistics.median(d)):>14.2f}" if d else f"{'-':>14}")
         print(f"{r:>5} " + " ".join(cols))
 
 
@@ -155,7 +155,7 @@ def main(argv=None):
     for c in range(min(n, 4)):
         land = [round(float(v - t0[c]) / ghz / 1000.0, 2) for v in chunks[c, 8:16] if v > 0]
         print(f"cta {c}: chunks landed at {land} us; threshold summary {int(marks[c, 14])}, "
-              f"list entries {int(marks[c, 15])}")
+              f"list entries {int(marks[c, 15])}, chunk-wait polls (lane 0 of each warp) {int(marks[c, 13])}")
 
 
 if __name__ == "__main__":
