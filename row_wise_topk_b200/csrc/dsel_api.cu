@@ -246,7 +246,9 @@ template <int DT>
 int run_resident(const KParams& base, int64_t rows, cudaStream_t st, DevInfo* di) {
   auto rk = topk_resident_kernel<DT>;
   if (!di->res_attrs_set[DT]) {
-    if (cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) != cudaSuccess)
+    if (cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) != cudaSuccess ||
+        cudaFuncSetAttribute(rk, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
+            cudaSuccess)
       return DSEL_ERR_CUDA;
     di->res_attrs_set[DT] = true;
   }
@@ -254,10 +256,12 @@ int run_resident(const KParams& base, int64_t rows, cudaStream_t st, DevInfo* di
   KParams kp = base;
   kp.off_bars = rl.bars;
   kp.off_hist = rl.hist;
-  kp.off_tab = rl.tab;
+  kp.off_cv = rl.el;
+  kp.off_tab = rl.vl;
   kp.off_cb = rl.cb;
   kp.off_ci = rl.ci;
   kp.off_ctl = rl.ctl;
+  kp.seg = rl.seg;
   if (rows > 0x7FFFFFFF) return DSEL_ERR_ROWS;
   if (launch_cluster(rk, unsigned(rows), kResThreads, 1, rl.total, st, kp) != cudaSuccess) return DSEL_ERR_CUDA;
   return DSEL_OK;

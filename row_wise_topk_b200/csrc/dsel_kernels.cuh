@@ -169,9 +169,9 @@ __device__ __noinline__ void write_short_row(const KParams& p, int64_t row, int6
 // Float32 throughout; each thread sums a contiguous chunk, so prefix sums are
 // the chunk's running sum on top of a block scan of the chunk sums.
 // ---------------------------------------------------------------------------
-template <int THREADS>
+template <int THREADS, class CtlT>
 __device__ __noinline__ void sample_draw(const KParams& p, int64_t row, const uint32_t* zb, const uint32_t* ci,
-                                         int m, Ctl& ctl) {
+                                         int m, CtlT& ctl) {
   constexpr int NW = THREADS / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (m <= 0) {   // uniform: nothing to draw from
@@ -267,9 +267,9 @@ __device__ __noinline__ void sample_draw(const KParams& p, int64_t row, const ui
 // order-preserving key gives it: sign clear above +inf, sign set below -inf) --
 // then padding; for a sampling call, the draw among the n entries, which are
 // checked for NaN first (the softmax has no meaning with one).
-template <int DT, int THREADS>
+template <int DT, int THREADS, class CtlT>
 __device__ __noinline__ void finish_short_row(const KParams& p, int64_t row, int64_t n,
-                                              typename Elem<DT>::bits_t* cb, uint32_t* ci, Ctl& ctl) {
+                                              typename Elem<DT>::bits_t* cb, uint32_t* ci, CtlT& ctl) {
   const bool sampling = DT == DSEL_F32 && p.token_out != nullptr;
   if (p.order != DSEL_ORDER_VALUE && !sampling) {
     write_short_row<DT, THREADS>(p, row, n);

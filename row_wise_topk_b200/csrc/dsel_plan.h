@@ -1,6 +1,7 @@
 // Host-side launch planner for the row-wise TopK kernels.  Pure C++: no CUDA call,
 // so it is unit-tested on machines without a GPU through dsel_plan().
 #pragma once
+#include <algorithm>
 #include <cstdint>
 
 #include "../../include/dsel.h"
@@ -123,34 +124,64 @@ inline SmemLayout stream_layout(int64_t stages, int64_t block, int64_t capacity,
   return l;
 }
 
-// Row-resident kernel: the row, one mbarrier per 4 KB chunk (256 threads x 16
-// bytes), three 1024-bin histograms, the scan table ([8 rounds][8 warps] totals,
-// then [8 warps][8 rounds] offsets), candidate arrays of next_pow2(k) entries
-// (value order and the sampling step sort there) and the control block.
+// Row-resident kernel: the row; one mbarrier per 4 KB chunk (256 threads x 16
+// bytes); two 1024-bin histograms followed by the per-warp candidate lists (16-bit
+// row indices, at least 4 KB: the exact fallback keeps a third histogram there);
+// the row's candidate vectors (16-bit vector indices; the fallback's 512-byte
+// scan table in the same space); candidate arrays of next_pow2(k) entries (value
+// order and the sampling step sort there); the control block.  The lists take
+// what shared memory is left below the size that keeps the most CTAs on an SM (at
+// most four: 256 threads of at most 64 registers), and no more than a warp can
+// fill (its share of the row's vectors, every element a candidate).
+constexpr int kResCtlBytes = 1024;
+constexpr int kResMaxCtasPerSm = 4;
+constexpr int kResMinListBytes = 4096;
+constexpr int64_t kSmemPerSm = 228 * 1024;        // B200: shared memory per SM
+constexpr int64_t kSmemReservedPerCta = 1024;     // reserved by the system for every resident CTA
+
 struct ResLayout {
-  uint32_t bars, hist, tab, cb, ci, ctl, total;
+  uint32_t bars, hist, el, vl, cb, ci, ctl, total;
+  int32_t seg;   // list entries per warp
 };
 
 inline ResLayout resident_layout(int64_t row_stride, int32_t k, int eb) {
   auto up = [](int64_t v, int64_t a) { return (v + a - 1) / a * a; };
   const int vpt = kResRowBytes / (kResThreads * kVecBytes);
-  const int threads = kResThreads;
-  ResLayout l{};
-  int64_t off = up(row_stride * eb, 128);
-  l.bars = uint32_t(off);
-  off += up(int64_t(vpt) * 8, 16);
-  l.hist = uint32_t(off);
-  off += 3 * 1024 * 4;
-  l.tab = uint32_t(off);
-  off += 2 * int64_t(vpt) * (threads / 32) * 4;
+  const int nw = kResThreads / 32;
+  const int pv = kVecBytes / eb;
+  const int64_t nvec = (row_stride + pv - 1) / pv;
   const int64_t kp2 = next_pow2(k);
+  const int64_t row = up(row_stride * eb, 128);
+  const int64_t bars = up(int64_t(vpt) * 8, 16);
+  const int64_t hist = 2 * 1024 * 4;
+  const int64_t vl = std::max<int64_t>(up(nvec * 2, 16), 2 * int64_t(vpt) * nw * 4);
+  const int64_t cbb = up(kp2 * eb, 16), cib = up(kp2 * 4, 16);
+  const int64_t fixed = row + bars + hist + vl + cbb + cib + kResCtlBytes;
+  int occ = kResMaxCtasPerSm;
+  while (occ > 1 && occ * (fixed + kResMinListBytes + kSmemReservedPerCta) > kSmemPerSm) --occ;
+  const int64_t budget = kSmemPerSm / occ - kSmemReservedPerCta - fixed;
+  const int64_t full = 2 * nw * ((nvec + nw - 1) / nw) * pv;   // every element of a warp's share
+  int64_t el = std::min<int64_t>(std::max<int64_t>(budget, kResMinListBytes), std::max<int64_t>(full, kResMinListBytes));
+  const int64_t seg = el / (2 * nw);
+  el = up(seg * 2 * nw, 16);
+  ResLayout l{};
+  int64_t off = row;
+  l.bars = uint32_t(off);
+  off += bars;
+  l.hist = uint32_t(off);
+  off += hist;
+  l.el = uint32_t(off);   // right after the histograms: the fallback's third buffer
+  off += el;
+  l.vl = uint32_t(off);
+  off += vl;
   l.cb = uint32_t(off);
-  off += up(kp2 * eb, 16);
+  off += cbb;
   l.ci = uint32_t(off);
-  off += up(kp2 * 4, 16);
+  off += cib;
   l.ctl = uint32_t(off);
-  off += kSharedFixedBytes;
+  off += kResCtlBytes;
   l.total = uint32_t(off);
+  l.seg = int32_t(seg);
   return l;
 }
 

@@ -114,32 +114,7 @@ __device__ __forceinline__ uint32_t key16(uint32_t key) {
   return DT == DSEL_BF16 ? key : (key >> 16);
 }
 
-// Largest key of a whole vector, without a NaN test: NaN-propagating packed
-// maxima, folded into the thread's running accumulator `nacc`, which is tested once
-// when the slice is done (a row with a NaN is flagged whole, so the key of a vector
-// holding one is never used).
-template <int DT>
-__device__ __forceinline__ uint32_t vec_max_key_fast(const uint4& x, uint32_t& nacc) {
-  using E = Elem<DT>;
-  if (DT == DSEL_BF16) {
-    const uint32_t m2 = bf16x2_max_nan(bf16x2_max_nan(x.x, x.y), bf16x2_max_nan(x.z, x.w));
-    nacc = bf16x2_max_nan(nacc, m2);
-    const uint32_t m1 = bf16x2_max_nan(m2, __byte_perm(m2, 0u, 0x1032u));   // both halves: the larger
-    return E::key(m1 & 0xFFFFu);
-  } else {
-    const float m = f32_max_nan(f32_max_nan(__uint_as_float(x.x), __uint_as_float(x.y)),
-                                f32_max_nan(__uint_as_float(x.z), __uint_as_float(x.w)));
-    nacc = __float_as_uint(f32_max_nan(__uint_as_float(nacc), m));
-    return E::key(__float_as_uint(m));
-  }
-}
-
-// True when the accumulator of vec_max_key_fast saw a NaN.
-template <int DT>
-__device__ __forceinline__ bool nacc_is_nan(uint32_t nacc) {
-  using E = Elem<DT>;
-  return DT == DSEL_BF16 ? (E::is_nan(nacc & 0xFFFFu) || E::is_nan(nacc >> 16)) : E::is_nan(nacc);
-}
+// vec_max_key_fast and nacc_is_nan: dsel_resident.cuh.
 
 // Largest key of the first `valid` elements of a vector (all of them when valid
 // >= PV); true on a NaN among them.
