@@ -58,7 +58,8 @@ struct __align__(16) ResCtl {
   float smp_ec;                 //   weight sum of the kept candidates
   int flags;                    // bit 0: NaN seen, bit 1: a candidate list overflowed, bit 2: a wait gave up
   uint32_t kmax;                // the row's largest key
-  uint32_t lmin;                // its smallest vector maximum (rows of >= k vectors), else smallest key
+  uint32_t lmin;                // one less than its smallest vector maximum (rows of >= k vectors), else
+                                //   than its smallest key
   uint32_t t0;                  // the candidate threshold
   int bin, before, cnt;         // a bin search, broadcast to the CTA
   int tie_n;                    // members of a small boundary bin gathered so far
@@ -482,36 +483,59 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
   // ---- 2. vector maxima, the row's largest key, NaN; the smallest vector maximum
   //         (rows of at least k vectors) or the smallest key (shorter rows) ----
   const bool by_vec = nvec >= k;
+  const int nfull = n / (T * PV);   // rounds whose vectors are all whole
   uint32_t gk[VPT];   // largest key of vector i * T + tid; 0 = no vector (keys of numbers are >= 1)
-  uint32_t nacc = 0u, kmax = 0u, lmin = 0xFFFFFFFFu;
+  uint32_t nacc = 0u;
   bool nan = false, late = false;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     gk[i] = 0u;
-    if (i < nch) {
+    if (i < nfull) {
+      if (!mbar_wait(smem_u32(&bars[i]), 0u)) late = true;
+      gk[i] = vec_max_key_fast<DT>(load_vec(i * T + tid), nacc);
+    } else if (i < nch) {
       if (!mbar_wait(smem_u32(&bars[i]), 0u)) late = true;
       const int v = i * T + tid;
       if (v < nvec) {
         const uint4 x = load_vec(v);
         const int valid = n - v * PV;
-        uint32_t mx;
         if (valid >= PV) {
-          mx = vec_max_key_fast<DT>(x, nacc);
-          if (!by_vec) lmin = min(lmin, vec_min_key<DT>(x));
+          gk[i] = vec_max_key_fast<DT>(x, nacc);
         } else {   // the row's last vector, cut short
-          mx = 0u;
+          uint32_t mx = 0u;
 #pragma unroll 1
           for (int e = 0; e < valid; ++e) {
             const uint32_t b = vec_elem_dyn<DT>(x, e);
             nan |= E::is_nan(b);
-            const uint32_t kk = E::key(b);
-            mx = max(mx, kk);
-            if (!by_vec) lmin = min(lmin, kk);
+            mx = max(mx, E::key(b));
           }
+          gk[i] = mx;
         }
-        gk[i] = mx;
-        kmax = max(kmax, mx);
-        if (by_vec) lmin = min(lmin, mx);
+      }
+    }
+  }
+  // kmax, and lmin - 1 (the row has at least one key, which is >= 1: the CTA
+  // minimum does not wrap; a thread without vectors contributes 0 - 1 = 2^32 - 1)
+  uint32_t kmax = 0u, lmin = 0xFFFFFFFFu;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    kmax = max(kmax, gk[i]);
+    lmin = min(lmin, gk[i] - 1u);
+  }
+  if (!by_vec) {   // shorter rows: the smallest key instead
+    lmin = 0xFFFFFFFFu;
+#pragma unroll 1
+    for (int i = 0; i < nch; ++i) {
+      const int v = i * T + tid;
+      if (v < nvec) {
+        const uint4 x = load_vec(v);
+        const int valid = n - v * PV;
+        if (valid >= PV) {
+          lmin = min(lmin, vec_min_key<DT>(x) - 1u);
+        } else {
+#pragma unroll 1
+          for (int e = 0; e < valid; ++e) lmin = min(lmin, E::key(vec_elem_dyn<DT>(x, e)) - 1u);
+        }
       }
     }
   }
@@ -540,7 +564,7 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
     }
   }
   kmax = ctl.kmax;
-  lmin = ctl.lmin;
+  lmin = ctl.lmin + 1u;
 
   // ---- 3. the threshold T0: at least k elements are >= T0 ----
   if (by_vec) {
@@ -632,18 +656,19 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
       }
       const int cnt = __popc(m);
       const int incl = warp_incl_scan(cnt, lane);
-      int pos = wrun + incl - cnt;
-      const uint32_t e0 = v * PV;
-#pragma unroll
-      for (int e = 0; e < PV; ++e) {
-        if ((m >> e) & 1u) {
-          if (pos < seg) el[pos] = static_cast<uint16_t>(e0 + static_cast<uint32_t>(e));
-          ++pos;
+      const int tot = __shfl_sync(0xffffffffu, incl, 31);
+      if (wrun + tot <= seg) {   // warp-uniform; past it the list has overflowed and stays unwritten
+        uint16_t* dst = el + (wrun + incl - cnt);
+        const uint32_t e0 = v * PV;
+#pragma unroll 1
+        while (m != 0u) {
+          *dst++ = static_cast<uint16_t>(e0 + static_cast<uint32_t>(__ffs(m) - 1));
+          m &= m - 1u;
         }
       }
-      wrun += __shfl_sync(0xffffffffu, incl, 31);
+      wrun += tot;
     }
-    wcnt = min(wrun, seg);
+    wcnt = wrun <= seg ? wrun : 0;   // an overflowed list is incomplete: the fallback takes the row
     if (lane == 0 && wrun > seg) atomicOr(&ctl.flags, 2);
   }
   __syncwarp();   // the warp's list is visible to all its lanes
@@ -731,17 +756,20 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
   }
 
   // ---- 7. output slots in index order ----
-  auto kinds = [&](uint32_t kk, bool& a, bool& t) {
-    a = all_bin ? kk >= kb : kk > kb;
-    t = !all_bin && kk == kb;
-  };
-  {
+  {   // per-warp counts; each entry keeps its kind in the index's two spare bits
+      // (bit 15: above the boundary, bit 14: equal to it) for the write pass
     int na = 0, nt = 0;
 #pragma unroll 1
     for (int j0 = 0; j0 < wcnt; j0 += 32) {
       const int j = j0 + lane;
       bool a = false, t = false;
-      if (j < wcnt) kinds(key_of(j), a, t);
+      if (j < wcnt) {
+        const uint32_t gi = el[j];
+        const uint32_t kk = E::key(rowe[gi]);
+        a = all_bin ? kk >= kb : kk > kb;
+        t = !all_bin && kk == kb;
+        el[j] = static_cast<uint16_t>(gi | (a ? 0x8000u : 0u) | (t ? 0x4000u : 0u));
+      }
       na += __popc(__ballot_sync(0xffffffffu, a));
       nt += __popc(__ballot_sync(0xffffffffu, t));
     }
@@ -754,32 +782,30 @@ __global__ void __launch_bounds__(kResThreads, 4) topk_resident_kernel(const __g
   int total;
   int ra = warp_prefix_of<NW>(ctl.w_a, warp, lane, total);   // above-boundary entries of earlier warps
   int rt = warp_prefix_of<NW>(ctl.w_b, warp, lane, total);   // boundary-key entries of earlier warps
-  const int my_ties = all_bin ? 0 : need;
+  const int my_ties = all_bin ? 0 : need;   // boundary-key entries taken, the first ones in index order
   const bool to_smem = p.order == DSEL_ORDER_VALUE || p.token_out != nullptr;
   const int64_t obase = row * static_cast<int64_t>(k);
+  int32_t* o32 = static_cast<int32_t*>(p.indices_out) + obase;
+  int64_t* o64 = static_cast<int64_t*>(p.indices_out) + obase;
+  bits_t* ov = static_cast<bits_t*>(p.values_out) + obase;
+  const int mode = to_smem ? 0 : (p.index_i64 ? 2 : 1) | (p.return_value ? 4 : 0);
 #pragma unroll 1
-  for (int j0 = 0; j0 < wcnt; j0 += 32) {
+  for (int j0 = 0; j0 < wcnt; j0 += 32) {   // the same entries per lane as the count pass
     const int j = j0 + lane;
-    bool a = false, t = false;
-    uint32_t gi = 0u, b = 0u;
-    if (j < wcnt) {
-      gi = el[j];
-      b = rowe[gi];
-      kinds(E::key(b), a, t);
-    }
+    const uint32_t ent = j < wcnt ? el[j] : 0u;
+    const bool a = ent & 0x8000u, t = ent & 0x4000u;
+    const uint32_t gi = ent & 0x3FFFu;
     const unsigned am = __ballot_sync(0xffffffffu, a), tm = __ballot_sync(0xffffffffu, t);
     const int rank_t = rt + __popc(tm & below);   // boundary-key entries before this one
-    if (a || (t && rank_t < my_ties)) {
+    if (a || (t && rank_t < my_ties)) {   // its slot: entries selected before it (fewer than k)
       const int pos = ra + __popc(am & below) + min(rank_t, my_ties);
-      if (pos < k) {
-        if (to_smem) {
-          cb[pos] = static_cast<bits_t>(b);
-          ci[pos] = gi;
-        } else {
-          if (p.index_i64) static_cast<int64_t*>(p.indices_out)[obase + pos] = static_cast<int64_t>(gi);
-          else static_cast<int32_t*>(p.indices_out)[obase + pos] = static_cast<int32_t>(gi);
-          if (p.return_value) static_cast<bits_t*>(p.values_out)[obase + pos] = static_cast<bits_t>(b);
-        }
+      if (mode == 0) {
+        cb[pos] = rowe[gi];
+        ci[pos] = gi;
+      } else {
+        if (mode & 2) o64[pos] = static_cast<int64_t>(gi);
+        else o32[pos] = static_cast<int32_t>(gi);
+        if (mode & 4) ov[pos] = rowe[gi];
       }
     }
     ra += __popc(am);
