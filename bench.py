@@ -432,8 +432,10 @@ def run_ours(args, w, world, rank, local, pg):
             ev_a[i].record()
             step(i)
             ev_b[i].record()
-    plan = T.dsel_plan_for(dt, w.rows, w.row_stride, w.k, T.DSEL_ORDER_VALUE if sampling else w.sorted_index,
-                           num_sms=torch.cuda.get_device_properties(dev).multi_processor_count)[1]
+    st_plan, plan = T.dsel_plan_device(dt, w.rows, w.row_stride, w.k,
+                                       T.DSEL_ORDER_VALUE if sampling else w.sorted_index)
+    if st_plan != 0:
+        raise T.DselError(st_plan)
     launches_per_step = 1 + (1 if plan["groups"] > 1 else 0)
 
     # warm-up
@@ -668,8 +670,7 @@ def run_long_split(args, world, rank, local, pg):
     l1.record()
     torch.cuda.synchronize(dev)
     local_ms = l0.elapsed_time(l1) / reps
-    plan = T.dsel_plan_for(T.DSEL_F32, 1, shard_len, k, T.DSEL_ORDER_INDEX,
-                           num_sms=torch.cuda.get_device_properties(dev).multi_processor_count)[1]
+    plan = T.dsel_plan_device(T.DSEL_F32, 1, shard_len, k, T.DSEL_ORDER_INDEX)[1]
     local_launches = 1 + (1 if plan["groups"] > 1 else 0)
     shard_bytes = shard_len * 4 + k * (4 + 8)
     peak, peak_kind = hbm_peak()

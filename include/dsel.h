@@ -314,6 +314,16 @@ DSEL_API int dsel_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k,
 DSEL_API int dsel_plan_for(int dtype, int64_t rows, int64_t row_stride, int32_t k, int sorted_index,
                            int32_t num_sms, int32_t smem_optin, int32_t max_cluster, dsel_plan_t* out);
 
+/* The plan dsel_topk would use with this sorted_index on the current device (pass
+ * DSEL_ORDER_VALUE for the plan of dsel_topk_sample): dsel_plan_for with the
+ * device's SM count and opt-in shared memory, the slice kernel's cluster size the
+ * device can schedule, and streaming-kernel clusters above the portable 8 where the
+ * occupancy calculator says the device holds every cluster of the launch at once.
+ * Queries the device; launches nothing.  Returns DSEL_OK, DSEL_ERR_CUDA,
+ * DSEL_ERR_NULL for a NULL out, or a DSEL_ERR_* code for invalid arguments. */
+DSEL_API int dsel_plan_device(int dtype, int64_t rows, int64_t row_stride, int32_t k, int sorted_index,
+                              dsel_plan_t* out);
+
 /* Reads and clears the device-side status word that kernels set when a bounded
  * wait runs out (it should never happen).  Synchronises `stream`.  *status_out
  * receives 0 or DSEL_ERR_DEVICE_TIMEOUT.  Returns DSEL_OK or DSEL_ERR_CUDA. */

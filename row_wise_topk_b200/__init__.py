@@ -83,6 +83,8 @@ def _load() -> ctypes.CDLL:
     lib.dsel_plan_for.restype = c_int
     lib.dsel_plan_for.argtypes = [c_int, c_i64, c_i64, ctypes.c_int32, c_int, ctypes.c_int32, ctypes.c_int32,
                                   ctypes.c_int32, ctypes.POINTER(DselPlan)]
+    lib.dsel_plan_device.restype = c_int
+    lib.dsel_plan_device.argtypes = [c_int, c_i64, c_i64, ctypes.c_int32, c_int, ctypes.c_void_p]
     lib.dsel_plan.restype = c_int
     lib.dsel_plan.argtypes = [c_int, c_i64, c_i64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                               ctypes.c_int32, ctypes.POINTER(DselPlan)]
@@ -152,6 +154,13 @@ def dsel_plan_for(dtype: int, rows: int, row_stride: int, k: int, sorted_index: 
     p = DselPlan()
     st = lib.dsel_plan_for(dtype, rows, row_stride, k, sorted_index, num_sms, smem_optin, max_cluster,
                            ctypes.byref(p))
+    return st, p.as_dict()
+
+
+def dsel_plan_device(dtype: int, rows: int, row_stride: int, k: int, sorted_index: int) -> Tuple[int, dict]:
+    """The plan dsel_topk uses on the current device (DSEL_ORDER_VALUE: dsel_topk_sample's)."""
+    p = DselPlan()
+    st = lib.dsel_plan_device(dtype, rows, row_stride, k, sorted_index, ctypes.byref(p))
     return st, p.as_dict()
 
 

@@ -25,6 +25,8 @@ struct DevInfo {
   bool res_attrs_set[2] = {false, false};                                  // [dtype], resident kernel
   bool slice_attrs_set[4] = {false, false, false, false};                  // [dtype][shape], slice kernel
   int slice_cluster = 0;   // largest cluster the slice kernel launches with (16 when schedulable, else 8)
+  bool stream_fit_ready = false;
+  int32_t stream_fit[kSliceMaxCluster + 1] = {};   // streaming-kernel clusters of each size held at once
 };
 
 std::mutex g_mu;
@@ -242,6 +244,45 @@ int slice_cluster_limit(DevInfo* di) {
   return lim;
 }
 
+// For each cluster size above the portable 8: how many clusters of streaming
+// CTAs the device holds at once, for the largest configuration (512 threads, all
+// opt-in shared memory: one CTA per SM), so a lower bound for the others; 0 where
+// the query fails.
+const int32_t* stream_cluster_fit(DevInfo* di) {
+  if (di->stream_fit_ready) return di->stream_fit;
+  auto kc = topk_stream_kernel<DSEL_F32, kThreads>;
+  if (cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) == cudaSuccess &&
+      cudaFuncSetAttribute(kc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+    for (int c = kMaxCluster + 1; c <= kSliceMaxCluster; ++c) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(unsigned(c), 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = uint32_t(di->smem_optin);
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = unsigned(c);
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int nc = 0;
+      if (cudaOccupancyMaxActiveClusters(&nc, kc, &cfg) == cudaSuccess) di->stream_fit[c] = nc;
+    }
+  }
+  cudaGetLastError();   // a refused query leaves no sticky error
+  di->stream_fit_ready = true;
+  return di->stream_fit;
+}
+
+// The plan of a call on this device (sorted_index DSEL_ORDER_VALUE also stands for
+// the sampling call): the slice kernel up to its schedulable cluster size unless
+// the order is by value, the streaming kernel's larger clusters where they fit.
+int device_plan(DevInfo* di, int dtype, int64_t rows, int64_t row_stride, int32_t k, int sorted_index,
+                dsel_plan_t* pl) {
+  return make_plan_ex(dtype, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster,
+                      sorted_index == DSEL_ORDER_VALUE ? 0 : slice_cluster_limit(di), pl, stream_cluster_fit(di));
+}
+
 template <int DT>
 int run_resident(const KParams& base, int64_t rows, cudaStream_t st, DevInfo* di) {
   auto rk = topk_resident_kernel<DT>;
@@ -362,6 +403,19 @@ DSEL_API int dsel_plan_for(int dtype, int64_t rows, int64_t row_stride, int32_t 
                       sorted_index == DSEL_ORDER_VALUE ? 0 : kSliceMaxCluster, out);
 }
 
+DSEL_API int dsel_plan_device(int dtype, int64_t rows, int64_t row_stride, int32_t k, int sorted_index,
+                              dsel_plan_t* out) {
+  if (sorted_index < DSEL_ORDER_NONE || sorted_index > DSEL_ORDER_VALUE) return DSEL_ERR_ORDER;
+  if (out == nullptr) return DSEL_ERR_NULL;
+  std::lock_guard<std::mutex> lock(g_mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSEL_ERR_CUDA;
+  DevInfo* di = nullptr;
+  const int st = device_info(dev, &di);
+  if (st != DSEL_OK) return st;
+  return device_plan(di, dtype, rows, row_stride, k, sorted_index, out);
+}
+
 DSEL_API int dsel_topk(const void* x, int dtype, int64_t rows, int64_t row_stride, const int32_t* end,
                        int32_t k, int sorted_index, int return_value, int index_dtype, int nan_mode,
                        void* values_out, void* indices_out, void* stream) {
@@ -385,8 +439,7 @@ DSEL_API int dsel_topk(const void* x, int dtype, int64_t rows, int64_t row_strid
   st = device_info(dev, &di);
   if (st != DSEL_OK) return st;
   dsel_plan_t pl;
-  st = make_plan_ex(dtype, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster,
-                    sorted_index == DSEL_ORDER_VALUE ? 0 : slice_cluster_limit(di), &pl);
+  st = device_plan(di, dtype, rows, row_stride, k, sorted_index, &pl);
   if (st != DSEL_OK) return st;
 
   KParams kp = {};
@@ -435,7 +488,7 @@ DSEL_API int dsel_topk_sample(const void* x, int64_t rows, int64_t row_stride, c
   st = device_info(dev, &di);
   if (st != DSEL_OK) return st;
   dsel_plan_t pl;
-  st = make_plan_ex(DSEL_F32, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster, 0, &pl);
+  st = device_plan(di, DSEL_F32, rows, row_stride, k, DSEL_ORDER_VALUE, &pl);
   if (st != DSEL_OK) return st;
 
   KParams kp = {};
@@ -523,8 +576,7 @@ DSEL_API int dsel_topk_noalloc(const void* x, int dtype, int64_t rows, int64_t r
     g_noalloc_scratch_addr[dev] = ptr;
   }
   dsel_plan_t pl;
-  st = make_plan_ex(dtype, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster,
-                    sorted_index == DSEL_ORDER_VALUE ? 0 : slice_cluster_limit(di), &pl);
+  st = device_plan(di, dtype, rows, row_stride, k, sorted_index, &pl);
   if (st != DSEL_OK) return st;
 
   KParams kp = {};

@@ -66,7 +66,8 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
 }
 
 int make_plan_ex(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t num_sms,
-                 int32_t smem_optin, int32_t max_cluster, int32_t slice_cluster, dsel_plan_t* out) {
+                 int32_t smem_optin, int32_t max_cluster, int32_t slice_cluster, dsel_plan_t* out,
+                 const int32_t* cluster_fit) {
   int st = check_shape(dtype, rows, row_stride, k);
   if (st != DSEL_OK) return st;
   if (out == nullptr || num_sms < 1 || smem_optin < 48 * 1024 || max_cluster < 1)
@@ -175,6 +176,18 @@ int make_plan_ex(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t
   const int64_t max_groups =
       std::min<int64_t>(kMaxGroups, std::max<int64_t>(1, int64_t(kMaxCluster) * p.capacity / k));
   groups = std::min(groups, max_groups);
+  // a larger cluster (non-portable sizes) when the device holds every cluster of
+  // the launch at once and more CTAs (SMs) take part
+  if (cluster_fit != nullptr && splits > cluster) {
+    const int64_t cmax = std::min<int64_t>(splits, kSliceMaxCluster);
+    for (int64_t c = std::max<int64_t>(cluster, kMaxCluster) + 1; c <= cmax; ++c) {
+      const int64_t g = std::min<int64_t>(std::max<int64_t>(1, splits / c), max_groups);
+      if (rows * g <= cluster_fit[c] && c * g > cluster * groups) {
+        cluster = c;
+        groups = g;
+      }
+    }
+  }
   p.cluster = int(cluster);
   p.groups = int(groups);
 

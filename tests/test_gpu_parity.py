@@ -87,6 +87,31 @@ def test_plans_cover_split_and_merge(dtype, rows, stride, k):
         assert st == 0 and p["kernel"] == T.DSEL_KERNEL_STREAM and p["groups"] > 1
 
 
+@pytest.mark.parametrize("rows", [10, 14, 16])
+def test_split_rows_wide_clusters(rows):
+    """rows too long for the slice kernel, split over the streaming kernel's clusters:
+    past the portable 8 CTAs where the device holds every cluster of the launch at
+    once (16 rows: clusters of 9 on a 148-SM B200)"""
+    st, p = T.dsel_plan_device(T.DSEL_F32, rows, 1 << 20, 1024, T.DSEL_ORDER_INDEX)
+    assert st == 0 and p["kernel"] == T.DSEL_KERNEL_STREAM and 8 <= p["cluster"] <= 16
+    assert rows * p["cluster"] * p["groups"] <= torch.cuda.get_device_properties(0).multi_processor_count
+    w = W.random_small(23 + rows, "f32", rows, 1 << 20, 1024, dist="ties", sorted_index=1)
+    check(w, order=T.DSEL_ORDER_INDEX)
+    check(w, order=T.DSEL_ORDER_VALUE)
+
+
+def test_device_plan_matches_host_plan_below_eight():
+    """the device plan differs from the host planner only in the larger clusters"""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for args in [(T.DSEL_BF16, 64, 131072, 512, 1), (T.DSEL_F32, 256, 129280, 1024, 2),
+                 (T.DSEL_BF16, 4096, 16384, 512, 1), (T.DSEL_F32, 1, 1 << 28, 1000, 1)]:
+        st, dp = T.dsel_plan_device(*args)
+        hst, hp = T.dsel_plan_for(*args, num_sms=sms, max_cluster=8)
+        assert st == 0 and hst == 0
+        if dp["cluster"] <= 8 and dp["kernel"] != T.DSEL_KERNEL_SLICE:
+            assert dp == hp
+
+
 def test_all_rows_short():
     w = W.random_small(3, "bf16", 10, 16, 4096, dist="normal")
     check(w, order=1)
