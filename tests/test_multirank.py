@@ -178,3 +178,19 @@ def test_roofline_launch_time():
     # one launch per step: the timed region's average; two (stream + merge): the isolated mean
     assert bench.roofline_launch_ms(0.0225, 1, [0.0286, 0.0290]) == 0.0225
     assert abs(bench.roofline_launch_ms(0.5, 2, [0.2, 0.4]) - 0.3) < 1e-12
+
+
+def test_recorded_traffic_follows_the_kernel_sources(monkeypatch):
+    """roofline.traffic comes from the committed ncu record only while the kernel
+    sources hash to the ones it was captured on; any other hash reports null."""
+    import json
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)
+    for name, e in rec.items():
+        assert name in ("indexer", "indexer_varlen", "sampler_256_1024", "long_16_4096"), name
+        assert e["dram_bytes_per_launch"] > 0 and os.path.exists(os.path.join(bench.ROOT, "profiles", e["source"]))
+        want = e["dram_bytes_per_launch"] if e["kernel_hash"] == bench.kernel_hash() else None
+        assert bench.recorded_traffic(name) == want
+    monkeypatch.setattr(bench, "kernel_hash", lambda: "0000000000000000")
+    assert all(bench.recorded_traffic(name) is None for name in rec)
+    assert bench.recorded_traffic("no_such_workload") is None
