@@ -121,8 +121,13 @@ int make_plan_ex(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t
     // write, so batches needing many waves of slices go to the streaming kernel,
     // whose two CTAs per SM overlap one row's tail with the next row's loads
     if (cmin > 0 && rows * cmin <= kSliceMaxWaves * int64_t(num_sms)) {
+      // more slices than needed only to put idle SMs to work, and then at most the
+      // portable 8: a cluster of 16 ranks has the longer finish (one row of 129,280
+      // f32 logits: 10.3 us in 16 slices of 32 KB, 9.1 us in 8 of 64 KB; eight rows:
+      // 25.2 against 12.7 us); rows that need more than 8 slices to fit keep cmin
       int64_t c = std::max<int64_t>(1, num_sms / std::max<int64_t>(rows, 1));
-      c = std::min<int64_t>({c, slice_cluster, std::max<int64_t>(1, ceil_div(row_stride, kSliceMinElems))});
+      c = std::min<int64_t>({c, std::min<int64_t>(slice_cluster, kMaxCluster),
+                             std::max<int64_t>(1, ceil_div(row_stride, kSliceMinElems))});
       c = std::max(c, cmin);
       while (c > cmin && !fits(c)) --c;
       const int64_t ch = slice_chunks(row_stride, c, eb);

@@ -155,7 +155,7 @@ def test_plan_invariants(dtype, rows, stride, k):
             return ch <= 8 and lcap >= k + 2048
         assert fits(p["cluster"])
         assert p["cluster"] == 1 or not fits(p["cluster"] - 1) or \
-            (rows * p["cluster"] <= PEAK["num_sms"] and p["cluster"] <= -(-stride // 8192))
+            (rows * p["cluster"] <= PEAK["num_sms"] and p["cluster"] <= min(8, -(-stride // 8192)))
         return
     if rows >= PEAK["num_sms"] and stride * eb <= 32 * 1024:
         # rows that fit in shared memory: one 256-thread CTA per row holds the whole row
@@ -228,10 +228,14 @@ def test_plan_splits():
     # 64 indexer rows: two slices per row, each held in one CTA's shared memory
     p = T.dsel_plan(T.DSEL_BF16, 64, 131072, 512, **PEAK)[1]
     assert (p["kernel"], p["cluster"], p["groups"]) == (T.DSEL_KERNEL_SLICE, 2, 1)
-    # one or eight sampler rows: sixteen slices per row; 256 rows (several waves of
+    # one or eight sampler rows: eight slices per row (spreading a row further only to
+    # fill idle SMs stops at the portable cluster size); 256 rows (several waves of
     # slices): the streaming kernel
-    assert T.dsel_plan(T.DSEL_F32, 1, 129280, 50, **PEAK)[1]["cluster"] == 16
-    assert T.dsel_plan(T.DSEL_F32, 8, 129280, 1024, **PEAK)[1]["cluster"] == 16
+    assert T.dsel_plan(T.DSEL_F32, 1, 129280, 50, **PEAK)[1]["cluster"] == 8
+    assert T.dsel_plan(T.DSEL_F32, 8, 129280, 1024, **PEAK)[1]["cluster"] == 8
+    # a row that needs more than eight slices to fit still takes a larger cluster
+    p = T.dsel_plan(T.DSEL_F32, 1, 393216, 512, **PEAK)[1]   # 1.5 MB: twelve slices of 128 KB
+    assert (p["kernel"], p["cluster"]) == (T.DSEL_KERNEL_SLICE, 12)
     p = T.dsel_plan(T.DSEL_F32, 256, 129280, 1024, **PEAK)[1]
     assert p["kernel"] == T.DSEL_KERNEL_STREAM
     # a single 2^28 row uses several clusters
