@@ -123,7 +123,8 @@ typedef struct {
   int32_t threads;       /* threads per CTA: 512 (one CTA per SM); with at least as many rows as
                             SMs, 256 for the row-resident kernel (rows of at most 32 KB, four
                             CTAs per SM), 128 for other short rows (several CTAs per SM) or 256
-                            for long rows with k <= 1024 (two CTAs per SM) */
+                            for long rows with k <= 1024 (two CTAs per SM); the slice kernel:
+                            512 for slices of four 16 KB chunks or more, else 256 */
   int32_t cluster;       /* CTAs per thread-block cluster working on one row */
   int32_t groups;        /* clusters per row (> 1: split-row plan with a merge launch) */
   int32_t block;         /* B: elements per contiguous block visited in random order */
@@ -141,8 +142,9 @@ typedef struct {
                             whole row in shared memory (block = the 4 KB bulk-copy chunk,
                             round = row_stride, stages = chunks per row, b2 = 0), or
                             DSEL_KERNEL_SLICE: rows cut into `cluster` slices of at most 128 KB,
-                            one 256-thread CTA per slice holding it whole in shared memory, the
-                            slices of a row in one cluster (round = slice elements, block =
+                            one CTA per slice holding it whole in shared memory, the slices of
+                            a row in one cluster (up to 8 to fill idle SMs, up to 16 when the
+                            row needs that many slices) (round = slice elements, block =
                             elements per 16 KB bulk-copy chunk, stages = chunks per slice,
                             capacity = candidate-list entries of each CTA, b2 = 0); index
                             order and unspecified order only */
