@@ -185,7 +185,10 @@ DSEL_API int dsel_topk(const void* x, int dtype, int64_t rows, int64_t row_strid
  * uses a static device array of DSEL_NOALLOC_SCRATCH_BYTES that every GPU loading
  * the library holds until the process exits.  The call never calls cudaMalloc,
  * cudaFree or any allocating routine.
- *   - A call whose plan needs more scratch than that returns DSEL_ERR_SCRATCH_LIMIT
+ *   - It plans a long row's split as dsel_plan does (clusters of up to 8), not
+ *     with dsel_topk's split fitted to the device's cluster capacity, so the
+ *     scratch a call needs is known on the host: a call whose plan (dsel_plan's
+ *     workspace_bytes) needs more than the array returns DSEL_ERR_SCRATCH_LIMIT
  *     and launches nothing (on a 148-SM B200 this happens only for k >= 3640, on
  *     at most nine long rows split over several clusters).
  *   - The first call on a device, whatever its shape, looks up the array's
@@ -319,8 +322,9 @@ DSEL_API int dsel_plan_for(int dtype, int64_t rows, int64_t row_stride, int32_t 
 /* The plan dsel_topk would use with this sorted_index on the current device (pass
  * DSEL_ORDER_VALUE for the plan of dsel_topk_sample): dsel_plan_for with the
  * device's SM count and opt-in shared memory, the slice kernel's cluster size the
- * device can schedule, and streaming-kernel clusters above the portable 8 where the
- * occupancy calculator says the device holds every cluster of the launch at once.
+ * device can schedule, and a long row split over the streaming kernel's clusters
+ * (any size up to 16) and groups chosen for the most CTAs whose clusters the
+ * occupancy calculator says the device holds all at once (one wave).
  * Queries the device; launches nothing.  Returns DSEL_OK, DSEL_ERR_CUDA,
  * DSEL_ERR_NULL for a NULL out, or a DSEL_ERR_* code for invalid arguments. */
 DSEL_API int dsel_plan_device(int dtype, int64_t rows, int64_t row_stride, int32_t k, int sorted_index,

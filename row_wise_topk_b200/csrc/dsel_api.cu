@@ -244,16 +244,17 @@ int slice_cluster_limit(DevInfo* di) {
   return lim;
 }
 
-// For each cluster size above the portable 8: how many clusters of streaming
-// CTAs the device holds at once, for the largest configuration (512 threads, all
-// opt-in shared memory: one CTA per SM), so a lower bound for the others; 0 where
-// the query fails.
+// For each cluster size: how many clusters of streaming CTAs the device holds at
+// once, for the largest configuration (512 threads, all opt-in shared memory: one
+// CTA per SM), so a lower bound for the others; 0 where the query fails.  A split
+// row's plan keeps every cluster of its launch inside one wave with these counts.
 const int32_t* stream_cluster_fit(DevInfo* di) {
   if (di->stream_fit_ready) return di->stream_fit;
   auto kc = topk_stream_kernel<DSEL_F32, kThreads>;
+  di->stream_fit[1] = di->sms;
   if (cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, di->smem_optin) == cudaSuccess &&
       cudaFuncSetAttribute(kc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
-    for (int c = kMaxCluster + 1; c <= kSliceMaxCluster; ++c) {
+    for (int c = 2; c <= kSliceMaxCluster; ++c) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(unsigned(c), 1, 1);
       cfg.blockDim = dim3(kThreads, 1, 1);
@@ -276,7 +277,8 @@ const int32_t* stream_cluster_fit(DevInfo* di) {
 
 // The plan of a call on this device (sorted_index DSEL_ORDER_VALUE also stands for
 // the sampling call): the slice kernel up to its schedulable cluster size unless
-// the order is by value, the streaming kernel's larger clusters where they fit.
+// the order is by value; a split row over the streaming kernel's clusters and
+// groups that the device holds in one wave.
 int device_plan(DevInfo* di, int dtype, int64_t rows, int64_t row_stride, int32_t k, int sorted_index,
                 dsel_plan_t* pl) {
   return make_plan_ex(dtype, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster,
@@ -575,8 +577,12 @@ DSEL_API int dsel_topk_noalloc(const void* x, int dtype, int64_t rows, int64_t r
     if (cudaGetSymbolAddress(&ptr, dsel_noalloc_scratch) != cudaSuccess || ptr == nullptr) return DSEL_ERR_CUDA;
     g_noalloc_scratch_addr[dev] = ptr;
   }
+  // the portable split of a long row (clusters of up to 8, the split dsel_plan
+  // gives), not the one fitted to this device's cluster capacity: the scratch a
+  // call needs, and so whether it is refused, is known on the host before any launch
   dsel_plan_t pl;
-  st = device_plan(di, dtype, rows, row_stride, k, sorted_index, &pl);
+  st = make_plan_ex(dtype, rows, row_stride, k, di->sms, di->smem_optin, kMaxCluster,
+                    sorted_index == DSEL_ORDER_VALUE ? 0 : slice_cluster_limit(di), &pl, nullptr);
   if (st != DSEL_OK) return st;
 
   KParams kp = {};

@@ -184,16 +184,27 @@ int make_plan_ex(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t
   const int64_t max_groups =
       std::min<int64_t>(kMaxGroups, std::max<int64_t>(1, int64_t(kMaxCluster) * p.capacity / k));
   groups = std::min(groups, max_groups);
-  // a larger cluster (non-portable sizes) when the device holds every cluster of
-  // the launch at once and more CTAs (SMs) take part
-  if (cluster_fit != nullptr && splits > cluster) {
+  // On a device whose cluster capacity is known: the split with the most CTAs
+  // whose clusters the device holds all at once (non-portable sizes included),
+  // fewer groups first among equals.  A launch whose clusters need two waves
+  // takes about twice as long: sixteen rows of 2^24 f32 ran in 1,064 us in
+  // clusters of 8 (one group) and in 613 us in clusters of 4 (two groups).
+  if (cluster_fit != nullptr && splits > 1) {
+    int64_t bc = 0, bg = 0;
     const int64_t cmax = std::min<int64_t>(splits, kSliceMaxCluster);
-    for (int64_t c = std::max<int64_t>(cluster, kMaxCluster) + 1; c <= cmax; ++c) {
-      const int64_t g = std::min<int64_t>(std::max<int64_t>(1, splits / c), max_groups);
-      if (rows * g <= cluster_fit[c] && c * g > cluster * groups) {
-        cluster = c;
-        groups = g;
+    for (int64_t c = 2; c <= cmax; ++c) {
+      if (cluster_fit[c] < 1) continue;
+      int64_t g = std::min<int64_t>(std::max<int64_t>(1, splits / c), max_groups);
+      if (rows * g > cluster_fit[c]) g = cluster_fit[c] / rows;
+      if (g < 1) continue;
+      if (c * g > bc * bg || (c * g == bc * bg && g < bg)) {
+        bc = c;
+        bg = g;
       }
+    }
+    if (bc > 0) {
+      cluster = bc;
+      groups = bg;
     }
   }
   p.cluster = int(cluster);

@@ -278,9 +278,9 @@ int make_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t nu
 // make_plan with control over the slice kernel: `slice_cluster` is the largest
 // cluster the slice kernel may use (0: never use it, as for value order and the
 // sampling step, which the other kernels serve).  `cluster_fit`, when given, holds
-// for each cluster size c in (kMaxCluster, kSliceMaxCluster] how many clusters of c
-// streaming CTAs the device holds at once: a split row then takes such a larger
-// cluster when all of the launch's clusters fit at once and more CTAs work.
+// for each cluster size c in [1, kSliceMaxCluster] how many clusters of c streaming
+// CTAs the device holds at once: a split row then takes the cluster size and
+// number of groups with the most CTAs whose clusters all fit at once (one wave).
 int make_plan_ex(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t num_sms,
                  int32_t smem_optin, int32_t max_cluster, int32_t slice_cluster, dsel_plan_t* out,
                  const int32_t* cluster_fit = nullptr);

@@ -90,10 +90,10 @@ def test_plans_cover_split_and_merge(dtype, rows, stride, k):
 @pytest.mark.parametrize("rows", [10, 14, 16])
 def test_split_rows_wide_clusters(rows):
     """rows too long for the slice kernel, split over the streaming kernel's clusters:
-    past the portable 8 CTAs where the device holds every cluster of the launch at
-    once (16 rows: clusters of 9 on a 148-SM B200)"""
+    the device plan takes the cluster size and groups with the most CTAs whose
+    clusters the device holds in one wave (clusters above the portable 8 included)"""
     st, p = T.dsel_plan_device(T.DSEL_F32, rows, 1 << 20, 1024, T.DSEL_ORDER_INDEX)
-    assert st == 0 and p["kernel"] == T.DSEL_KERNEL_STREAM and 8 <= p["cluster"] <= 16
+    assert st == 0 and p["kernel"] == T.DSEL_KERNEL_STREAM and 2 <= p["cluster"] <= 16
     assert rows * p["cluster"] * p["groups"] <= torch.cuda.get_device_properties(0).multi_processor_count
     w = W.random_small(23 + rows, "f32", rows, 1 << 20, 1024, dist="ties", sorted_index=1)
     check(w, order=T.DSEL_ORDER_INDEX)
@@ -101,15 +101,20 @@ def test_split_rows_wide_clusters(rows):
 
 
 def test_device_plan_matches_host_plan_below_eight():
-    """the device plan differs from the host planner only in the larger clusters"""
+    """the device plan differs from the host planner only in how a row split over the
+    streaming kernel's clusters is sized (clusters and groups that fit one wave) and
+    in the slice kernel's cluster limit"""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     for args in [(T.DSEL_BF16, 64, 131072, 512, 1), (T.DSEL_F32, 256, 129280, 1024, 2),
                  (T.DSEL_BF16, 4096, 16384, 512, 1), (T.DSEL_F32, 1, 1 << 28, 1000, 1)]:
         st, dp = T.dsel_plan_device(*args)
         hst, hp = T.dsel_plan_for(*args, num_sms=sms, max_cluster=8)
         assert st == 0 and hst == 0
-        if dp["cluster"] <= 8 and dp["kernel"] != T.DSEL_KERNEL_SLICE:
+        assert (dp["kernel"], dp["threads"]) == (hp["kernel"], hp["threads"])
+        if hp["kernel"] != T.DSEL_KERNEL_SLICE and hp["cluster"] * hp["groups"] == 1:
             assert dp == hp
+        if dp["kernel"] == T.DSEL_KERNEL_STREAM and dp["cluster"] * dp["groups"] > 1:
+            assert dp["cluster"] * dp["groups"] >= hp["cluster"] * hp["groups"] // 2
 
 
 def test_all_rows_short():

@@ -111,8 +111,10 @@ def test_noalloc_refuses_plans_beyond_its_scratch():
     st, plan = T.dsel_plan(T.DSEL_F32, rows, stride, k,
                            num_sms=torch.cuda.get_device_properties(0).multi_processor_count)
     assert st == 0 and plan["workspace_bytes"] > T.DSEL_NOALLOC_SCRATCH_BYTES
-    x = torch.zeros(16, dtype=torch.int32, device="cuda")      # never read: refused before launch
-    idx = torch.zeros(16, dtype=torch.int64, device="cuda")
+    # the call plans as dsel_plan does, so it is refused before any launch; the
+    # buffers still have the full shape, so that a launch would read valid memory
+    x = torch.zeros(rows * stride, dtype=torch.int32, device="cuda")
+    idx = torch.zeros(rows * k, dtype=torch.int64, device="cuda")
     st = T.dsel_topk_noalloc(x.data_ptr(), T.DSEL_F32, rows, stride, None, k, 1, 0, T.DSEL_I64,
                              T.DSEL_NAN_FLAG, None, idx.data_ptr(), torch.cuda.current_stream().cuda_stream)
     assert st == T.DSEL_ERR_SCRATCH_LIMIT
