@@ -101,14 +101,14 @@ int make_plan_ex(int dtype, int64_t rows, int64_t row_stride, int32_t k, int32_t
   // Rows that fit, a few slices each, in the shared memory of one cluster: the
   // slice kernel.  The fewest slices that fit, or more while the batch leaves SMs
   // idle (but no slice under kSliceMinElems); the candidate list takes the rest of
-  // the shared memory and must hold at least k + 2048 entries: a slice that holds
+  // the shared memory and must hold at least k + kSliceListSlack entries: a slice that holds
   // the whole top k (a sorted row) still fits its list, with room for the keys
   // equal to the threshold; a list that overflows sends the row to the exact
   // selection on the resident slices.
   if (slice_cluster >= 1 && !resident_rows) {
     auto fits = [&](int64_t c) {
       const int64_t ch = slice_chunks(row_stride, c, eb);
-      return ch <= kSliceMaxChunks && slice_list_cap(ch, smem_optin, eb) >= int64_t(k) + 2048;
+      return ch <= kSliceMaxChunks && slice_list_cap(ch, smem_optin, eb) >= int64_t(k) + kSliceListSlack;
     };
     int64_t cmin = 0;
     for (int64_t c = 1; c <= slice_cluster; ++c) {

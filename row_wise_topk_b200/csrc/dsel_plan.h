@@ -40,6 +40,11 @@ constexpr int kSliceMinElems = 8192;          // smallest slice worth its own CT
 constexpr int kSliceMaxWaves = 4;             // batches of more slices than this many SM waves stream
 constexpr int kSliceCtlBytes = 1024;          // its control block
 constexpr int kSliceMaxList = 16384;          // candidate-list entries
+// list entries beyond k a slice plan must hold: room for keys equal to the
+// threshold when one slice holds a sorted row's whole top k (2000 rather than
+// 2048 lets 64 rows of 129,280 f32 at k = 4096 take clusters of 4, two waves of
+// slices instead of three)
+constexpr int kSliceListSlack = 2000;
 // Vectors each thread screens per round (a warp owns whole blocks): 16 for bf16
 // (a 64K-element round, the whole slice of a 131,072-position row split in two),
 // 8 for f32 (16K elements, so that two rounds fit the ring for double buffering).

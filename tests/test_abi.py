@@ -141,18 +141,18 @@ def test_plan_invariants(dtype, rows, stride, k):
         assert p["groups"] == 1 and 1 <= p["cluster"] <= 16
         assert p["round"] % 16 == 0 and p["round"] * p["cluster"] >= stride
         assert p["block"] * eb == 16384 and p["stages"] == -(-p["round"] // p["block"]) <= 8
-        assert p["capacity"] >= k + 2048 and p["capacity"] % 32 == 0          # candidate list
+        assert p["capacity"] >= k + 2000 and p["capacity"] % 32 == 0          # candidate list
         assert p["smem_bytes"] >= p["stages"] * (16384 + 2048) + p["capacity"] * (eb + 4) + 5 * 4096
         assert p["b2"] == 0 and p["workspace_bytes"] == 0
         assert (1 << p["idx_bits"]) >= stride
-        # as few slices as fit (8 chunks and a list of k + 2048), or more while the
+        # as few slices as fit (8 chunks and a list of k + 2000), or more while the
         # batch leaves SMs idle (but no slice under 8192 elements)
         def fits(c):
             sl = (-(-stride // c) + 15) // 16 * 16
             ch = -(-sl * eb // 16384)
             fixed = ch * (16384 + 2048) + -(-ch * 8 // 16) * 16 + 5632 * 4 + 1024 + 64
             lcap = min(16384, (PEAK["smem_optin"] - fixed) // (eb + 6)) // 32 * 32
-            return ch <= 8 and lcap >= k + 2048
+            return ch <= 8 and lcap >= k + 2000
         assert fits(p["cluster"])
         assert p["cluster"] == 1 or not fits(p["cluster"] - 1) or \
             (rows * p["cluster"] <= PEAK["num_sms"] and p["cluster"] <= min(8, -(-stride // 8192)))

@@ -268,11 +268,11 @@ def test_sampler_full(batch, k):
 
 @pytest.mark.parametrize("dist", ["ascending", "equal"])
 def test_slice_lists_hold_a_sorted_top_k(dist):
-    """64 sampler-sized rows at k = 4096 on the slice kernel, whose lists hold k + 2048
+    """64 sampler-sized rows at k = 4096 on the slice kernel, whose lists hold k + 2000
     entries or more: with ascending rows the last slice holds the whole top k; with
     equal keys every list overflows and the exact selection takes over"""
     st, p = T.dsel_plan_device(T.DSEL_F32, 64, 129280, 4096, T.DSEL_ORDER_INDEX)
-    assert st == 0 and p["kernel"] == T.DSEL_KERNEL_SLICE and p["capacity"] >= 4096 + 2048
+    assert st == 0 and p["kernel"] == T.DSEL_KERNEL_SLICE and p["capacity"] >= 4096 + 2000
     w = W.random_small(31, "f32", 64, 129280, 4096, dist=dist, sorted_index=1)
     check(w, order=T.DSEL_ORDER_INDEX)
     check(w, order=T.DSEL_ORDER_NONE)
