@@ -319,6 +319,17 @@ DSEL_API int dsel_plan(int dtype, int64_t rows, int64_t row_stride, int32_t k,
 DSEL_API int dsel_plan_for(int dtype, int64_t rows, int64_t row_stride, int32_t k, int sorted_index,
                            int32_t num_sms, int32_t smem_optin, int32_t max_cluster, dsel_plan_t* out);
 
+/* dsel_plan_for with a given cluster capacity: cluster_fit[c], for c = 0..16 (17
+ * entries; index 0 unused), is how many clusters of c streaming CTAs (512 threads,
+ * all opt-in shared memory) the device holds at once, as the occupancy calculator
+ * reports it; 0 where a size cannot be launched.  A row split over the streaming
+ * kernel's clusters then takes the cluster size and group count with the most CTAs
+ * whose clusters all fit at once, as dsel_plan_device does with the device's own
+ * counts.  Host only, no CUDA call.  Returns DSEL_OK, DSEL_ERR_NULL for a NULL
+ * array or out, or a DSEL_ERR_* code for invalid arguments. */
+DSEL_API int dsel_plan_fit(int dtype, int64_t rows, int64_t row_stride, int32_t k, int sorted_index,
+                           int32_t num_sms, int32_t smem_optin, const int32_t* cluster_fit, dsel_plan_t* out);
+
 /* The plan dsel_topk would use with this sorted_index on the current device (pass
  * DSEL_ORDER_VALUE for the plan of dsel_topk_sample): dsel_plan_for with the
  * device's SM count and opt-in shared memory, the slice kernel's cluster size the

@@ -85,6 +85,9 @@ def _load() -> ctypes.CDLL:
                                   ctypes.c_int32, ctypes.POINTER(DselPlan)]
     lib.dsel_plan_device.restype = c_int
     lib.dsel_plan_device.argtypes = [c_int, c_i64, c_i64, ctypes.c_int32, c_int, ctypes.c_void_p]
+    lib.dsel_plan_fit.argtypes = [c_int, c_i64, c_i64, ctypes.c_int32, c_int, ctypes.c_int32, ctypes.c_int32,
+                                  ctypes.c_void_p, ctypes.c_void_p]
+    lib.dsel_plan_fit.restype = c_int
     lib.dsel_plan.restype = c_int
     lib.dsel_plan.argtypes = [c_int, c_i64, c_i64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                               ctypes.c_int32, ctypes.POINTER(DselPlan)]
@@ -154,6 +157,17 @@ def dsel_plan_for(dtype: int, rows: int, row_stride: int, k: int, sorted_index: 
     p = DselPlan()
     st = lib.dsel_plan_for(dtype, rows, row_stride, k, sorted_index, num_sms, smem_optin, max_cluster,
                            ctypes.byref(p))
+    return st, p.as_dict()
+
+
+def dsel_plan_fit(dtype: int, rows: int, row_stride: int, k: int, sorted_index: int, cluster_fit,
+                  num_sms: int = 148, smem_optin: int = 232448) -> Tuple[int, dict]:
+    """dsel_plan_for with a given cluster capacity: cluster_fit[c] (c = 0..16) clusters
+    of c streaming CTAs fit the device at once (host only)."""
+    fit = (ctypes.c_int32 * 17)(*[int(v) for v in cluster_fit])
+    p = DselPlan()
+    st = lib.dsel_plan_fit(dtype, rows, row_stride, k, sorted_index, num_sms, smem_optin,
+                           ctypes.cast(fit, ctypes.c_void_p), ctypes.byref(p))
     return st, p.as_dict()
 
 

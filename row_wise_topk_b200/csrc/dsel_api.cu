@@ -405,6 +405,14 @@ DSEL_API int dsel_plan_for(int dtype, int64_t rows, int64_t row_stride, int32_t 
                       sorted_index == DSEL_ORDER_VALUE ? 0 : kSliceMaxCluster, out);
 }
 
+DSEL_API int dsel_plan_fit(int dtype, int64_t rows, int64_t row_stride, int32_t k, int sorted_index,
+                           int32_t num_sms, int32_t smem_optin, const int32_t* cluster_fit, dsel_plan_t* out) {
+  if (sorted_index < DSEL_ORDER_NONE || sorted_index > DSEL_ORDER_VALUE) return DSEL_ERR_ORDER;
+  if (cluster_fit == nullptr || out == nullptr) return DSEL_ERR_NULL;
+  return make_plan_ex(dtype, rows, row_stride, k, num_sms, smem_optin, kMaxCluster,
+                      sorted_index == DSEL_ORDER_VALUE ? 0 : kSliceMaxCluster, out, cluster_fit);
+}
+
 DSEL_API int dsel_plan_device(int dtype, int64_t rows, int64_t row_stride, int32_t k, int sorted_index,
                               dsel_plan_t* out) {
   if (sorted_index < DSEL_ORDER_NONE || sorted_index > DSEL_ORDER_VALUE) return DSEL_ERR_ORDER;

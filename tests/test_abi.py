@@ -257,3 +257,62 @@ def test_resident_plan_fits_four_ctas_per_sm():
     # value order with the largest k on f32 rows still fits one CTA's opt-in limit
     p = T.dsel_plan(T.DSEL_F32, 4096, 8192, 4096, **PEAK)[1]
     assert p["kernel"] == T.DSEL_KERNEL_RESIDENT and p["smem_bytes"] <= PEAK["smem_optin"]
+
+
+def _best_split(rows, stride, k, capacity, fit, sms=148):
+    """The largest number of CTAs over the (cluster, groups) splits of a row whose
+    clusters all fit at once, and the fewest groups reaching it (the rule stated for
+    dsel_plan_fit); None when no size fits."""
+    splits = max(1, min(sms // max(rows, 1), stride // 8192))
+    max_groups = min(255, max(1, 8 * capacity // k))
+    best = None
+    for c in range(2, min(splits, 16) + 1):
+        if fit[c] < 1:
+            continue
+        g = min(max(1, splits // c), max_groups)
+        if rows * g > fit[c]:
+            g = fit[c] // rows
+        if g >= 1 and (best is None or (c * g, -g) > (best[0] * best[1], -best[1])):
+            best = (c, g)
+    return best
+
+
+@pytest.mark.parametrize("fit", [
+    [0] + [148 // c for c in range(1, 17)],                                   # every SM usable by any cluster
+    [0, 148, 74, 49, 36, 29, 24, 21, 12, 9, 8, 8, 8, 8, 8, 8, 8],             # large clusters scarce (GPC bound)
+    [0, 148, 70, 45, 32, 24, 20, 16, 14, 0, 0, 0, 0, 0, 0, 0, 0],             # no cluster above the portable 8
+])
+@pytest.mark.parametrize("rows,stride,k", [(16, 1 << 24, 4096), (16, 1 << 24, 1000), (1, 1 << 28, 1000),
+                                           (1, 1 << 28, 4096), (10, 1 << 20, 1024), (3, 1 << 21, 2000),
+                                           (2, 1 << 20, 64)])
+def test_fitted_split_keeps_every_cluster_in_one_wave(fit, rows, stride, k):
+    st, p = T.dsel_plan_fit(T.DSEL_F32, rows, stride, k, T.DSEL_ORDER_INDEX, fit)
+    assert st == 0 and p["kernel"] == T.DSEL_KERNEL_STREAM
+    c, g = p["cluster"], p["groups"]
+    assert rows * g <= fit[c]                                   # every cluster of the launch at once
+    assert (c, g) == _best_split(rows, stride, k, p["capacity"], fit)
+    assert p["workspace_bytes"] == (rows * g * (k * 8 + 8) if g > 1 else 0)
+
+
+def test_fitted_split_when_sixteen_clusters_of_eight_do_not_fit():
+    # a capacity in which sixteen clusters of 8 (or 9) do not fit at once, nor 48 of
+    # 3: two groups of clusters of 4 (128 CTAs) beat one of 7 (112)
+    fit = [0, 148, 74, 40, 36, 28, 24, 21, 12, 9, 8, 8, 8, 8, 8, 8, 8]
+    p = T.dsel_plan_fit(T.DSEL_F32, 16, 1 << 24, 4096, T.DSEL_ORDER_INDEX, fit)[1]
+    assert (p["cluster"], p["groups"]) == (4, 2)
+    # the host planner, with no capacity to go by, keeps the portable split
+    h = T.dsel_plan_for(T.DSEL_F32, 16, 1 << 24, 4096, T.DSEL_ORDER_INDEX, **PEAK)[1]
+    assert (h["cluster"], h["groups"]) == (8, 1)
+
+
+def test_fitted_plan_is_the_host_plan_without_a_split():
+    fit = [0] + [148 // c for c in range(1, 17)]
+    for args in [(T.DSEL_BF16, 64, 131072, 512, 0), (T.DSEL_F32, 256, 129280, 1024, 1),
+                 (T.DSEL_BF16, 4096, 16384, 512, 1), (T.DSEL_F32, 8, 129280, 50, 1),
+                 (T.DSEL_F32, 256, 129280, 1024, T.DSEL_ORDER_VALUE)]:
+        assert T.dsel_plan_fit(*args, fit) == T.dsel_plan_for(*args, **PEAK)
+    # no cluster size fits at all: the portable split
+    none = [0, 148] + [0] * 15
+    assert T.dsel_plan_fit(T.DSEL_F32, 16, 1 << 24, 4096, 1, none) == \
+        T.dsel_plan_for(T.DSEL_F32, 16, 1 << 24, 4096, 1, **PEAK)
+    assert T.dsel_plan_fit(T.DSEL_F32, 16, 1 << 24, 4096, 3, none)[0] == header_define("DSEL_ERR_ORDER")
