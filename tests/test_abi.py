@@ -131,6 +131,12 @@ PEAK = dict(num_sms=148, smem_optin=232448, max_cluster=8)
 def test_plan_invariants(dtype, rows, stride, k):
     st, p = T.dsel_plan(dtype, rows, stride, k, **PEAK)
     assert st == 0
+    check_plan(dtype, rows, stride, k, p)
+
+
+def check_plan(dtype, rows, stride, k, p, fit=None):
+    """What a plan must hold for its kernel's buffers and launch (fit: the cluster
+    capacity a fitted plan was made for, else None for the host plan)."""
     eb = 2 if dtype == T.DSEL_BF16 else 4
     assert p["smem_bytes"] <= PEAK["smem_optin"]
     assert p["kernel"] in (T.DSEL_KERNEL_STREAM, T.DSEL_KERNEL_RESIDENT, T.DSEL_KERNEL_SLICE)
@@ -187,8 +193,10 @@ def test_plan_invariants(dtype, rows, stride, k):
         assert (p["cluster"], p["groups"]) == (1, 1)
         assert 2 * (p["smem_bytes"] + 1024) <= PEAK["smem_optin"] + 1024
     assert p["round"] % p["block"] == 0 and (p["block"] * eb) % 16 == 0
-    assert 1 <= p["cluster"] <= PEAK["max_cluster"]
+    assert 1 <= p["cluster"] <= (PEAK["max_cluster"] if fit is None else 16)
     assert p["groups"] >= 1 and p["groups"] * k <= 8 * p["capacity"]
+    if fit is not None and p["cluster"] > PEAK["max_cluster"]:
+        assert rows * p["groups"] <= fit[p["cluster"]]          # non-portable sizes only where they fit
     assert (1 << p["idx_bits"]) >= stride
     assert p["idx_bits"] + 8 * eb <= 63
     if p["groups"] > 1:
@@ -316,3 +324,51 @@ def test_fitted_plan_is_the_host_plan_without_a_split():
     assert T.dsel_plan_fit(T.DSEL_F32, 16, 1 << 24, 4096, 1, none) == \
         T.dsel_plan_for(T.DSEL_F32, 16, 1 << 24, 4096, 1, **PEAK)
     assert T.dsel_plan_fit(T.DSEL_F32, 16, 1 << 24, 4096, 3, none)[0] == header_define("DSEL_ERR_ORDER")
+
+
+FITS = [
+    [0] + [148 // c for c in range(1, 17)],
+    [0, 148, 74, 49, 36, 29, 24, 21, 12, 9, 8, 8, 8, 8, 8, 8, 8],
+    [0, 148, 70, 45, 32, 24, 20, 16, 14, 0, 0, 0, 0, 0, 0, 0, 0],
+]
+
+
+def _random_shapes(seed, n):
+    """Seeded shapes spread log-uniformly: 1..8192 rows, row strides of 16..2^28
+    elements (multiples of 16), k = 1..4096, both dtypes."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    for _ in range(n):
+        dtype = T.DSEL_BF16 if rng.random() < 0.5 else T.DSEL_F32
+        rows = int(np.exp(rng.uniform(0, np.log(8192))))
+        stride = 16 * max(1, int(np.exp(rng.uniform(0, np.log(1 << 24)))))
+        k = max(1, min(4096, int(np.exp(rng.uniform(0, np.log(4097))))))
+        yield dtype, rows, stride, k
+
+
+@pytest.mark.parametrize("seed", [11, 12, 13])
+def test_random_shapes_plan_within_their_buffers(seed):
+    # every valid shape gets a plan, in every order, on the host and on each fitted
+    # capacity, and each plan holds what its kernel's buffers and launch need
+    orders = [T.DSEL_ORDER_NONE, T.DSEL_ORDER_INDEX, T.DSEL_ORDER_VALUE]
+    for dtype, rows, stride, k in _random_shapes(seed, 200):
+        for order in orders:
+            if order == T.DSEL_ORDER_VALUE and dtype == T.DSEL_BF16:
+                continue
+            st, h = T.dsel_plan_for(dtype, rows, stride, k, order, **PEAK)
+            assert st == 0, (dtype, rows, stride, k, order)
+            check_plan(dtype, rows, stride, k, h)
+            if order == T.DSEL_ORDER_VALUE:
+                assert h["kernel"] != T.DSEL_KERNEL_SLICE
+            for fit in FITS:
+                st, f = T.dsel_plan_fit(dtype, rows, stride, k, order, fit)
+                assert st == 0, (dtype, rows, stride, k, order, fit)
+                check_plan(dtype, rows, stride, k, f, fit=fit)
+                # the capacity only moves a long row's split over clusters and groups
+                assert (f["kernel"], f["threads"], f["round"], f["block"], f["b2"]) == \
+                    (h["kernel"], h["threads"], h["round"], h["block"], h["b2"])
+                if (f["cluster"], f["groups"]) != (h["cluster"], h["groups"]):
+                    assert f["kernel"] == T.DSEL_KERNEL_STREAM and rows < PEAK["num_sms"]
+                    assert rows * f["groups"] <= fit[f["cluster"]]
+                    assert (f["cluster"], f["groups"]) == \
+                        _best_split(rows, stride, k, f["capacity"], fit)
