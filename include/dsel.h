@@ -51,9 +51,10 @@
  * dsel_topk_noalloc never allocates.
  *
  * Special rows and sentinel values
- *   - end[r] <= k ("short row"): all end[r] entries are returned in index order
- *     and the NaN check is skipped (narracomm NaN paragraph); slots end[r]..k-1
- *     hold index DSEL_IDX_PAD and value -inf.
+ *   - end[r] <= k ("short row"): all end[r] entries are returned, in index order
+ *     (DSEL_ORDER_VALUE: value descending, equal values by index), and the NaN
+ *     check is skipped (narracomm NaN paragraph); slots end[r]..k-1 hold index
+ *     DSEL_IDX_PAD and value -inf.
  *   - a NaN in a row with end[r] > k: DSEL_NAN_TRAP (default, the pages'
  *     abort_when_nan_found=True) executes the PTX `trap` instruction, which
  *     aborts the CUDA context; DSEL_NAN_FLAG instead writes DSEL_IDX_NAN in every
