@@ -130,3 +130,129 @@ def test_infinite_logits():
     res = S.oracle_sample(f32_bits(x), 3, 1.0, 1.0, np.array([0.75, 0.7]))
     assert res.token[0] == 11 and res.prob[0] == pytest.approx(0.5)
     assert res.token[1] == 2 and res.prob[1] == pytest.approx(1 / 3)   # candidates 0, 1, 2
+
+
+def test_top_p_reached_exactly_keeps_the_shortest_prefix():
+    # an all-equal row of k = 50 candidates: weights all 1, E_c = c, E_m = 50; top_p = 0.5
+    # is reached exactly at c = 25 (0.5 * 50 = 25, exact in binary), and top_p = 0.02 at c = 1
+    x = np.full((1, 400), -1.5, dtype=np.float32)
+    for top_p, c in ((0.5, 25), (0.02, 1), (0.5 + 1e-9, 26)):
+        res = S.oracle_sample(f32_bits(x), 50, 1.0, top_p, np.array([0.999]))
+        assert res.kept[0] == c
+        assert res.token[0] == c - 1 and res.prob[0] == pytest.approx(1.0 / c)
+
+
+# Mutants of the draw: each changes one step of the reading in a way a careless
+# restatement could, and at least one pin above must fail on it.
+
+def _mutant_temperature_multiplies(z, temperature, top_p, u):
+    return _with_weights(z, top_p, u, lambda: np.where(z == z[0], 1.0, np.exp((z - z[0]) * temperature))
+                         if temperature > 0 else _greedy(len(z)))
+
+
+def _mutant_top_p_one_short(z, temperature, top_p, u):
+    pos, p, c, pre = _REAL_SAMPLE_ROW(z, temperature, top_p, u)
+    if c <= 1 or top_p >= 1.0:
+        return pos, p, c, pre
+    c -= 1
+    target = u * pre[c - 1]
+    pos = min(int(np.searchsorted(pre[:c], target, side="right")), c - 1)
+    e = np.diff(np.concatenate([[0.0], pre]))
+    return pos, float(e[pos] / pre[c - 1]), c, pre
+
+
+def _mutant_top_p_strict(z, temperature, top_p, u):
+    e = _weights(z, temperature)
+    pre = np.cumsum(e)
+    c = m = len(z)
+    if top_p < 1.0:
+        c = min(max(int(np.searchsorted(pre, top_p * pre[-1], side="right")) + 1, 1), m)
+    pos = min(int(np.searchsorted(pre[:c], u * pre[c - 1], side="right")), c - 1)
+    return pos, float(e[pos] / pre[c - 1]), c, pre
+
+
+def _mutant_draw_at_or_above(z, temperature, top_p, u):
+    pos, p, c, pre = _REAL_SAMPLE_ROW(z, temperature, top_p, u)
+    e = np.diff(np.concatenate([[0.0], pre]))
+    pos = min(int(np.searchsorted(pre[:c], u * pre[c - 1], side="left")), c - 1)
+    return pos, float(e[pos] / pre[c - 1]), c, pre
+
+
+def _mutant_probability_not_renormalised(z, temperature, top_p, u):
+    pos, p, c, pre = _REAL_SAMPLE_ROW(z, temperature, top_p, u)
+    return pos, p * pre[c - 1] / pre[-1], c, pre
+
+
+def _mutant_leaders_not_forced_to_one(z, temperature, top_p, u):
+    return _with_weights(z, top_p, u, lambda: np.exp((z - z[0]) / temperature) if temperature > 0
+                         else _greedy(len(z)))
+
+
+def _greedy(m):
+    e = np.zeros(m)
+    e[0] = 1.0
+    return e
+
+
+def _weights(z, temperature):
+    if temperature <= 0.0:
+        return _greedy(len(z))
+    with np.errstate(invalid="ignore", over="ignore"):
+        return np.where(z == z[0], 1.0, np.exp((z - z[0]) / temperature))
+
+
+def _with_weights(z, top_p, u, make):
+    with np.errstate(invalid="ignore", over="ignore"):
+        e = make()
+    pre = np.cumsum(e)
+    c = m = len(z)
+    if top_p < 1.0:
+        c = min(max(int(np.searchsorted(pre, top_p * pre[-1], side="left")) + 1, 1), m)
+    pos = min(int(np.searchsorted(pre[:c], u * pre[c - 1], side="right")), c - 1)
+    return pos, float(e[pos] / pre[c - 1]), c, pre
+
+
+_REAL_SAMPLE_ROW = S.sample_row
+_PINS = [test_greedy_and_tiny_top_p_pick_the_argmax, test_all_equal_row_is_a_uniform_draw_over_the_lowest_indices,
+         test_two_candidates_closed_form, test_top_p_cut_worked_example, test_ties_are_ordered_by_index_and_high_temperature_flattens,
+         test_row_rules, test_token_is_always_in_the_top_k, test_infinite_logits,
+         test_top_p_reached_exactly_keeps_the_shortest_prefix]
+
+
+def _pins_fail():
+    for pin in _PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin()
+        except (AssertionError, ValueError, IndexError):
+            return True
+    return False
+
+
+def test_the_mutants_stand_apart_from_the_oracle():
+    # each mutant really differs from the oracle somewhere, so catching it means something
+    z = np.array([np.inf, 2.0, 2.0, 1.0, 0.5, -1.0, -1.0, -4.0])
+    zf = np.array([3.0, 2.0, 2.0, 1.0, 0.5, -1.0, -1.0, -4.0])
+    for mutant in _MUTANTS:
+        differs = False
+        for zz in (z, zf, np.zeros(50)):
+            for t in (0.5, 1.0, 2.0):
+                for tp in (0.3, 0.5, 0.9, 1.0):
+                    for u in (0.0, 0.25, 0.5, 0.77, 0.999):
+                        with np.errstate(all="ignore"):
+                            a = _REAL_SAMPLE_ROW(zz, t, tp, u)
+                            b = mutant(zz, t, tp, u)
+                        if a[0] != b[0] or a[2] != b[2] or not (a[1] == b[1] or (np.isnan(a[1]) and np.isnan(b[1]))):
+                            differs = True
+        assert differs, mutant.__name__
+
+
+_MUTANTS = [_mutant_temperature_multiplies, _mutant_top_p_one_short, _mutant_top_p_strict,
+            _mutant_draw_at_or_above, _mutant_probability_not_renormalised, _mutant_leaders_not_forced_to_one]
+
+
+@pytest.mark.parametrize("mutant", _MUTANTS, ids=lambda f: f.__name__[len("_mutant_"):])
+def test_sample_mutants_are_caught(monkeypatch, mutant):
+    assert not _pins_fail()                     # the pins pass on the oracle itself
+    monkeypatch.setattr(S, "sample_row", mutant)
+    assert _pins_fail()
