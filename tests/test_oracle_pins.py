@@ -273,6 +273,44 @@ def test_mutant_short_rule_is_caught(monkeypatch):
     assert hand_case_failures(strict_short)
 
 
+def _rows_ignore_end(real):
+    return lambda x_bits, dtype, k, **kw: real(x_bits, dtype, k, **{**kw, "end": None})
+
+
+def _bad_end_clamped_in_flag_mode(real):
+    def f(x_bits, dtype, k, **kw):
+        end = kw.get("end")
+        if end is not None:
+            kw = {**kw, "end": np.clip(np.asarray(end), 0, x_bits.shape[1])}
+        return real(x_bits, dtype, k, **kw)
+    return f
+
+
+def _padding_zero(real):
+    def f(x_bits, dtype, k, **kw):
+        res = real(x_bits, dtype, k, **kw)
+        res.indices[res.indices == O.IDX_PAD] = 0
+        return res
+    return f
+
+
+def _end_one_past(real):
+    # reads one entry past the valid range (end + 1, where that stays inside the row)
+    def f(x_bits, dtype, k, **kw):
+        end = kw.get("end")
+        if end is not None:
+            end = np.asarray(end)
+            kw = {**kw, "end": np.where((end >= 0) & (end < x_bits.shape[1]), end + 1, end)}
+        return real(x_bits, dtype, k, **kw)
+    return f
+
+
+@pytest.mark.parametrize("mutant", [_rows_ignore_end, _bad_end_clamped_in_flag_mode, _padding_zero, _end_one_past])
+def test_mutant_row_rule_is_caught(mutant):
+    assert not hand_case_failures(O.oracle_topk)
+    assert hand_case_failures(mutant(O.oracle_topk))
+
+
 def nan_flag_failures(oracle_fn):
     w = W.long_rows(6, 2048, 10, "uniform", inject_nan=True)
     res = oracle_fn(w.x, w.dtype, w.k, nan_mode="flag")
