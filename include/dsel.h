@@ -289,7 +289,10 @@ DSEL_API int dsel_shard_stack(const void* vals_in, const int64_t* idx_in, int dt
  * (a sentinel code) otherwise: maps the positions returned by dsel_topk on a
  * dsel_shard_stack row back to indices in the whole row.
  *   table        device int64 [rows][table_stride]
- *   pos          device [rows][k], int32 or int64 (pos_dtype: DSEL_I32 / DSEL_I64)
+ *   pos          device [rows][k], int32 or int64 (pos_dtype: DSEL_I32 / DSEL_I64):
+ *                each entry a negative code or a position < table_stride (what
+ *                dsel_topk returns on rows of table_stride elements); the kernel
+ *                reads table[r][pos] without a further check
  *   indices_out  device [rows][k], int32 or int64 (index_dtype)
  * Returns DSEL_OK, DSEL_ERR_K / _ROWS / _INDEX_DTYPE / _NULL, or DSEL_ERR_CUDA.
  */

@@ -79,6 +79,79 @@ def test_host_argument_checks(kw, err):
     assert call(**kw) == header_define(err)
 
 
+@pytest.mark.parametrize("kw,err", [
+    (dict(dtype=2), "DSEL_ERR_DTYPE"),
+    (dict(k=4097), "DSEL_ERR_K"),
+    (dict(rows=-1), "DSEL_ERR_ROWS"),
+    (dict(row_stride=8200), "DSEL_ERR_STRIDE"),
+    (dict(index_dtype=2), "DSEL_ERR_INDEX_DTYPE"),
+    (dict(nan_mode=-1), "DSEL_ERR_NAN_MODE"),
+    (dict(sorted_index=2, dtype=T.DSEL_BF16), "DSEL_ERR_ORDER"),
+    (dict(x=None), "DSEL_ERR_NULL"),
+    (dict(values_out=None), "DSEL_ERR_VALUES"),
+    (dict(x=0x1002), "DSEL_ERR_ALIGN"),
+])
+def test_noalloc_host_argument_checks(kw, err):
+    assert call_noalloc(**kw) == header_define(err)
+
+
+def call_noalloc(**kw):
+    a = dict(x=0x1000, dtype=T.DSEL_F32, rows=4, row_stride=8192, end=None, k=64, sorted_index=1,
+             return_value=1, index_dtype=T.DSEL_I64, nan_mode=T.DSEL_NAN_TRAP, values_out=0x2000,
+             indices_out=0x3000, stream=None)
+    a.update(kw)
+    return T.dsel_topk_noalloc(**a)
+
+
+def test_noalloc_zero_rows_is_a_noop():
+    assert call_noalloc(rows=0, x=None, indices_out=None, values_out=None, return_value=0) == 0
+
+
+def _stack(**kw):
+    a = dict(vals_in=0x1000, idx_in=0x2000, dtype=T.DSEL_F32, rows=3, k=64, shards=2, shard_len=4096,
+             out_stride=128, vals_out=0x3000, idx_out=0x4000, stream=None)
+    a.update(kw)
+    return T.lib.dsel_shard_stack(*a.values())
+
+
+def _take(**kw):
+    a = dict(table=0x1000, table_stride=128, pos=0x2000, pos_dtype=T.DSEL_I64, rows=3, k=64,
+             index_dtype=T.DSEL_I32, indices_out=0x3000, stream=None)
+    a.update(kw)
+    return T.lib.dsel_take_index(*a.values())
+
+
+@pytest.mark.parametrize("kw,err", [
+    (dict(dtype=5), "DSEL_ERR_DTYPE"),
+    (dict(k=0), "DSEL_ERR_K"),
+    (dict(shards=0), "DSEL_ERR_K"),
+    (dict(shard_len=63), "DSEL_ERR_K"),                 # every shard must give k real candidates
+    (dict(rows=-2), "DSEL_ERR_ROWS"),
+    (dict(out_stride=112), "DSEL_ERR_STRIDE"),          # < shards * k
+    (dict(out_stride=136), "DSEL_ERR_STRIDE"),          # not a multiple of 16
+    (dict(idx_out=None), "DSEL_ERR_NULL"),
+])
+def test_shard_stack_host_argument_checks(kw, err):
+    assert _stack(**kw) == header_define(err)
+
+
+@pytest.mark.parametrize("kw,err", [
+    (dict(k=4097), "DSEL_ERR_K"),
+    (dict(table_stride=0), "DSEL_ERR_K"),
+    (dict(rows=-1), "DSEL_ERR_ROWS"),
+    (dict(pos_dtype=2), "DSEL_ERR_INDEX_DTYPE"),
+    (dict(index_dtype=7), "DSEL_ERR_INDEX_DTYPE"),
+    (dict(pos=None), "DSEL_ERR_NULL"),
+])
+def test_take_index_host_argument_checks(kw, err):
+    assert _take(**kw) == header_define(err)
+
+
+def test_shard_steps_with_zero_rows_are_noops():
+    assert _stack(rows=0, vals_in=None, idx_in=None, vals_out=None, idx_out=None) == 0
+    assert _take(rows=0, table=None, pos=None, indices_out=None) == 0
+
+
 def call_sample(**kw):
     a = dict(x=0x1000, rows=4, row_stride=8192, end=None, k=64, temperature=1.0, top_p=0.9, u=0x4000,
              nan_mode=T.DSEL_NAN_FLAG, values_out=0x2000, indices_out=0x3000, token_out=0x5000, prob_out=None,
