@@ -10,7 +10,10 @@ ranks is reported.  Under torchrun every rank processes its own batch (weak
 scaling, no collective on the data path).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                       [--impl ours|reference]
+                       [--impl ours|reference] [--torch-topk]
+
+``--torch-topk`` adds ``context_torch_topk`` to the line: torch.topk timed on the same
+inputs, as context for the pages' comparison with it (never part of ``value``).
 """
 from __future__ import annotations
 
@@ -554,6 +557,8 @@ def run_ours(args, w, world, rank, local, pg):
         d2h = idx_out.numel() * idx_out.element_size() + (0 if val_out is None else val_out.numel() * val_out.element_size())
     e2e_value = world * eff / (e2e_ms / 1e3) / 1e9
 
+    torch_ctx = torch_topk_context(args, w, copies, stream, eff, ms_per_step, sampling) if args.torch_topk else None
+
     if rank != 0:
         return
     cpu = None
@@ -591,7 +596,46 @@ def run_ours(args, w, world, rank, local, pg):
         "plan": {k_: plan[k_] for k_ in ("kernel", "threads", "cluster", "groups", "stages", "smem_bytes")},
         "input_copies": n_copies,
     }
+    if torch_ctx is not None:
+        line["context_torch_topk"] = torch_ctx
     print(json.dumps(line), flush=True)
+
+
+def torch_topk_context(args, w, copies, stream, eff, ms_per_step, sampling):
+    """Context only (the pages compare their kernel with torch.topk): torch.topk with
+    sorted=False on the same input copies, eager launches on the same stream, timed
+    with CUDA events over at least 20 calls and about half a second.  Whole rows
+    only: torch.topk has no per-row valid length."""
+    import torch
+    if sampling or w.end is not None:
+        return {"skipped": "per-row end or sampling: torch.topk has no counterpart"}
+    try:
+        dtype = torch.bfloat16 if w.elem_bytes == 2 else torch.float32
+        views = [c.view(dtype) for c in copies]
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                torch.topk(views[i % len(views)], w.k, dim=-1, largest=True, sorted=False)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record()
+            torch.topk(views[0], w.k, dim=-1, largest=True, sorted=False)
+            b.record()
+        torch.cuda.synchronize()
+        reps = int(max(20, min(2000, 500.0 / max(a.elapsed_time(b), 1e-3))))
+        with torch.cuda.stream(stream):
+            a.record()
+            for i in range(reps):
+                torch.topk(views[i % len(views)], w.k, dim=-1, largest=True, sorted=False)
+            b.record()
+        torch.cuda.synchronize()
+        t_ms = a.elapsed_time(b) / reps
+    except Exception as e:   # context only: never costs the line
+        return {"skipped": f"torch.topk failed: {type(e).__name__}"}
+    return {"call": f"torch.topk(x, {w.k}, dim=-1, sorted=False)", "calls": reps, "ms_per_call": round(t_ms, 5),
+            "value": round(eff / (t_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+            "ratio_of_ours": round(t_ms / ms_per_step, 2), "torch": torch.__version__,
+            "note": "eager launches; same effective bytes as the line's value"}
 
 
 def kernel_name(T, plan, launches_per_step):
@@ -739,6 +783,8 @@ def main():
     ap.add_argument("--min-seconds", type=float, default=1.0,
                     help="the timed region runs at least this long (more steps than --steps if needed)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--torch-topk", action="store_true",
+                    help="also time torch.topk on the same inputs (context only, not part of the line's value)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
