@@ -194,3 +194,17 @@ def test_recorded_traffic_follows_the_kernel_sources(monkeypatch):
     monkeypatch.setattr(bench, "kernel_hash", lambda: "0000000000000000")
     assert all(bench.recorded_traffic(name) is None for name in rec)
     assert bench.recorded_traffic("no_such_workload") is None
+
+
+def test_torch_topk_context_skips_what_it_has_no_counterpart_for():
+    # per-row end and the sampling step have no torch.topk counterpart: skipped without
+    # touching a device
+    import numpy as np
+
+    class Wk:
+        end = np.zeros(2, dtype=np.int32)
+        elem_bytes = 2
+        k = 4
+    assert "skipped" in bench.torch_topk_context(None, Wk(), [], None, 1, 1.0, sampling=False)
+    Wk.end = None
+    assert "skipped" in bench.torch_topk_context(None, Wk(), [], None, 1, 1.0, sampling=True)
