@@ -50,6 +50,10 @@ def make_workload(name: str) -> W.Workload:
         return W.indexer_drift()
     if name == "indexer_varlen":
         return W.indexer_varlen()
+    if name == "indexer_varlen_values":     # the same batch with the values returned too
+        w = W.indexer_varlen(return_value=1)
+        w.name += "_values"
+        return w
     if name.startswith("sampler"):        # sampler_B_k, e.g. sampler_256_4096
         _, b, k = name.split("_")
         return W.sampler_logits(int(b), int(k))
