@@ -333,7 +333,8 @@ def run_reference(args, w, world, rank):
     the workload per step (rank 0 only)."""
     if rank != 0:
         return
-    per_step_budget = max(0.5, 60.0 / max(args.steps + args.warmup, 1))
+    # about a minute for the whole run, and no more than --cpu-seconds per step
+    per_step_budget = max(0.2, min(args.cpu_seconds, 60.0 / max(args.steps + args.warmup, 1)))
     pool = OraclePool(w, args.workload.startswith("sample_"))
     try:
         for i in range(args.warmup):
