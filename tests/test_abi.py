@@ -445,3 +445,15 @@ def test_random_shapes_plan_within_their_buffers(seed):
                     assert rows * f["groups"] <= fit[f["cluster"]]
                     assert (f["cluster"], f["groups"]) == \
                         _best_split(rows, stride, k, f["capacity"], fit)
+
+
+def test_binding_fails_loudly_without_the_library():
+    # no CPU fallback: importing the binding with its library absent raises
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, ROW_WISE_TOPK_LIB="libdsel_not_built.so")
+    res = subprocess.run([sys.executable, "-c", "import row_wise_topk_b200"], cwd=root, env=env,
+                         capture_output=True, text=True, timeout=120)
+    assert res.returncode != 0
+    assert "ImportError" in res.stderr and "no fallback" in res.stderr
